@@ -1,0 +1,10 @@
+"""CPU oracle of the RoM projection block (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
+reference arm may import this package. The product path never does.
+"""
+from .rom_oracle import (block_backward, block_forward, dispatch, inproj_forward, route,
+                         sigmoid, silu, silu_grad, softmax)
+
+__all__ = ["block_backward", "block_forward", "dispatch", "inproj_forward", "route", "sigmoid",
+           "silu", "silu_grad", "softmax"]

@@ -1,0 +1,275 @@
+"""CPU oracle of the Routing Mamba (RoM) mixture-of-experts projection block.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this module:
+only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+arm of ``bench.py`` call it. It shares no code with the CUDA library.
+
+Plain, slow, float64 numpy. Every function follows a passage of the pages:
+
+* "Routing Mamba: Scaling State Space Models with Mixture-of-Experts
+  Projection" (chapterpal summary page), Knowl 1 -- the router
+  p_t = Softmax(x_t W_r), the top-K set S_t, the routing weights
+  r_{t,i} = p_{t,i} 1[i in S_t], the shared-selection input and gate
+  projections H_t and G_t = SiLU(sum ...), and the block output
+  O_t = sum_i r_{t,i} (Y_t (.) G_t) W_out,i.
+* Same page, Knowl 12 -- dropless dispatch: no expert parallelism, no
+  capacity factor, no token dropping (every selected (token, expert) pair is
+  computed).
+* "Swimba: Switch Mamba Model Scales State Space Models" (project page),
+  Extended abstract, second paragraph -- expert in-projections emit the X, B
+  and C streams, and the routing-weighted streams are summed.
+
+Readings taken where the pages are silent (each is listed in the design doc):
+
+* The short convolution and selective scan between the projections are not
+  changed by the method; the oracle stands the identity in for them (Y = H).
+* S_t is chosen on the logits (softmax is strictly increasing, so the K
+  largest logits are the K largest probabilities); equal logits go to the
+  lower expert index, and the slots of S_t are ordered by descending logit.
+* ``renorm=True`` divides the selected probabilities by their sum (the top-2
+  workload); otherwise r = p as the formula states.
+* An optional additive router bias is added to the logits before softmax.
+* The expert permutation is expert-major and, inside an expert, ascending
+  in token (slot) index.
+* The backward treats S_t as fixed (piecewise-constant selection) and returns
+  the exact gradient of the forward above.
+
+Weights are taken in the pages' notation: W_in,i and W_g,i are [D_m, D_e]
+(used as x W), W_out,i is [D_e, D_m]. Arrays are stacked on a leading expert
+axis.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(a):
+    return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+def sigmoid(z):
+    """Logistic function 1 / (1 + exp(-z)), written to avoid overflow."""
+    z = np.asarray(z, dtype=np.float64)
+    out = np.empty_like(z)
+    pos = z >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-z[pos]))
+    ez = np.exp(z[~pos])
+    out[~pos] = ez / (1.0 + ez)
+    return out
+
+
+def silu(z):
+    """SiLU(z) = z * sigmoid(z) (Elfwing et al., cited by the RoM page for SiLU)."""
+    return np.asarray(z, dtype=np.float64) * sigmoid(z)
+
+
+def silu_grad(z):
+    """d/dz SiLU(z) = sigmoid(z) * (1 + z * (1 - sigmoid(z)))."""
+    s = sigmoid(z)
+    return s * (1.0 + np.asarray(z, np.float64) * (1.0 - s))
+
+
+def softmax(logits):
+    """Row-wise softmax exp(l - max) / sum exp(l - max)."""
+    l = _f64(logits)
+    m = l.max(axis=-1, keepdims=True)
+    e = np.exp(l - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def route(x, w_r, k, bias=None, renorm=False):
+    """RoM router (RoM page, Knowl 1): logits, probabilities, S_t and r_{t,i}.
+
+    Returns a dict with
+      logits [T,E], p [T,E],
+      topk_idx [T,k] int32: S_t, slot j holds the j-th largest logit
+        (equal logits: lower expert index first),
+      topk_w [T,k] float64: r_{t,S_t[j]} (= p, or p / sum_S p if renorm),
+      margin [T]: the smallest logit gap that decides S_t and its slot order
+        (used to flag tokens whose choice is numerically ambiguous).
+    """
+    x = _f64(x)
+    logits = x @ _f64(w_r)
+    if bias is not None:
+        logits = logits + _f64(bias)[None, :]
+    T, E = logits.shape
+    if not 1 <= k <= E:
+        raise ValueError("k must be in [1, E]")
+    p = softmax(logits)
+    # Order experts per token by (descending logit, ascending index).
+    order = np.empty((T, E), dtype=np.int64)
+    for t in range(T):
+        order[t] = sorted(range(E), key=lambda i: (-logits[t, i], i))
+    topk_idx = order[:, :k].astype(np.int32)
+    rows = np.arange(T)[:, None]
+    r = p[rows, topk_idx]
+    if renorm:
+        r = r / r.sum(axis=1, keepdims=True)
+    # Decision margin: gaps between consecutive sorted logits up to slot k.
+    srt = logits[rows, order]
+    ngaps = k if k < E else k - 1
+    if ngaps > 0:
+        gaps = srt[:, :ngaps] - srt[:, 1:ngaps + 1]
+        margin = gaps.min(axis=1)
+    else:
+        margin = np.full(T, np.inf)
+    return dict(logits=logits, p=p, topk_idx=topk_idx, topk_w=r, margin=margin)
+
+
+def dispatch(topk_idx, E):
+    """Dropless dispatch order (RoM page, Knowl 12; order reading in the header).
+
+    Slots are numbered s = t*k + j. Returns
+      counts [E]: number of slots routed to each expert,
+      offsets [E+1]: exclusive prefix sum of counts,
+      sorted_slot [R]: sorted position -> slot (expert-major, ascending slot),
+      slot_pos [R]: slot -> sorted position.
+    Written as a counting sort with explicit loops.
+    """
+    idx = np.asarray(topk_idx).reshape(-1)
+    R = idx.shape[0]
+    counts = np.zeros(E, dtype=np.int64)
+    for s in range(R):
+        counts[int(idx[s])] += 1
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    for e in range(E):
+        offsets[e + 1] = offsets[e] + counts[e]
+    cursor = offsets[:E].copy()
+    sorted_slot = np.empty(R, dtype=np.int64)
+    slot_pos = np.empty(R, dtype=np.int64)
+    for s in range(R):
+        e = int(idx[s])
+        sorted_slot[cursor[e]] = s
+        slot_pos[s] = cursor[e]
+        cursor[e] += 1
+    return dict(counts=counts.astype(np.int32), offsets=offsets.astype(np.int32),
+                sorted_slot=sorted_slot.astype(np.int32), slot_pos=slot_pos.astype(np.int32))
+
+
+def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=None):
+    """RoM projection block forward (RoM page, Knowl 1).
+
+    H_t = sum_i 1[i in S_t] x_t W_in,i ;  G_t = SiLU(sum_i 1[i in S_t] x_t W_g,i)
+    Y_t = H_t (identity stand-in for the unchanged conv + SSM core)
+    O_t = sum_i r_{t,i} (Y_t (.) G_t) W_out,i
+
+    ``tokens`` (optional index array) evaluates only those tokens; every
+    token is independent of the others in this block.
+    Returns a dict with O [T,Dm], H, Gpre (the sum before SiLU), G, YG [T,De]
+    and the router outputs.
+    """
+    x = _f64(x)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+    rt = route(x, w_r, k, bias=bias, renorm=renorm)
+    S, r = rt["topk_idx"], rt["topk_w"]
+    T = x.shape[0]
+    E, Dm, De = np.shape(w_in)
+    H = np.zeros((T, De))
+    Gpre = np.zeros((T, De))
+    for i in range(E):
+        for j in range(k):
+            sel = np.nonzero(S[:, j] == i)[0]
+            if sel.size == 0:
+                continue
+            H[sel] += x[sel] @ _f64(w_in[i])
+            Gpre[sel] += x[sel] @ _f64(w_g[i])
+    G = silu(Gpre)
+    Y = H
+    YG = Y * G
+    O = np.zeros((T, Dm))
+    for i in range(E):
+        for j in range(k):
+            sel = np.nonzero(S[:, j] == i)[0]
+            if sel.size == 0:
+                continue
+            O[sel] += r[sel, j][:, None] * (YG[sel] @ _f64(w_out[i]))
+    return dict(O=O, H=H, Gpre=Gpre, G=G, YG=YG, **rt)
+
+
+def inproj_forward(x, w_r, w, k=1, bias=None, renorm=False, tokens=None):
+    """Swimba routed in-projection (Swimba page, Extended abstract, paragraph 2).
+
+    s_t = sum_i r_{t,i} x_t W_i, with W_i [D_m, N_out] producing the X | B | C
+    streams side by side. Returns a dict with S [T,N_out] and router outputs.
+    """
+    x = _f64(x)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+    rt = route(x, w_r, k, bias=bias, renorm=renorm)
+    idx, r = rt["topk_idx"], rt["topk_w"]
+    T = x.shape[0]
+    E, Dm, N = np.shape(w)
+    s = np.zeros((T, N))
+    for i in range(E):
+        for j in range(k):
+            sel = np.nonzero(idx[:, j] == i)[0]
+            if sel.size == 0:
+                continue
+            s[sel] += r[sel, j][:, None] * (x[sel] @ _f64(w[i]))
+    return dict(S=s, **rt)
+
+
+def block_backward(x, w_r, w_in, w_g, w_out, dout, k, bias=None, renorm=False):
+    """Exact gradient of ``block_forward`` for L = sum_t <O_t, dO_t>, S_t held fixed.
+
+    With g_{t,j} = dO_t W_out,S_j^T and dr_{t,j} = <Y_t (.) G_t, g_{t,j}>:
+      d(YG)_t = sum_j r_{t,j} g_{t,j};  dH = d(YG) (.) G;  dGpre = d(YG) (.) Y (.) SiLU'(Gpre)
+      dW_in,i  = sum_{t: i in S_t} x_t^T dH_t
+      dW_g,i   = sum_{t: i in S_t} x_t^T dGpre_t
+      dW_out,i = sum_{(t,j): S_tj = i} r_{t,j} (Y_t (.) G_t)^T dO_t
+      dlogits  = Jacobian of r w.r.t. the logits applied to dr
+                 (full softmax if not renorm; softmax over S_t if renorm)
+      dX = sum_j (dH W_in,S_j^T + dGpre W_g,S_j^T) + dlogits W_r^T
+      dW_r = X^T dlogits, dbias = sum_t dlogits_t
+    """
+    x = _f64(x)
+    dout = _f64(dout)
+    fw = block_forward(x, w_r, w_in, w_g, w_out, k, bias=bias, renorm=renorm)
+    S, r, p = fw["topk_idx"], fw["topk_w"], fw["p"]
+    H, G, Gpre, YG = fw["H"], fw["G"], fw["Gpre"], fw["YG"]
+    T, Dm = x.shape
+    E, _, De = np.shape(w_in)
+    dYG = np.zeros((T, De))
+    dr = np.zeros((T, k))
+    dW_out = np.zeros((E, De, Dm))
+    for i in range(E):
+        for j in range(k):
+            sel = np.nonzero(S[:, j] == i)[0]
+            if sel.size == 0:
+                continue
+            g = dout[sel] @ _f64(w_out[i]).T
+            dr[sel, j] = np.sum(YG[sel] * g, axis=1)
+            dYG[sel] += r[sel, j][:, None] * g
+            dW_out[i] += (r[sel, j][:, None] * YG[sel]).T @ dout[sel]
+    dH = dYG * G
+    dGpre = dYG * H * silu_grad(Gpre)
+    dX = np.zeros((T, Dm))
+    dW_in = np.zeros((E, Dm, De))
+    dW_g = np.zeros((E, Dm, De))
+    for i in range(E):
+        for j in range(k):
+            sel = np.nonzero(S[:, j] == i)[0]
+            if sel.size == 0:
+                continue
+            dW_in[i] += x[sel].T @ dH[sel]
+            dW_g[i] += x[sel].T @ dGpre[sel]
+            dX[sel] += dH[sel] @ _f64(w_in[i]).T + dGpre[sel] @ _f64(w_g[i]).T
+    dlogits = np.zeros((T, E))
+    rows = np.arange(T)
+    if renorm:
+        # r_j = exp(l_Sj) / sum_{i in S} exp(l_i): softmax over the selected logits.
+        inner = np.sum(r * dr, axis=1)
+        for j in range(k):
+            dlogits[rows, S[:, j]] += r[:, j] * (dr[:, j] - inner)
+    else:
+        # r_j = p_{S_j}, p = softmax(l): dl_m = sum_j dr_j p_Sj (delta_{m,Sj} - p_m).
+        inner = np.sum(dr * p[rows[:, None], S], axis=1)
+        dlogits -= p * inner[:, None]
+        for j in range(k):
+            dlogits[rows, S[:, j]] += dr[:, j] * p[rows, S[:, j]]
+    dX += dlogits @ _f64(w_r).T
+    dW_r = x.T @ dlogits
+    dbias = dlogits.sum(axis=0)
+    return dict(dX=dX, dW_in=dW_in, dW_g=dW_g, dW_out=dW_out, dlogits=dlogits, dr=dr,
+                dW_r=dW_r, dbias=dbias, forward=fw)

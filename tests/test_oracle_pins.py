@@ -1,0 +1,340 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle.
+
+Each test fixes the oracle to a closed form, a library routine, a brute-force
+evaluation on tiny inputs, an invariant of the method, or finite differences.
+Sources: "Routing Mamba: Scaling State Space Models with Mixture-of-Experts
+Projection" (chapterpal summary page), Knowl 1; "Swimba: Switch Mamba Model
+Scales State Space Models" (project page), Extended abstract.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+from scipy.special import expit, softmax as sp_softmax
+
+from mixture_experts_projections_b200.inputs import make_block_inputs, make_inproj_inputs
+from oracle import rom_oracle as orc
+
+
+def _silu_ref(z):
+    return z * expit(z)
+
+
+# ---------------------------------------------------------------- closed forms
+
+
+def test_worked_example_closed_form():
+    """A 2-expert, d_model=2, d_inner=2 block evaluated by hand from Knowl 1.
+
+    Token 0: x=[1,0], logits [ln3, 0] -> p=[3/4,1/4], S={0}, r=3/4.
+      H = x W_in,0 = [2, 1]; z = x W_g,0 = [ln3, 0]; G = [ln3*3/4, 0]
+      Y(.)G = [1.5 ln3, 0];  (Y(.)G) W_out,0 = [1.5 ln3, -3 ln3];  O = 3/4 of that.
+    Token 1: x=[-1,0], logits [-ln3, 0] -> p=[1/4,3/4], S={1}, r=3/4.
+      H = x W_in,1 = [-1, 3]; z = x W_g,1 = [0, ln3]; G = [0, ln3*3/4]
+      Y(.)G = [0, 2.25 ln3]; (Y(.)G) W_out,1 = 2.25 ln3 * [4, -1]; O = 3/4 of that.
+    Token 2: x=[0,1], logits [0,0] (tie) -> expert 0, r = 1/2.
+      H = x W_in,0 = [0, 5]; z = x W_g,0 = [0, 0] -> G = 0 -> O = 0.
+    """
+    l3 = math.log(3.0)
+    x = np.array([[1.0, 0.0], [-1.0, 0.0], [0.0, 1.0]])
+    w_r = np.array([[l3, 0.0], [0.0, 0.0]])
+    w_in = np.array([[[2.0, 1.0], [0.0, 5.0]], [[1.0, -3.0], [7.0, 7.0]]])
+    w_g = np.array([[[l3, 0.0], [0.0, 0.0]], [[0.0, -l3], [1.0, 1.0]]])
+    w_out = np.array([[[1.0, -2.0], [5.0, 7.0]], [[9.0, 9.0], [4.0, -1.0]]])
+    fw = orc.block_forward(x, w_r, w_in, w_g, w_out, k=1)
+    assert fw["topk_idx"][:, 0].tolist() == [0, 1, 0]
+    np.testing.assert_allclose(fw["topk_w"][:, 0], [0.75, 0.75, 0.5], rtol=1e-15)
+    exp = np.array([[0.75 * 1.5 * l3, -0.75 * 3 * l3],
+                    [0.75 * 2.25 * l3 * 4, -0.75 * 2.25 * l3],
+                    [0.0, 0.0]])
+    np.testing.assert_allclose(fw["O"], exp, rtol=1e-14, atol=1e-14)
+
+
+def test_softmax_sums_to_one_and_matches_scipy():
+    inp = make_block_inputs(64, 32, 16, 8, seed=3)
+    rt = orc.route(inp["x"], inp["w_r"], 2)
+    np.testing.assert_allclose(rt["p"].sum(1), 1.0, atol=1e-12)
+    ref = sp_softmax(inp["x"].astype(np.float64) @ inp["w_r"].astype(np.float64), axis=1)
+    np.testing.assert_allclose(rt["p"], ref, rtol=1e-12)
+
+
+def test_renormalised_weights_are_softmax_over_selected_logits():
+    inp = make_block_inputs(50, 16, 8, 6, seed=5, router_std=0.5)
+    rt = orc.route(inp["x"], inp["w_r"], 2, renorm=True)
+    np.testing.assert_allclose(rt["topk_w"].sum(1), 1.0, atol=1e-12)
+    rows = np.arange(50)[:, None]
+    sel_logits = rt["logits"][rows, rt["topk_idx"]]
+    np.testing.assert_allclose(rt["topk_w"], sp_softmax(sel_logits, axis=1), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- brute force
+
+
+def _bruteforce_topk(logits, k):
+    """Rank of expert i = number of experts that beat it (larger logit, or
+    equal logit and lower index). S = ranks < k, slot = rank."""
+    T, E = logits.shape
+    idx = np.full((T, k), -1)
+    for t in range(T):
+        for i in range(E):
+            rank = sum(1 for j in range(E)
+                       if logits[t, j] > logits[t, i] or (logits[t, j] == logits[t, i] and j < i))
+            if rank < k:
+                idx[t, rank] = i
+    return idx
+
+
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_topk_matches_bruteforce_rank(k):
+    inp = make_block_inputs(40, 8, 4, 5, seed=11, router_std=1.0)
+    rt = orc.route(inp["x"], inp["w_r"], k)
+    assert np.array_equal(rt["topk_idx"], _bruteforce_topk(rt["logits"], k))
+    # p_{S_j} are the k largest probabilities
+    srt = np.sort(rt["p"], axis=1)[:, ::-1][:, :k]
+    np.testing.assert_allclose(rt["p"][np.arange(40)[:, None], rt["topk_idx"]], srt, rtol=0)
+
+
+def _bruteforce_block(x, w_r, w_in, w_g, w_out, k, renorm):
+    """Evaluate every expert densely for every token, then mask by S_t."""
+    x = x.astype(np.float64)
+    logits = x @ w_r.astype(np.float64)
+    p = sp_softmax(logits, axis=1)
+    S = _bruteforce_topk(logits, k)
+    T = x.shape[0]
+    E, Dm, De = w_in.shape
+    out = np.zeros((T, Dm))
+    for t in range(T):
+        mask = np.zeros(E)
+        mask[S[t]] = 1.0
+        r = p[t] * mask
+        if renorm:
+            r = r / r.sum()
+        u_all = np.stack([x[t] @ w_in[i] for i in range(E)])  # [E, De]
+        z_all = np.stack([x[t] @ w_g[i] for i in range(E)])
+        h = (mask @ u_all) * _silu_ref(mask @ z_all)
+        for i in range(E):
+            out[t] += r[i] * (h @ w_out[i])
+    return out
+
+
+@pytest.mark.parametrize("E,k,renorm", [(1, 1, False), (2, 1, False), (4, 1, False),
+                                        (8, 1, False), (4, 2, False), (4, 2, True),
+                                        (8, 2, True), (3, 3, False)])
+def test_block_matches_dense_bruteforce(E, k, renorm):
+    inp = make_block_inputs(24, 12, 10, E, seed=E * 10 + k, router_std=0.7)
+    args = (inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"])
+    fw = orc.block_forward(*args, k=k, renorm=renorm)
+    ref = _bruteforce_block(*args, k=k, renorm=renorm)
+    np.testing.assert_allclose(fw["O"], ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- special cases
+
+
+def test_single_expert_is_dense_mamba_projection():
+    inp = make_block_inputs(33, 16, 24, 1, seed=2)
+    x = inp["x"].astype(np.float64)
+    fw = orc.block_forward(x, inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], k=1)
+    assert np.all(fw["topk_idx"] == 0)
+    np.testing.assert_allclose(fw["topk_w"], 1.0, rtol=0, atol=0)
+    u = x @ inp["w_conv"][0].astype(np.float64)
+    z = x @ inp["w_gate"][0].astype(np.float64)
+    ref = (u * _silu_ref(z)) @ inp["w_out"][0].astype(np.float64)
+    np.testing.assert_allclose(fw["O"], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_top1_output_is_p_times_dense_block_of_chosen_expert():
+    """For K=1 the block equals p_{t,e} times the dense block of expert e:
+    only Out is routing-weighted, Conv and Gate use the indicator."""
+    inp = make_block_inputs(40, 16, 20, 4, seed=9, router_std=0.5)
+    x = inp["x"].astype(np.float64)
+    fw = orc.block_forward(x, inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], k=1)
+    logits = x @ inp["w_r"].astype(np.float64)
+    e = np.argmax(logits, axis=1)
+    p = sp_softmax(logits, axis=1)[np.arange(40), e]
+    for t in range(40):
+        we = [inp[n][e[t]].astype(np.float64) for n in ("w_conv", "w_gate", "w_out")]
+        dense = ((x[t] @ we[0]) * _silu_ref(x[t] @ we[1])) @ we[2]
+        np.testing.assert_allclose(fw["O"][t], p[t] * dense, rtol=1e-12, atol=1e-13)
+
+
+def test_all_experts_selected_sums_before_silu():
+    """K = E: indicators are all one, so H = x sum_i W_in,i and
+    G = SiLU(x sum_i W_g,i) (SiLU after the sum over experts)."""
+    inp = make_block_inputs(20, 8, 6, 2, seed=4, router_std=0.5)
+    x = inp["x"].astype(np.float64)
+    fw = orc.block_forward(x, inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], k=2)
+    p = sp_softmax(x @ inp["w_r"].astype(np.float64), axis=1)
+    h = (x @ inp["w_conv"].astype(np.float64).sum(0)) * _silu_ref(
+        x @ inp["w_gate"].astype(np.float64).sum(0))
+    ref = p[:, :1] * (h @ inp["w_out"][0].astype(np.float64)) + \
+        p[:, 1:] * (h @ inp["w_out"][1].astype(np.float64))
+    np.testing.assert_allclose(fw["O"], ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("k,renorm", [(1, False), (2, False), (2, True)])
+def test_zero_router_tie_rule(k, renorm):
+    """W_r = 0: every logit ties, so S_t = {0..k-1} in index order, p = 1/E."""
+    inp = make_block_inputs(10, 8, 4, 5, seed=1, zero_router=True)
+    rt = orc.route(inp["x"], inp["w_r"], k, renorm=renorm)
+    assert np.array_equal(rt["topk_idx"], np.tile(np.arange(k), (10, 1)))
+    np.testing.assert_allclose(rt["topk_w"], (1.0 / k) if renorm else 0.2, rtol=1e-15)
+
+
+def test_zero_gate_gives_zero_output():
+    inp = make_block_inputs(16, 8, 8, 4, seed=6)
+    fw = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], np.zeros_like(inp["w_gate"]),
+                           inp["w_out"], k=2)
+    assert np.all(fw["O"] == 0.0)
+
+
+# ---------------------------------------------------------------- invariants
+
+
+def test_token_permutation_equivariance():
+    inp = make_block_inputs(30, 8, 6, 4, seed=12, router_std=0.5)
+    perm = np.random.default_rng(0).permutation(30)
+    a = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], k=2)
+    b = orc.block_forward(inp["x"][perm], inp["w_r"], inp["w_conv"], inp["w_gate"],
+                          inp["w_out"], k=2)
+    np.testing.assert_allclose(b["O"], a["O"][perm], rtol=1e-13, atol=1e-14)
+    assert np.array_equal(b["topk_idx"], a["topk_idx"][perm])
+
+
+def test_expert_relabel_invariance():
+    inp = make_block_inputs(30, 8, 6, 5, seed=13, router_std=0.5)
+    pi = np.array([3, 0, 4, 1, 2])  # new expert n is old expert pi[n]
+    a = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], k=2)
+    b = orc.block_forward(inp["x"], inp["w_r"][:, pi], inp["w_conv"][pi], inp["w_gate"][pi],
+                          inp["w_out"][pi], k=2)
+    np.testing.assert_allclose(b["O"], a["O"], rtol=1e-13, atol=1e-14)
+    assert np.array_equal(pi[b["topk_idx"]], a["topk_idx"])
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_dispatch_is_stable_counting_sort(k):
+    inp = make_block_inputs(97, 8, 4, 6, seed=21, router_std=1.0)
+    idx = orc.route(inp["x"], inp["w_r"], k)["topk_idx"]
+    d = orc.dispatch(idx, 6)
+    flat = idx.reshape(-1)
+    assert np.array_equal(d["counts"], np.bincount(flat, minlength=6))
+    assert np.array_equal(d["offsets"], np.concatenate([[0], np.cumsum(d["counts"])]))
+    assert np.array_equal(d["sorted_slot"], np.argsort(flat, kind="stable"))
+    R = flat.size
+    assert np.array_equal(np.sort(d["sorted_slot"]), np.arange(R))  # bijection
+    assert np.array_equal(d["slot_pos"][d["sorted_slot"]], np.arange(R))  # inverse
+
+
+def test_dispatch_empty_expert_and_no_tokens():
+    idx = np.array([[2], [2], [0]], dtype=np.int32)
+    d = orc.dispatch(idx, 4)
+    assert d["counts"].tolist() == [1, 0, 2, 0]
+    assert d["offsets"].tolist() == [0, 1, 1, 3, 3]
+    assert d["sorted_slot"].tolist() == [2, 0, 1]
+    d0 = orc.dispatch(np.zeros((0, 1), np.int32), 3)
+    assert d0["offsets"].tolist() == [0, 0, 0, 0]
+
+
+# ---------------------------------------------------------------- Swimba in-projection
+
+
+def test_inproj_top1_is_p_times_dense_projection():
+    inp = make_inproj_inputs(20, 16, 12, 4, seed=7, router_std=0.5)
+    x = inp["x"].astype(np.float64)
+    res = orc.inproj_forward(x, inp["w_r"], inp["w"], k=1)
+    logits = x @ inp["w_r"].astype(np.float64)
+    e = np.argmax(logits, axis=1)
+    p = sp_softmax(logits, axis=1)[np.arange(20), e]
+    for t in range(20):
+        np.testing.assert_allclose(res["S"][t], p[t] * (x[t] @ inp["w"][e[t]].astype(np.float64)),
+                                   rtol=1e-12, atol=1e-13)
+
+
+def test_inproj_all_experts_is_probability_weighted_mix():
+    """K = E: the layer applies the p-weighted mixture of expert matrices
+    (parameter-space mixing: one projection with W = sum_i p_i W_i)."""
+    inp = make_inproj_inputs(15, 8, 10, 3, seed=8, router_std=0.5)
+    x = inp["x"].astype(np.float64)
+    res = orc.inproj_forward(x, inp["w_r"], inp["w"], k=3)
+    p = sp_softmax(x @ inp["w_r"].astype(np.float64), axis=1)
+    for t in range(15):
+        wmix = np.tensordot(p[t], inp["w"].astype(np.float64), axes=(0, 0))
+        np.testing.assert_allclose(res["S"][t], x[t] @ wmix, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- backward
+
+
+def _loss(inp, k, renorm, **over):
+    a = {n: over.get(n, inp[n]) for n in ("x", "w_r", "w_conv", "w_gate", "w_out")}
+    fw = orc.block_forward(a["x"], a["w_r"], a["w_conv"], a["w_gate"], a["w_out"], k=k,
+                           renorm=renorm)
+    return float(np.sum(fw["O"] * inp["dout"])), fw["topk_idx"]
+
+
+@pytest.mark.parametrize("k,renorm", [(1, False), (2, False), (2, True)])
+def test_backward_matches_central_differences(k, renorm):
+    inp = make_block_inputs(6, 5, 4, 3, seed=31 + k, router_std=0.8, with_dout=True)
+    inp = {n: (v.astype(np.float64) if v is not None else None) for n, v in inp.items()}
+    fw = orc.route(inp["x"], inp["w_r"], k)
+    assert fw["margin"].min() > 1e-3  # the selection cannot flip under the steps below
+    g = orc.block_backward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                           inp["dout"], k=k, renorm=renorm)
+    names = {"x": "dX", "w_r": "dW_r", "w_conv": "dW_in", "w_gate": "dW_g", "w_out": "dW_out"}
+    h = 1e-6
+    _, idx0 = _loss(inp, k, renorm)
+    for n, gn in names.items():
+        base = inp[n]
+        fd = np.zeros_like(base)
+        for pos in itertools.product(*[range(s) for s in base.shape]):
+            plus = base.copy()
+            plus[pos] += h
+            minus = base.copy()
+            minus[pos] -= h
+            lp, ip = _loss(inp, k, renorm, **{n: plus})
+            lm, im = _loss(inp, k, renorm, **{n: minus})
+            assert np.array_equal(ip, idx0) and np.array_equal(im, idx0)
+            fd[pos] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[gn], fd, rtol=1e-6, atol=1e-8, err_msg=n)
+
+
+def test_backward_router_gradient_closed_form_top1():
+    """K=1 without renormalisation: r = p_e, so dl_m = dr (delta_{m,e} - p_m) p_e."""
+    inp = make_block_inputs(9, 6, 5, 4, seed=40, router_std=0.5, with_dout=True)
+    g = orc.block_backward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                           inp["dout"], k=1)
+    fw = g["forward"]
+    e = fw["topk_idx"][:, 0]
+    p = fw["p"]
+    pe = p[np.arange(9), e]
+    exp = -p * (g["dr"][:, 0] * pe)[:, None]
+    exp[np.arange(9), e] += g["dr"][:, 0] * pe
+    np.testing.assert_allclose(g["dlogits"], exp, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(g["dlogits"].sum(1), 0.0, atol=1e-12)  # softmax shift-invariance
+
+
+# ---------------------------------------------------------------- regression fixture
+
+
+def test_oracle_regression_fixture():
+    """Frozen oracle results (tests/golden/make_golden.py) still reproduce."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "oracle_regression.json")
+    cases = json.load(open(path))["cases"]
+    for name, c in cases.items():
+        if name.startswith("inproj"):
+            inp = make_inproj_inputs(c["T"], c["Dm"], c["N"], c["E"], seed=c["seed"],
+                                     router_std=c["router_std"])
+            s = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=c["k"])
+            np.testing.assert_allclose(s["S"], c["S"], rtol=1e-12, atol=1e-14)
+            continue
+        inp = make_block_inputs(c["T"], c["Dm"], c["De"], c["E"], seed=c["seed"],
+                                router_std=c["router_std"], with_dout=True)
+        bw = orc.block_backward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"],
+                                inp["w_out"], inp["dout"], k=c["k"], renorm=c["renorm"])
+        assert bw["forward"]["topk_idx"].tolist() == c["topk_idx"]
+        np.testing.assert_allclose(bw["forward"]["O"], c["O"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(bw["dX"], c["dX"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(bw["dlogits"], c["dlogits"], rtol=1e-12, atol=1e-14)
