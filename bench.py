@@ -1,0 +1,438 @@
+"""Benchmark of the RoM projection block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = one pass of the whole block over one batch of synthetic input:
+route -> dispatch -> Conv+Gate grouped GEMM (+ gate combine for top-k > 1)
+-> Out grouped GEMM (+ slot sum for top-k > 1); for the Swimba decode
+workload: route -> dispatch -> routed in-projection. Inputs are resident in
+HBM when the timed region starts; L2 is flushed (a 256 MiB write) before
+every timed step, outside the step's events. Each step is timed with CUDA
+events on the launching stream; the dominant kernel is bracketed by its own
+events for the roofline. Under torchrun every rank runs an independent
+replica on its own GPU (the block needs no collective in the forward); the
+reported time is the max over ranks and `value` counts all ranks' tokens.
+
+`--impl reference` times the CPU oracle (the float64 numpy definition) on a
+bounded sample of the same workload on the host cores; under torchrun only
+rank 0 runs it.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_projections_b200.inputs import WORKLOADS, bf16_bits, make_workload_inputs  # noqa
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def block_flops(wl):
+    R = wl.T * wl.k
+    if wl.kind == "inproj":
+        return {"inproj": 2.0 * R * wl.Dm * wl.De}
+    return {"conv_gate": 4.0 * R * wl.Dm * wl.De, "out": 2.0 * R * wl.De * wl.Dm}
+
+
+def inproj_bytes(wl, n_experts_hit):
+    """Algorithmic HBM bytes of the routed in-projection: the weights of the
+    experts that received tokens, x in, the output out (bf16)."""
+    return n_experts_hit * wl.Dm * wl.De * 2 + wl.T * wl.Dm * 2 + wl.T * wl.De * 2
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_sample_run(wl, inp, tokens):
+    """One call of the CPU oracle on the given tokens; returns seconds."""
+    from oracle import rom_oracle as orc
+    t0 = time.perf_counter()
+    if wl.kind == "inproj":
+        orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=wl.k, tokens=tokens)
+    else:
+        orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                          k=wl.k, bias=inp["bias"], renorm=wl.renorm, tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, inp, budget_s=15.0):
+    """Time the oracle on a growing token sample until it takes ~budget_s."""
+    n = 16
+    rng = np.random.default_rng(0)
+    while True:
+        toks = np.sort(rng.choice(wl.T, size=min(n, wl.T), replace=False))
+        dt = oracle_sample_run(wl, inp, toks)
+        if dt >= budget_s / 3 or n >= wl.T:
+            break
+        n = min(wl.T, n * 4)
+    return {"value": len(toks) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(toks)} of {wl.T} tokens of {wl.name} (float64 numpy oracle), "
+                      f"{dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+
+def to_dev(torch, a, bf16):
+    if bf16:
+        return torch.from_numpy(bf16_bits(a).view(np.int16).copy()).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_projections_b200 import rom
+
+    torch.cuda.set_device(local_rank)
+    rom.load_library()
+    wl = WORKLOADS[args.workload]
+    bf16 = wl.dtype == "bf16"
+    inp = make_workload_inputs(wl, seed=0)
+    stream = torch.cuda.current_stream()
+    x = to_dev(torch, inp["x"], bf16)
+    w_r = to_dev(torch, inp["w_r"], False)
+    bias = None if inp.get("bias") is None else to_dev(torch, inp["bias"], False)
+    if wl.kind == "inproj":
+        w = to_dev(torch, inp["w"], bf16).transpose(1, 2).contiguous()
+        bufs = rom.RoutingBuffers(wl.T, wl.Dm, wl.E, wl.k, x.dtype, x.device)
+        out = torch.empty((wl.T, wl.De), dtype=x.dtype, device=x.device)
+        slots = (torch.empty((wl.T * wl.k, wl.De), dtype=torch.float32, device=x.device)
+                 if wl.k > 1 else None)
+    else:
+        ws = {n: to_dev(torch, inp[n], bf16).transpose(1, 2).contiguous()
+              for n in ("w_conv", "w_gate", "w_out")}
+        bufs = rom.BlockBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
+    del inp["x"]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=x.device)
+    ev = {}
+
+    def mark(name):
+        if name not in ev:
+            ev[name] = []
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        ev[name].append(e)
+
+    R = wl.T * wl.k
+
+    def step(record):
+        if wl.kind == "inproj":
+            if record:
+                mark("s")
+            rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, bufs)
+            if record:
+                mark("p0")
+            if wl.k == 1:
+                rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
+                                    bufs.offsets, bufs.sorted_slot, bufs.topk_w, out)
+            else:
+                rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
+                                    bufs.offsets, bufs.sorted_slot, bufs.topk_w, slots)
+            if record:
+                mark("p1")
+            if wl.k > 1:
+                rom.rom_combine(rom.ROM_COMBINE_SUM, rom.ROM_BF16, slots, wl.T, wl.k, wl.De, None,
+                                out)
+            if record:
+                mark("e")
+            return out
+        rb = bufs.routing
+        if record:
+            mark("s")
+        rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, rb)
+        if record:
+            mark("p0")
+        dt = rom.ROM_BF16 if bf16 else rom.ROM_F32
+        xs = rb.x_sorted[:R]
+        if wl.k == 1:
+            rom.rom_expert_proj(rom.ROM_PROJ_CONV_GATE, xs, ws["w_conv"], ws["w_gate"], wl.E, 1,
+                                rb.offsets, rb.sorted_slot, rb.topk_w, bufs.h_sorted)
+            if record:
+                mark("p1")
+            rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None, wl.E, 1,
+                                rb.offsets, rb.sorted_slot, rb.topk_w, bufs.out)
+            if record:
+                mark("p2")
+        else:
+            rom.rom_expert_proj(rom.ROM_PROJ_CONV_GATE, xs, ws["w_conv"], ws["w_gate"], wl.E,
+                                wl.k, rb.offsets, rb.sorted_slot, rb.topk_w, bufs.uz)
+            if record:
+                mark("p1")
+            rom.rom_combine(rom.ROM_COMBINE_GATE, dt, bufs.uz, wl.T, wl.k, wl.De, rb.slot_pos,
+                            bufs.h_sorted)
+            rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None, wl.E,
+                                wl.k, rb.offsets, rb.sorted_slot, rb.topk_w, bufs.o_slots)
+            if record:
+                mark("p2")
+            rom.rom_combine(rom.ROM_COMBINE_SUM, dt, bufs.o_slots, wl.T, wl.k, wl.Dm, None,
+                            bufs.out)
+        if record:
+            mark("e")
+        return bufs.out
+
+    launches_per_step = (3 if wl.kind == "inproj" else 4) + (2 if wl.k > 1 else 0)
+    if wl.kind == "inproj" and wl.k > 1:
+        launches_per_step = 4
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    if rom.rom_get_status() != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    for _ in range(args.steps):
+        flush.zero_()
+        step(True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+
+    def span(a, b):
+        return [s.elapsed_time(e) for s, e in zip(ev[a], ev[b])]
+
+    step_ms = span("s", "e")
+    t_total_ms = float(np.sum(step_ms))
+    parts = {"route_dispatch": span("s", "p0"), "proj0": span("p0", "p1")}
+    if wl.kind != "inproj":
+        parts["proj1"] = span("p1", "p2")
+    part_ms = {n: float(np.mean(v)) for n, v in parts.items()}
+
+    # ---------------------------------------------- e2e through host buffers
+    h_x = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    h_x.copy_(x)
+    out_t = out if wl.kind == "inproj" else bufs.out
+    h_out = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        x.copy_(h_x, non_blocking=True)
+        o = step(False)
+        h_out.copy_(o, non_blocking=True)
+        s1.record(stream)
+        s1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(s0.elapsed_time(s1))
+    e2e_total = float(np.sum(e2e_ms))
+
+    stats = torch.tensor([t_total_ms, e2e_total], dtype=torch.float64, device=x.device)
+    if world > 1:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    t_total_ms, e2e_total = float(stats[0]), float(stats[1])
+    res = dict(wl=wl, step_ms=t_total_ms / args.steps, part_ms=part_ms,
+               e2e_ms=e2e_total / args.steps, clocks=clk, launches=launches_per_step * args.steps,
+               counts=bufs.counts.cpu().numpy() if wl.kind == "inproj" else
+               bufs.routing.counts.cpu().numpy(), x_bytes=x.numel() * x.element_size(),
+               out_bytes=out_t.numel() * out_t.element_size())
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_16k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOADS[args.workload]
+    flops = block_flops(wl)
+    metric = "tokens/s for RoM projection block fwd"
+    config = {"workload": wl.name, "tokens": wl.T, "d_model": wl.Dm,
+              ("d_out" if wl.kind == "inproj" else "d_inner"): wl.De, "experts": wl.E,
+              "top_k": wl.k, "renorm": wl.renorm, "parallelism": f"replicas x{world}",
+              "l2": "flushed before every timed step (256 MiB write)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = make_workload_inputs(wl, seed=0)
+        rng = np.random.default_rng(1)
+        n = 64 if wl.kind == "block" else wl.T
+        times = []
+        for i in range(args.warmup + args.steps):
+            toks = np.sort(rng.choice(wl.T, size=min(n, wl.T), replace=False))
+            dt = oracle_sample_run(wl, inp, toks)
+            if i >= args.warmup:
+                times.append(dt)
+        t = float(np.sum(times))
+        val = len(toks) * args.steps / t
+        line = {"impl": "reference", "metric": metric, "value": val, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config,
+                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
+                                 "kind": "oracle",
+                                 "sample": f"{min(n, wl.T)} random tokens of {wl.T} per step"},
+                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        pass
+    if rank == 0:
+        peaks, src = load_peaks()
+        step_s = res["step_ms"] / 1e3
+        value = wl.T * world / step_s
+        tot_flops = sum(flops.values())
+        if wl.kind == "inproj":
+            n_hit = int(np.count_nonzero(res["counts"]))
+            t_k = res["part_ms"]["proj0"] / 1e3
+            ach = inproj_bytes(wl, n_hit) / t_k / 1e9
+            roof = {"bound": "hbm", "kernel": "rom_expert_proj(INPROJ)", "achieved": ach,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                    "traffic": None, "peak_source": f"{src} hbm_gbs"}
+        else:
+            t_k = res["part_ms"]["proj0"] / 1e3
+            ach = flops["conv_gate"] / t_k / 1e12
+            pk = peaks["bf16_tflops"]
+            roof = {"bound": "tensor", "kernel": "rom_expert_proj(CONV_GATE)", "achieved": ach,
+                    "peak": pk, "unit": "TFLOP/s", "frac": ach / pk, "traffic": None,
+                    "peak_source": f"{src} bf16_tflops (burst)"}
+        line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["step_ms"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+                "config": config, "roofline": roof,
+                "block_tflops": tot_flops / step_s / 1e12,
+                "block_frac_of_bf16_peak": tot_flops / step_s / 1e12 / peaks["bf16_tflops"],
+                "kernels_ms": res["part_ms"],
+                "e2e": {"value": wl.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": res["x_bytes"], "d2h_bytes_per_step": res["out_bytes"]},
+                "gpu_launches": res["launches"], "clocks": res["clocks"],
+                "expert_load": (res["counts"] / max(1, res["counts"].sum())).round(4).tolist()}
+        if not args.no_cpu_baseline and world == 1:
+            inp = make_workload_inputs(wl, seed=0)
+            line["cpu_baseline"] = cpu_baseline(wl, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

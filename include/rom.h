@@ -1,0 +1,184 @@
+/*
+ * rom.h -- C ABI of librom.so, the sm_100a (B200) implementation of the
+ * Routing Mamba (RoM) mixture-of-experts projection block.
+ *
+ * Method: "Routing Mamba: Scaling State Space Models with Mixture-of-Experts
+ * Projection" (chapterpal summary page), Knowl 1. For a token x_t in R^{D_m},
+ * a router W_r in R^{D_m x E} gives p_t = Softmax(x_t W_r) and the set S_t of
+ * the K largest probabilities; r_{t,i} = p_{t,i} 1[i in S_t]. The same S_t
+ * drives the input (Conv) and Gate projections
+ *     H_t = sum_i 1[i in S_t] x_t W_in,i,   G_t = SiLU(sum_i 1[i in S_t] x_t W_g,i)
+ * and, after the (unchanged, here identity) conv + SSM core Y_t, the output
+ *     O_t = sum_i r_{t,i} (Y_t (.) G_t) W_out,i.
+ * Knowl 12 of the same page: dropless (no capacity factor, no token dropping).
+ * The Swimba in-projection ("Swimba: Switch Mamba Model Scales State Space
+ * Models", project page, Extended abstract, paragraph 2) is the routed,
+ * routing-weighted projection s_t = sum_i r_{t,i} x_t W_i of the X|B|C streams.
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless stated otherwise. The caller owns all
+ *    memory; the library allocates nothing on these paths.
+ *  - Row-major, contiguous. bf16 data is passed as raw 16-bit words.
+ *  - Expert weights are stored [E][N][K] ("output feature major", the
+ *    nn.Linear layout): row n of expert e holds the K weights of output
+ *    feature n. In the pages' notation W_i in R^{K x N}, so the stored matrix
+ *    is W_i transposed.
+ *  - Slots: token t's j-th selected expert is slot s = t*k + j.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t, may be NULL for
+ *    the legacy default stream) and enqueues no host synchronisation.
+ *  - The return value reports argument validation and launch errors
+ *    (rom_status). Errors found on the device (a bounded wait that ran out)
+ *    are recorded in a per-device status word read by rom_get_status().
+ *  - Arguments are checked before anything is launched; on a non-zero return
+ *    nothing was enqueued, unless the code is ROM_ERR_CUDA from a launch.
+ */
+#ifndef ROM_H_
+#define ROM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ROM_OK = 0,
+  ROM_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad enum, k > E, ... */
+  ROM_ERR_UNSUPPORTED = 2, /* valid but not implemented (shape or alignment limit) */
+  ROM_ERR_WORKSPACE = 3,   /* workspace missing or smaller than rom_workspace_size() */
+  ROM_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  ROM_ERR_TIMEOUT = 5      /* device side: a bounded wait ran out (see rom_get_status) */
+} rom_status;
+
+typedef enum { ROM_F32 = 0, ROM_BF16 = 1 } rom_dtype;
+
+typedef enum {
+  ROM_PROJ_CONV_GATE = 0, /* Conv (input) and Gate projections, shared selection */
+  ROM_PROJ_OUT = 1,       /* Out projection, weighted by r */
+  ROM_PROJ_INPROJ = 2     /* Swimba routed in-projection, weighted by r */
+} rom_proj;
+
+typedef enum {
+  ROM_COMBINE_SUM = 0, /* out[t] = sum_j in[t*k+j]                     */
+  ROM_COMBINE_GATE = 1 /* h_t = (sum_j u_{t,j}) * SiLU(sum_j z_{t,j}) */
+} rom_combine_mode;
+
+/* Human-readable name of a rom_status value (static string). */
+const char* rom_status_string(int status);
+
+/* ABI version of this library (incremented on incompatible changes). */
+int rom_version(void);
+
+/*
+ * Bytes of workspace that rom_route() fills and rom_dispatch() reads for T
+ * tokens and E experts (the per-chunk expert histograms). Host function.
+ */
+size_t rom_workspace_size(int64_t T, int E);
+
+/*
+ * rom_route -- router: logits, softmax, top-k selection and expert histogram
+ * (RoM page, Knowl 1: p_t = Softmax(x_t W_r), S_t, r_{t,i}).
+ *
+ *  x        [T][Dm]   activations, dtype (ROM_BF16 words or float)
+ *  w_r      [Dm][E]   router weight, float32 (both dtypes)
+ *  bias     [E]       optional additive logit bias, float32, or NULL
+ *  k                  experts per token, 1 <= k <= min(E, 8); E <= 64
+ *  renorm             0: r = p (the formula); 1: r = p / sum_{S_t} p
+ *  topk_idx [T][k]    out, int32: S_t, slot j = j-th largest logit; equal
+ *                     logits go to the lower expert index
+ *  topk_w   [T][k]    out, float32: r_{t, topk_idx[t][j]}
+ *  counts   [E]       out, int32 per-expert slot count, or NULL (not written)
+ *  ws, ws_bytes       workspace of at least rom_workspace_size(T, E) bytes;
+ *                     rom_dispatch() must receive the same workspace, unchanged,
+ *                     on the same stream, after this call.
+ *
+ * Precision: logits are accumulated in float32 in a fixed order together with
+ * a rigorous bound on their rounding error; a token whose top-k decision is
+ * not certain under that bound has its logits recomputed in float64 before
+ * the decision. The softmax is evaluated in float32.
+ * Requires Dm % 8 == 0 for bf16 and Dm % 4 == 0 for float32 (16-byte rows).
+ */
+int rom_route(const void* x, int dtype, int64_t T, int Dm, const float* w_r, const float* bias,
+              int E, int k, int renorm, int32_t* topk_idx, float* topk_w, int32_t* counts,
+              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * rom_dispatch -- dropless permutation into expert-contiguous order
+ * (RoM page, Knowl 12: no capacity factor, no token dropping).
+ * Order: expert-major, ascending slot index inside an expert (stable).
+ *
+ *  x           [T][Dm]   activations (as given to rom_route)
+ *  topk_idx    [T][k]    from rom_route
+ *  ws, ws_bytes          the workspace rom_route filled
+ *  offsets     [E+1]     out, int32: exclusive prefix of the per-expert counts;
+ *                        offsets[E] = T*k
+ *  sorted_slot [T*k]     out, int32: sorted position -> slot
+ *  slot_pos    [T*k]     out, int32: slot -> sorted position
+ *  x_sorted    [T*k][Dm] out, dtype: x_sorted[p] = x[sorted_slot[p] / k]
+ */
+int rom_dispatch(const void* x, int dtype, int64_t T, int Dm, int E, int k,
+                 const int32_t* topk_idx, const void* ws, size_t ws_bytes, int32_t* offsets,
+                 int32_t* sorted_slot, int32_t* slot_pos, void* x_sorted, void* stream);
+
+/*
+ * rom_expert_proj -- grouped expert projection over the dispatched rows.
+ * For expert e, rows offsets[e] .. offsets[e+1]-1 of `a_sorted` ([R][K],
+ * R = T*k) are multiplied by expert e's matrix; the experts' row counts are
+ * read on the device (no host synchronisation).
+ *
+ *  ROM_PROJ_CONV_GATE (RoM page, Knowl 1, H_t and G_t):
+ *     w0 = W_in [E][N][K], w1 = W_g [E][N][K]  (K = D_m, N = D_e)
+ *     k == 1: out = h_sorted [R][N] dtype, h = u * SiLU(z) with u = x W_in,e,
+ *             z = x W_g,e (the identity stands in for the conv + SSM core);
+ *     k  > 1: out = float32 [2][R][N] in SLOT order: out[0][s] = u, out[1][s] = z
+ *             of slot s; rom_combine(ROM_COMBINE_GATE) then sums over the
+ *             slots before SiLU.
+ *  ROM_PROJ_OUT (RoM page, Knowl 1, O_t): w0 = W_out [E][N][K] (K = D_e, N = D_m),
+ *     w1 = NULL. Each row is scaled by r = topk_w[slot] in float32.
+ *     k == 1: out = O [T][N] dtype in token order;
+ *     k  > 1: out = float32 [R][N] in slot order (rom_combine(ROM_COMBINE_SUM)).
+ *  ROM_PROJ_INPROJ (Swimba page, Extended abstract): w0 = W [E][N][K], the
+ *     X|B|C in-projection; same weighting and outputs as ROM_PROJ_OUT.
+ *
+ *  bf16 (tensor cores, tcgen05 + TMA): requires K % 8 == 0, N % 128 == 0 and
+ *  16-byte aligned a_sorted, w0, w1 and out. float32 (CUDA-core FMA): any K, N.
+ */
+int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K, const void* w0,
+                    const void* w1, int N, int E, int k, const int32_t* offsets,
+                    const int32_t* sorted_slot, const float* topk_w, void* out, void* stream);
+
+/*
+ * rom_combine -- reduce the k slots of each token in slot order 0..k-1.
+ *  ROM_COMBINE_SUM:  in = float32 [T*k][N] (slot order); out = [T][N] dtype,
+ *                    out[t] = sum_j in[t*k+j]. slot_pos is unused (may be NULL).
+ *  ROM_COMBINE_GATE: in = float32 [2][T*k][N] (u then z, slot order);
+ *                    h_t = (sum_j u[t*k+j]) * SiLU(sum_j z[t*k+j]) (RoM page,
+ *                    Knowl 1: SiLU after the sum over the selected experts);
+ *                    out = h_sorted [T*k][N] dtype with h_t written to row
+ *                    slot_pos[t*k+j] for every j.
+ *  Requires N % 4 == 0.
+ */
+int rom_combine(int mode, int dtype, const void* in, int64_t T, int k, int N,
+                const int32_t* slot_pos, void* out, void* stream);
+
+/*
+ * rom_get_status -- synchronises `stream`, copies the calling device's status
+ * word to *host_status (host pointer) and resets it to ROM_OK. One word per
+ * device, shared by all streams.
+ */
+int rom_get_status(void* stream, int32_t* host_status);
+
+/*
+ * rom_debug_wait_timeout -- launches one CTA that waits on an mbarrier that
+ * nothing arrives on, with a limit of `limit_ns` nanoseconds (1e3 .. 1e10).
+ * The wait must run out and record ROM_ERR_TIMEOUT in the status word; used
+ * to test the bounded-wait path without hanging the GPU.
+ */
+int rom_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROM_H_ */

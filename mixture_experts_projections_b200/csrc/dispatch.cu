@@ -1,0 +1,149 @@
+// Dropless dispatch of the RoM block: a stable counting sort of the routed
+// slots by expert, and the gather of the token rows into expert-contiguous
+// order. ("Routing Mamba ..." chapterpal summary page, Knowl 12: no expert
+// parallelism, no capacity factor, no token dropping.)
+//
+// One CTA per 128-token chunk (the router's chunk). From the per-chunk expert
+// histograms the router left in the workspace, the CTA forms the global
+// offsets (exclusive prefix of the totals) and its own base per expert (sum
+// of the earlier chunks). Inside the chunk, slots are ranked per expert in
+// ascending slot order: warps rank 32 consecutive slots with __match_any_sync,
+// and a per-expert prefix over the 32-slot groups orders the groups. The
+// result needs no atomics on the global order and is deterministic.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "rom_internal.cuh"
+
+namespace rom {
+namespace {
+
+constexpr int kDispatchThreads = 256;
+constexpr int kDispatchWarps = kDispatchThreads / 32;
+constexpr int kMaxGroups = kChunkTokens * kMaxTopK / 32;  // 32-slot groups per chunk
+
+__global__ void __launch_bounds__(kDispatchThreads)
+    dispatch_kernel(const uint4* __restrict__ x, int64_t T, int row_vec16, int E, int k,
+                    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ chunk_hist,
+                    int64_t nchunks, int32_t* __restrict__ offsets,
+                    int32_t* __restrict__ sorted_slot, int32_t* __restrict__ slot_pos,
+                    uint4* __restrict__ x_sorted) {
+  __shared__ int s_tot[kMaxExperts];
+  __shared__ int s_base[kMaxExperts];
+  __shared__ int s_off[kMaxExperts + 1];
+  __shared__ int s_gcount[kMaxGroups][kMaxExperts];
+  __shared__ int s_pos[kChunkTokens * kMaxTopK];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t c = blockIdx.x;
+  const int64_t R = T * k;
+  const int64_t s0 = c * kChunkTokens * k;
+  const int ns = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(kChunkTokens) * k, R - s0));
+  const int ngroups = (ns + 31) / 32;
+
+  for (int e = tid; e < E; e += kDispatchThreads) {
+    s_tot[e] = 0;
+    s_base[e] = 0;
+  }
+  for (int i = tid; i < ngroups * kMaxExperts; i += kDispatchThreads)
+    s_gcount[i / kMaxExperts][i % kMaxExperts] = 0;
+  __syncthreads();
+  for (int64_t i = tid; i < nchunks * E; i += kDispatchThreads) {
+    const int v = chunk_hist[i];
+    const int e = static_cast<int>(i % E);
+    if (v) {
+      atomicAdd(&s_tot[e], v);
+      if (i / E < c) atomicAdd(&s_base[e], v);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = run;
+      run += s_tot[e];
+    }
+    s_off[E] = run;
+  }
+  __syncthreads();
+  if (c == 0)
+    for (int e = tid; e <= E; e += kDispatchThreads) offsets[e] = s_off[e];
+
+  // Per-group, per-expert counts and the rank of each slot inside its group.
+  int my_rank[kMaxGroups / kDispatchWarps];
+  int my_e[kMaxGroups / kDispatchWarps];
+#pragma unroll
+  for (int q = 0; q < kMaxGroups / kDispatchWarps; ++q) {
+    const int g = warp + q * kDispatchWarps;
+    my_e[q] = -1;
+    my_rank[q] = 0;
+    if (g < ngroups) {
+      const int ls = g * 32 + lane;
+      const int e = (ls < ns) ? topk_idx[s0 + ls] : -1 - lane;  // unique key for idle lanes
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      my_rank[q] = __popc(same & ((1u << lane) - 1u));
+      my_e[q] = (ls < ns) ? e : -1;
+      if (ls < ns && my_rank[q] == 0) s_gcount[g][e] = __popc(same);
+    }
+  }
+  __syncthreads();
+  // Exclusive prefix over groups, per expert (in place).
+  for (int e = tid; e < E; e += kDispatchThreads) {
+    int run = 0;
+    for (int g = 0; g < ngroups; ++g) {
+      const int v = s_gcount[g][e];
+      s_gcount[g][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < kMaxGroups / kDispatchWarps; ++q) {
+    const int g = warp + q * kDispatchWarps;
+    if (g < ngroups && my_e[q] >= 0) {
+      const int ls = g * 32 + lane;
+      const int e = my_e[q];
+      const int pos = s_off[e] + s_base[e] + s_gcount[g][e] + my_rank[q];
+      sorted_slot[pos] = static_cast<int32_t>(s0 + ls);
+      slot_pos[s0 + ls] = pos;
+      s_pos[ls] = pos;
+    }
+  }
+  __syncthreads();
+  // Gather: one warp per slot row, 16-byte vectors, 4 in flight per lane.
+  for (int ls = warp; ls < ns; ls += kDispatchWarps) {
+    const int64_t src = (s0 + ls) / k;
+    const uint4* srow = x + src * row_vec16;
+    uint4* drow = x_sorted + static_cast<int64_t>(s_pos[ls]) * row_vec16;
+    int i = lane;
+    for (; i + 96 < row_vec16; i += 128) {
+      const uint4 a = __ldg(srow + i), b = __ldg(srow + i + 32), cc = __ldg(srow + i + 64),
+                  d = __ldg(srow + i + 96);
+      drow[i] = a;
+      drow[i + 32] = b;
+      drow[i + 64] = cc;
+      drow[i + 96] = d;
+    }
+    for (; i < row_vec16; i += 32) drow[i] = __ldg(srow + i);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const void* x, bool bf16, int64_t T, int Dm, int E, int k,
+                            const int32_t* topk_idx, const int32_t* chunk_hist,
+                            int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,
+                            void* x_sorted, cudaStream_t stream) {
+  const int64_t nchunks = num_chunks(T);
+  if (nchunks == 0) {
+    // No tokens: offsets are all zero.
+    return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream);
+  }
+  const int row_bytes = Dm * (bf16 ? 2 : 4);
+  dispatch_kernel<<<static_cast<unsigned>(nchunks), kDispatchThreads, 0, stream>>>(
+      static_cast<const uint4*>(x), T, row_bytes / 16, E, k, topk_idx, chunk_hist, nchunks,
+      offsets, sorted_slot, slot_pos, static_cast<uint4*>(x_sorted));
+  return cudaGetLastError();
+}
+
+}  // namespace rom

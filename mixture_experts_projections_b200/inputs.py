@@ -76,9 +76,13 @@ WORKLOAD_ORDER = ["tiny_fp32", "prefill_16k", "imbalanced_8x4096", "decode_swimb
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 (ties to even); returns float32."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = a.view(np.uint32)
+    # finite inputs only: the largest finite pattern + 0x8000 stays below 2^32
+    r = (u >> 16) & 1
+    r += 0x7FFF
+    r += u
+    r &= 0xFFFF0000
+    return r.view(np.float32)
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:

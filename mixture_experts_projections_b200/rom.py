@@ -1,0 +1,244 @@
+"""Python binding of librom.so (the C ABI in include/rom.h).
+
+Argument marshalling only: every step of the RoM block runs in the CUDA
+library. PyTorch supplies device memory and the current stream. The functions
+keep the C names (rom_route, rom_dispatch, rom_expert_proj, rom_combine, ...);
+``block_forward`` and ``inproj_forward`` chain them for one block.
+
+Importing this module does not need a GPU; calling into the library does, and
+a missing library raises at once (there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librom.so")
+
+ROM_OK, ROM_ERR_INVALID_ARG, ROM_ERR_UNSUPPORTED, ROM_ERR_WORKSPACE, ROM_ERR_CUDA, \
+    ROM_ERR_TIMEOUT = range(6)
+ROM_F32, ROM_BF16 = 0, 1
+ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ = 0, 1, 2
+ROM_COMBINE_SUM, ROM_COMBINE_GATE = 0, 1
+
+# Every exported symbol of include/rom.h with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_int64
+SIGNATURES = {
+    "rom_status_string": (ctypes.c_char_p, [_I]),
+    "rom_version": (_I, []),
+    "rom_workspace_size": (ctypes.c_size_t, [_L, _I]),
+    "rom_route": (_I, [_P, _I, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "rom_dispatch": (_I, [_P, _I, _L, _I, _I, _I, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P]),
+    "rom_expert_proj": (_I, [_I, _I, _P, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "rom_combine": (_I, [_I, _I, _P, _L, _I, _I, _P, _P, _P]),
+    "rom_get_status": (_I, [_P, ctypes.POINTER(ctypes.c_int32)]),
+    "rom_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+}
+
+_lib = None
+
+
+class RomError(RuntimeError):
+    pass
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load librom.so (once) and declare the signatures of its entry points."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RomError(f"{path} is missing: build it with "
+                           "`python -m mixture_experts_projections_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != ROM_OK:
+        msg = load_library().rom_status_string(code).decode()
+        raise RomError(f"{what} failed: {msg} ({code})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ROM_BF16
+    if t.dtype == torch.float32:
+        return ROM_F32
+    raise RomError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise RomError(f"{name} must be a contiguous CUDA tensor")
+
+
+# ------------------------------------------------------------------ C entry points
+
+
+def rom_workspace_size(T: int, E: int) -> int:
+    return int(load_library().rom_workspace_size(T, E))
+
+
+def rom_route(x, w_r, bias, k, renorm, topk_idx, topk_w, counts, ws, stream=None):
+    for t, n in ((x, "x"), (w_r, "w_r"), (topk_idx, "topk_idx"), (topk_w, "topk_w")):
+        _need(t, n)
+    T, Dm = x.shape
+    E = w_r.shape[1]
+    _check(load_library().rom_route(
+        _ptr(x), _dtype_code(x), T, Dm, _ptr(w_r), _ptr(bias), E, k, int(renorm),
+        _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)), "rom_route")
+
+
+def rom_dispatch(x, E, k, topk_idx, ws, offsets, sorted_slot, slot_pos, x_sorted, stream=None):
+    T, Dm = x.shape
+    _check(load_library().rom_dispatch(
+        _ptr(x), _dtype_code(x), T, Dm, E, k, _ptr(topk_idx), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(offsets), _ptr(sorted_slot),
+        _ptr(slot_pos), _ptr(x_sorted), _stream(stream)), "rom_dispatch")
+
+
+def rom_expert_proj(proj, a_sorted, w0, w1, E, k, offsets, sorted_slot, topk_w, out,
+                    stream=None):
+    R, K = a_sorted.shape
+    N = w0.shape[1]
+    _check(load_library().rom_expert_proj(
+        proj, _dtype_code(a_sorted), _ptr(a_sorted), R, K, _ptr(w0), _ptr(w1), N, E, k,
+        _ptr(offsets), _ptr(sorted_slot), _ptr(topk_w), _ptr(out), _stream(stream)),
+        "rom_expert_proj")
+
+
+def rom_combine(mode, dtype_code, inp, T, k, N, slot_pos, out, stream=None):
+    _check(load_library().rom_combine(mode, dtype_code, _ptr(inp), T, k, N, _ptr(slot_pos),
+                                      _ptr(out), _stream(stream)), "rom_combine")
+
+
+def rom_get_status(stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(load_library().rom_get_status(_stream(stream), ctypes.byref(v)), "rom_get_status")
+    return int(v.value)
+
+
+def rom_debug_wait_timeout(limit_ns: int, stream=None):
+    _check(load_library().rom_debug_wait_timeout(limit_ns, _stream(stream)),
+           "rom_debug_wait_timeout")
+
+
+# ------------------------------------------------------------------ block helpers
+
+
+def expert_weight_layout(w_pages: torch.Tensor) -> torch.Tensor:
+    """[E, K, N] (the pages' x W notation) -> the library's [E, N, K] layout."""
+    return w_pages.transpose(1, 2).contiguous()
+
+
+class RoutingBuffers:
+    """Device buffers of one routing + dispatch pass (allocated by torch)."""
+
+    def __init__(self, T, Dm, E, k, dtype, device):
+        R = T * k
+        self.T, self.Dm, self.E, self.k = T, Dm, E, k
+        self.topk_idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.counts = torch.empty((E,), dtype=torch.int32, device=device)
+        nws = max(1, rom_workspace_size(T, E) // 4)
+        self.ws = torch.empty((nws,), dtype=torch.int32, device=device)
+        self.offsets = torch.empty((E + 1,), dtype=torch.int32, device=device)
+        self.sorted_slot = torch.empty((max(R, 1),), dtype=torch.int32, device=device)
+        self.slot_pos = torch.empty((max(R, 1),), dtype=torch.int32, device=device)
+        self.x_sorted = torch.empty((max(R, 1), Dm), dtype=dtype, device=device)
+
+
+def route_and_dispatch(x, w_r, bias, E, k, renorm, bufs=None, stream=None):
+    T, Dm = x.shape
+    if bufs is None:
+        bufs = RoutingBuffers(T, Dm, E, k, x.dtype, x.device)
+    rom_route(x, w_r, bias, k, renorm, bufs.topk_idx, bufs.topk_w, bufs.counts, bufs.ws, stream)
+    rom_dispatch(x, E, k, bufs.topk_idx, bufs.ws, bufs.offsets, bufs.sorted_slot, bufs.slot_pos,
+                 bufs.x_sorted, stream)
+    return bufs
+
+
+class BlockBuffers:
+    """Intermediate and output buffers of one RoM block forward."""
+
+    def __init__(self, T, Dm, De, E, k, dtype, device):
+        R = T * k
+        self.routing = RoutingBuffers(T, Dm, E, k, dtype, device)
+        self.h_sorted = torch.empty((max(R, 1), De), dtype=dtype, device=device)
+        self.uz = (torch.empty((2, R, De), dtype=torch.float32, device=device)
+                   if k > 1 else None)
+        self.o_slots = (torch.empty((R, Dm), dtype=torch.float32, device=device)
+                        if k > 1 else None)
+        self.out = torch.empty((T, Dm), dtype=dtype, device=device)
+
+
+def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=None, stream=None):
+    """RoM block forward: route, dispatch, Conv+Gate, (gate combine), Out, (sum).
+
+    x [T, Dm] (bf16 or float32), w_r [Dm, E] float32, bias [E] float32 or None,
+    w_conv, w_gate [E, De, Dm] and w_out [E, Dm, De] in the library layout.
+    Returns the BlockBuffers holding O (``.out``) and the intermediates.
+    """
+    T, Dm = x.shape
+    E, De, _ = w_conv.shape
+    if bufs is None:
+        bufs = BlockBuffers(T, Dm, De, E, k, x.dtype, x.device)
+    rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs.routing, stream)
+    R = T * k
+    xs = rb.x_sorted[:R]
+    if k == 1:
+        rom_expert_proj(ROM_PROJ_CONV_GATE, xs, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
+                        rb.topk_w, bufs.h_sorted, stream)
+        rom_expert_proj(ROM_PROJ_OUT, bufs.h_sorted[:R], w_out, None, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, bufs.out, stream)
+    else:
+        rom_expert_proj(ROM_PROJ_CONV_GATE, xs, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
+                        rb.topk_w, bufs.uz, stream)
+        rom_combine(ROM_COMBINE_GATE, _dtype_code(x), bufs.uz, T, k, De, rb.slot_pos,
+                    bufs.h_sorted, stream)
+        rom_expert_proj(ROM_PROJ_OUT, bufs.h_sorted[:R], w_out, None, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, bufs.o_slots, stream)
+        rom_combine(ROM_COMBINE_SUM, _dtype_code(x), bufs.o_slots, T, k, Dm, None, bufs.out,
+                    stream)
+    return bufs
+
+
+def inproj_forward(x, w_r, w, k=1, renorm=False, bias=None, bufs=None, out=None, slots=None,
+                   stream=None):
+    """Swimba routed in-projection: s_t = sum_j r_{t,j} x_t W_{S_j} (W as [E, N, Dm])."""
+    T, Dm = x.shape
+    E, N, _ = w.shape
+    rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs, stream)
+    if out is None:
+        out = torch.empty((T, N), dtype=x.dtype, device=x.device)
+    R = T * k
+    if k == 1:
+        rom_expert_proj(ROM_PROJ_INPROJ, rb.x_sorted[:R], w, None, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, out, stream)
+    else:
+        if slots is None:
+            slots = torch.empty((R, N), dtype=torch.float32, device=x.device)
+        rom_expert_proj(ROM_PROJ_INPROJ, rb.x_sorted[:R], w, None, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, slots, stream)
+        rom_combine(ROM_COMBINE_SUM, _dtype_code(x), slots, T, k, N, None, out, stream)
+    return out, rb

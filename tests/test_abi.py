@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads,
+exports every entry point that include/rom.h declares, and rejects invalid
+arguments before it enqueues anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixture_experts_projections_b200.build import build
+    build()
+    from mixture_experts_projections_b200 import rom
+    return rom.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "rom.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(rom_\w+)\s*\(", text,
+                                 flags=re.M)))
+
+
+def test_header_declares_the_four_block_entry_points():
+    names = declared_functions()
+    for n in ("rom_route", "rom_dispatch", "rom_expert_proj", "rom_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from mixture_experts_projections_b200 import rom
+    names = declared_functions()
+    assert names, "no declarations parsed from include/rom.h"
+    for n in names:
+        assert hasattr(lib, n), f"librom.so does not export {n}"
+        assert n in rom.SIGNATURES, f"the Python binding does not declare {n}"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.rom_status_string(0) == b"ROM_OK"
+    assert lib.rom_status_string(5) == b"ROM_ERR_TIMEOUT"
+    assert lib.rom_status_string(99) == b"ROM_ERR_UNKNOWN"
+    assert lib.rom_version() >= 1
+
+
+def test_workspace_size(lib):
+    assert lib.rom_workspace_size(0, 8) == 0
+    assert lib.rom_workspace_size(1, 8) == 8 * 4
+    assert lib.rom_workspace_size(128, 8) == 8 * 4
+    assert lib.rom_workspace_size(129, 8) == 2 * 8 * 4
+    assert lib.rom_workspace_size(16384, 8) == 128 * 8 * 4
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced by these calls
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), 1), (dict(E=0), 1), (dict(E=65), 1), (dict(k=9, E=16), 1), (dict(k=3, E=2), 1),
+    (dict(renorm=2), 1), (dict(Dm=0), 1), (dict(T=-1), 1), (dict(Dm=12), 2), (dict(x=None), 1),
+    (dict(ws=None), 3), (dict(ws_bytes=4), 3), (dict(x=ctypes.c_void_p((1 << 20) + 2)), 2),
+])
+def test_route_rejects_bad_arguments(lib, kw, code):
+    a = dict(x=FAKE, dtype=1, T=256, Dm=64, w_r=FAKE, bias=None, E=8, k=1, renorm=0,
+             topk_idx=FAKE, topk_w=FAKE, counts=None, ws=FAKE, ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    assert lib.rom_route(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(proj=3), 1), (dict(dtype=2), 1), (dict(K=0), 1), (dict(N=0), 1), (dict(k=2, R=7), 1),
+    (dict(w1=None), 1), (dict(offsets=None), 1), (dict(N=200), 2), (dict(K=12), 2),
+    (dict(out=ctypes.c_void_p((1 << 20) + 8)), 2),
+    (dict(proj=1, N=320), 2),
+    (dict(proj=1, topk_w=None), 1),
+])
+def test_expert_proj_rejects_bad_arguments(lib, kw, code):
+    a = dict(proj=0, dtype=1, a_sorted=FAKE, R=256, K=64, w0=FAKE, w1=FAKE, N=256, E=8, k=1,
+             offsets=FAKE, sorted_slot=FAKE, topk_w=FAKE, out=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_expert_proj(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=2), 1), (dict(dtype=3), 1), (dict(k=0), 1), (dict(k=9), 1), (dict(N=6), 2),
+    (dict(mode=1, slot_pos=None), 1), (dict(inp=None), 1),
+])
+def test_combine_rejects_bad_arguments(lib, kw, code):
+    a = dict(mode=0, dtype=1, inp=FAKE, T=10, k=2, N=64, slot_pos=FAKE, out=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_combine(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(E=0), 1), (dict(k=3, E=2), 1), (dict(offsets=None), 1), (dict(x_sorted=None), 1),
+    (dict(ws_bytes=0), 3), (dict(Dm=4), 2),
+])
+def test_dispatch_rejects_bad_arguments(lib, kw, code):
+    a = dict(x=FAKE, dtype=1, T=300, Dm=64, E=8, k=1, topk_idx=FAKE, ws=FAKE, ws_bytes=1 << 20,
+             offsets=FAKE, sorted_slot=FAKE, slot_pos=FAKE, x_sorted=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_dispatch(*a.values()) == code
+
+
+def test_debug_wait_rejects_out_of_range_limits(lib):
+    assert lib.rom_debug_wait_timeout(10, None) == 1
+    assert lib.rom_debug_wait_timeout(10 ** 11, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from mixture_experts_projections_b200 import rom
+    with pytest.raises(rom.RomError):
+        old = rom._lib
+        rom._lib = None
+        try:
+            rom.load_library(str(tmp_path / "missing.so"))
+        finally:
+            rom._lib = old

@@ -1,0 +1,101 @@
+"""GPU parity of the whole RoM block forward and of the Swimba in-projection
+against the float64 oracle, on sizes that span several tiles with ragged
+tails, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_projections_b200 import rom
+from mixture_experts_projections_b200.inputs import (WORKLOADS, make_block_inputs,
+                                                     make_inproj_inputs, make_workload_inputs)
+from oracle import rom_oracle as orc
+from parity_util import (assert_close, assert_routing_matches, block_to_dev, to_dev, to_np,
+                         weights_to_dev)
+
+pytestmark = pytest.mark.gpu
+
+BLOCK_CASES = [
+    # T, Dm, De, E, k, renorm, dtype, router_std, bias
+    (1000, 256, 384, 8, 1, False, "bf16", 0.02, None),
+    (700, 512, 256, 4, 1, False, "bf16", 0.05, {0: 1.0}),
+    (600, 256, 256, 16, 2, True, "bf16", 0.05, None),
+    (300, 128, 128, 8, 2, False, "bf16", 0.1, None),
+    (333, 256, 128, 6, 3, True, "bf16", 0.1, None),
+    (200, 256, 256, 1, 1, False, "bf16", 0.02, None),
+    (517, 64, 128, 8, 1, False, "f32", 0.05, None),
+    (300, 96, 72, 5, 2, True, "f32", 0.2, None),
+    (150, 512, 512, 8, 1, False, "bf16", 0.02, {3: -40.0, 5: -40.0}),  # two empty experts
+]
+
+
+def oracle_block(inp, k, renorm):
+    return orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                             k=k, bias=inp["bias"], renorm=renorm)
+
+
+@pytest.mark.parametrize("T,Dm,De,E,k,renorm,dtype,std,bias", BLOCK_CASES)
+def test_block_forward_matches_oracle(T, Dm, De, E, k, renorm, dtype, std, bias):
+    b = None
+    if bias is not None:
+        b = np.zeros(E, np.float32)
+        for e, v in bias.items():
+            b[e] = v
+    inp = make_block_inputs(T, Dm, De, E, seed=T + De, dtype=dtype, router_std=std, bias=b)
+    ref = oracle_block(inp, k, renorm)
+    d = block_to_dev(inp, dtype)
+    out = rom.block_forward(d["x"], d["w_r"], d["bias"], d["w_conv"], d["w_gate"], d["w_out"],
+                            k=k, renorm=renorm)
+    torch.cuda.synchronize()
+    assert rom.rom_get_status() == 0
+    rb = out.routing
+    assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
+                           ref)
+    assert_close(to_np(out.out), ref["O"], dtype, "O")
+    if k == 1:
+        # the intermediate h in sorted order matches Y (.) G of the oracle
+        R = T
+        srt = rb.sorted_slot.cpu().numpy()[:R]
+        assert_close(to_np(out.h_sorted[:R]), ref["YG"][srt], dtype, "h")
+
+
+def test_tiny_fp32_workload():
+    wl = WORKLOADS["tiny_fp32"]
+    inp = make_workload_inputs(wl)
+    ref = oracle_block(inp, wl.k, wl.renorm)
+    d = block_to_dev(inp, "f32")
+    out = rom.block_forward(d["x"], d["w_r"], d["bias"], d["w_conv"], d["w_gate"], d["w_out"],
+                            k=wl.k)
+    assert_routing_matches(out.routing.topk_idx.cpu().numpy(),
+                           out.routing.topk_w.cpu().numpy().astype(np.float64), ref)
+    assert_close(to_np(out.out), ref["O"], "f32", "O")
+
+
+def test_block_forward_is_deterministic_and_repeatable():
+    inp = make_block_inputs(900, 256, 256, 8, seed=2, router_std=0.05)
+    d = block_to_dev(inp, "bf16")
+    args = (d["x"], d["w_r"], None, d["w_conv"], d["w_gate"], d["w_out"])
+    a = rom.block_forward(*args, k=2, renorm=True).out.clone()
+    bufs = rom.BlockBuffers(900, 256, 256, 8, 2, torch.bfloat16, "cuda")
+    for _ in range(3):
+        b = rom.block_forward(*args, k=2, renorm=True, bufs=bufs).out
+        assert torch.equal(a, b)
+
+
+INPROJ_CASES = [
+    # T, Dm, N, E, k, renorm
+    (64, 512, 1280, 4, 1, False),
+    (200, 256, 768, 4, 2, True),
+    (37, 1024, 512, 8, 1, False),
+]
+
+
+@pytest.mark.parametrize("T,Dm,N,E,k,renorm", INPROJ_CASES)
+def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
+    inp = make_inproj_inputs(T, Dm, N, E, seed=T + N, router_std=0.05)
+    ref = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=k, renorm=renorm)
+    out, rb = rom.inproj_forward(to_dev(inp["x"], "bf16"), to_dev(inp["w_r"], "f32"),
+                                 weights_to_dev(inp["w"], "bf16"), k=k, renorm=renorm)
+    torch.cuda.synchronize()
+    assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
+                           ref)
+    assert_close(to_np(out), ref["S"], "bf16", "S")
