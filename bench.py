@@ -371,6 +371,7 @@ def main():
                 times.append(dt)
         t = float(np.sum(times))
         val = len(toks) * args.steps / t
+        config["l2"] = "n/a (host CPU run)"
         line = {"impl": "reference", "metric": metric, "value": val, "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,

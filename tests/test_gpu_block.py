@@ -50,12 +50,12 @@ def test_block_forward_matches_oracle(T, Dm, De, E, k, renorm, dtype, std, bias)
     rb = out.routing
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
                            ref)
-    assert_close(to_np(out.out), ref["O"], dtype, "O")
+    assert_close(to_np(out.out), ref["O"], dtype, "O", magnitude_scaled_abs=True)
     if k == 1:
         # the intermediate h in sorted order matches Y (.) G of the oracle
         R = T
         srt = rb.sorted_slot.cpu().numpy()[:R]
-        assert_close(to_np(out.h_sorted[:R]), ref["YG"][srt], dtype, "h")
+        assert_close(to_np(out.h_sorted[:R]), ref["YG"][srt], dtype, "h", magnitude_scaled_abs=True)
 
 
 def test_tiny_fp32_workload():
@@ -98,4 +98,4 @@ def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
     torch.cuda.synchronize()
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
                            ref)
-    assert_close(to_np(out), ref["S"], "bf16", "S")
+    assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
