@@ -200,112 +200,116 @@ def run_ours(args, rank, world, local_rank):
         bufs = rom.BlockBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
     del inp["x"]
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=x.device)
-    ev = {}
-
-    def mark(name):
-        if name not in ev:
-            ev[name] = []
-        e = torch.cuda.Event(enable_timing=True)
-        e.record(stream)
-        ev[name].append(e)
-
     R = wl.T * wl.k
+    dt = rom.ROM_BF16 if bf16 else rom.ROM_F32
 
-    def step(record):
-        if wl.kind == "inproj":
-            if record:
-                mark("s")
+    # The step as three phases: route + dispatch, the dominant projection
+    # (Conv+Gate, or the in-projection), and the rest.
+    if wl.kind == "inproj":
+        def ph_route():
             rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, bufs)
-            if record:
-                mark("p0")
-            if wl.k == 1:
-                rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
-                                    bufs.offsets, bufs.sorted_slot, bufs.topk_w, out)
-            else:
-                rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
-                                    bufs.offsets, bufs.sorted_slot, bufs.topk_w, slots)
-            if record:
-                mark("p1")
-            if wl.k > 1:
-                rom.rom_combine(rom.ROM_COMBINE_SUM, rom.ROM_BF16, slots, wl.T, wl.k, wl.De, None,
-                                out)
-            if record:
-                mark("e")
-            return out
-        rb = bufs.routing
-        if record:
-            mark("s")
-        rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, rb)
-        if record:
-            mark("p0")
-        dt = rom.ROM_BF16 if bf16 else rom.ROM_F32
-        xs = rb.x_sorted[:R]
-        if wl.k == 1:
-            rom.rom_expert_proj(rom.ROM_PROJ_CONV_GATE, xs, ws["w_conv"], ws["w_gate"], wl.E, 1,
-                                rb.offsets, rb.sorted_slot, rb.topk_w, bufs.h_sorted)
-            if record:
-                mark("p1")
-            rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None, wl.E, 1,
-                                rb.offsets, rb.sorted_slot, rb.topk_w, bufs.out)
-            if record:
-                mark("p2")
-        else:
-            rom.rom_expert_proj(rom.ROM_PROJ_CONV_GATE, xs, ws["w_conv"], ws["w_gate"], wl.E,
-                                wl.k, rb.offsets, rb.sorted_slot, rb.topk_w, bufs.uz)
-            if record:
-                mark("p1")
-            rom.rom_combine(rom.ROM_COMBINE_GATE, dt, bufs.uz, wl.T, wl.k, wl.De, rb.slot_pos,
-                            bufs.h_sorted)
-            rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None, wl.E,
-                                wl.k, rb.offsets, rb.sorted_slot, rb.topk_w, bufs.o_slots)
-            if record:
-                mark("p2")
-            rom.rom_combine(rom.ROM_COMBINE_SUM, dt, bufs.o_slots, wl.T, wl.k, wl.Dm, None,
-                            bufs.out)
-        if record:
-            mark("e")
-        return bufs.out
 
-    launches_per_step = (3 if wl.kind == "inproj" else 4) + (2 if wl.k > 1 else 0)
-    if wl.kind == "inproj" and wl.k > 1:
-        launches_per_step = 4
+        def ph_p0():
+            rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
+                                bufs.offsets, bufs.sorted_slot, bufs.topk_w,
+                                out if wl.k == 1 else slots)
+
+        def ph_p1():
+            if wl.k > 1:
+                rom.rom_combine(rom.ROM_COMBINE_SUM, dt, slots, wl.T, wl.k, wl.De, None, out)
+        out_t = out
+        counts_t = bufs.counts
+    else:
+        rb = bufs.routing
+
+        def ph_route():
+            rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, rb)
+
+        def ph_p0():
+            rom.rom_expert_proj(rom.ROM_PROJ_CONV_GATE, rb.x_sorted[:R], ws["w_conv"],
+                                ws["w_gate"], wl.E, wl.k, rb.offsets, rb.sorted_slot, rb.topk_w,
+                                bufs.h_sorted if wl.k == 1 else bufs.uz)
+
+        def ph_p1():
+            if wl.k == 1:
+                rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None, wl.E,
+                                    1, rb.offsets, rb.sorted_slot, rb.topk_w, bufs.out)
+            else:
+                rom.rom_combine(rom.ROM_COMBINE_GATE, dt, bufs.uz, wl.T, wl.k, wl.De,
+                                rb.slot_pos, bufs.h_sorted)
+                rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None,
+                                    wl.E, wl.k, rb.offsets, rb.sorted_slot, rb.topk_w,
+                                    bufs.o_slots)
+                rom.rom_combine(rom.ROM_COMBINE_SUM, dt, bufs.o_slots, wl.T, wl.k, wl.Dm, None,
+                                bufs.out)
+        out_t = bufs.out
+        counts_t = rb.counts
+    phases = [ph_route, ph_p0, ph_p1]
+
+    def step():
+        for ph in phases:
+            ph()
+        return out_t
+
+    # our kernels per step: router + dispatch (+ the memset of counts, not ours),
+    # the projection(s) and, for top-k > 1, the combines
+    if wl.kind == "inproj":
+        launches_per_step = 3 + (1 if wl.k > 1 else 0)
+    else:
+        launches_per_step = 4 + (2 if wl.k > 1 else 0)
 
     for _ in range(args.warmup):
         flush.zero_()
-        step(False)
+        step()
     torch.cuda.synchronize()
     if rom.rom_get_status() != 0:
         raise RuntimeError("device status word reports an error after warm-up")
 
+    # Each phase captured once as a CUDA graph (the launch sequence of the
+    # library is static: its kernels read the expert counts on the device).
+    graphs = []
+    for ph in phases:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            ph()
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    def timed_loop(run_phase, n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)]
+               for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            torch.cuda._sleep(200_000)  # GPU-side head start so that the host stays ahead
+            evs[i][0].record(stream)
+            for j in range(len(phases)):
+                run_phase(j)
+                evs[i][j + 1].record(stream)
+        torch.cuda.synchronize()
+        return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(phases))]
+                         for i in range(n)])
+
+    for _ in range(2):  # graph warm-up
+        timed_loop(lambda j: graphs[j].replay(), 1)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    for _ in range(args.steps):
-        flush.zero_()
-        step(True)
-    torch.cuda.synchronize()
+    ph_ms = timed_loop(lambda j: graphs[j].replay(), args.steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-
-    def span(a, b):
-        return [s.elapsed_time(e) for s, e in zip(ev[a], ev[b])]
-
-    step_ms = span("s", "e")
-    t_total_ms = float(np.sum(step_ms))
-    parts = {"route_dispatch": span("s", "p0"), "proj0": span("p0", "p1")}
-    if wl.kind != "inproj":
-        parts["proj1"] = span("p1", "p2")
-    part_ms = {n: float(np.mean(v)) for n, v in parts.items()}
+    eager_ms = timed_loop(lambda j: phases[j](), args.steps)
+    t_total_ms = float(ph_ms.sum())
+    part_names = ["route_dispatch", "proj0", "proj1"]
+    part_ms = {n: float(ph_ms[:, j].mean()) for j, n in enumerate(part_names)}
 
     # ---------------------------------------------- e2e through host buffers
     h_x = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     h_x.copy_(x)
-    out_t = out if wl.kind == "inproj" else bufs.out
     h_out = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
     e2e_ms = []
     for i in range(args.warmup + args.steps):
@@ -314,22 +318,23 @@ def run_ours(args, rank, world, local_rank):
         s1 = torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         x.copy_(h_x, non_blocking=True)
-        o = step(False)
+        o = step()
         h_out.copy_(o, non_blocking=True)
         s1.record(stream)
         s1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(s0.elapsed_time(s1))
     e2e_total = float(np.sum(e2e_ms))
+    del graphs
 
     stats = torch.tensor([t_total_ms, e2e_total], dtype=torch.float64, device=x.device)
     if world > 1:
         dist.all_reduce(stats, op=dist.ReduceOp.MAX)
     t_total_ms, e2e_total = float(stats[0]), float(stats[1])
     res = dict(wl=wl, step_ms=t_total_ms / args.steps, part_ms=part_ms,
+               eager_ms=float(eager_ms.sum()) / args.steps,
                e2e_ms=e2e_total / args.steps, clocks=clk, launches=launches_per_step * args.steps,
-               counts=bufs.counts.cpu().numpy() if wl.kind == "inproj" else
-               bufs.routing.counts.cpu().numpy(), x_bytes=x.numel() * x.element_size(),
+               counts=counts_t.cpu().numpy(), x_bytes=x.numel() * x.element_size(),
                out_bytes=out_t.numel() * out_t.element_size())
     return res
 
@@ -421,7 +426,9 @@ def main():
                 "config": config, "roofline": roof,
                 "block_tflops": tot_flops / step_s / 1e12,
                 "block_frac_of_bf16_peak": tot_flops / step_s / 1e12 / peaks["bf16_tflops"],
-                "kernels_ms": res["part_ms"],
+                "kernels_ms": res["part_ms"], "eager_ms_per_step": res["eager_ms"],
+                "timing": "each phase replayed as a CUDA graph; CUDA events on the launching "
+                          "stream between phases",
                 "e2e": {"value": wl.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": res["x_bytes"], "d2h_bytes_per_step": res["out_bytes"]},
                 "gpu_launches": res["launches"], "clocks": res["clocks"],

@@ -3,18 +3,25 @@
 // ("Routing Mamba ..." chapterpal summary page, Knowl 1: p_t = Softmax(x_t W_r),
 // S_t = the K largest probabilities, r_{t,i} = p_{t,i} 1[i in S_t].)
 //
-// Work split: a CTA of 8 warps owns a chunk of 128 tokens; a warp handles
-// TPW tokens at a time, its 32 lanes splitting d_model into 16-byte slices.
-// Each lane accumulates its slice sequentially in float32 FMA, then a 5-level
-// xor butterfly sums the lanes (every lane ends with the identical sum).
-// The same pass accumulates |x|^2, which with the per-expert |w_e| gives the
-// Cauchy-Schwarz bound sum_i |x_i w_ie| <= |x| |w_e| and hence a rigorous
-// bound gamma_n |x| |w_e| on the rounding error of each float32 logit
-// (n = the longest accumulation chain, gamma_n = n u / (1 - n u)).
-// If a gap that decides S_t or its slot order is not larger than the two
-// bounds, the warp recomputes that token's logits in float64 before deciding.
-// The routing decision is therefore the one exact arithmetic would take,
-// except for gaps below the float64 rounding level.
+// Work split. A CTA of 16 warps owns a chunk of 128 tokens. A warp takes TPW
+// tokens per pass and holds NV = TPW * EB partial logits per lane (EB = the
+// expert count rounded up to a power of two); its 32 lanes split d_model so
+// that every shared-memory read of the router weight is conflict-free.
+// Each lane accumulates its slice sequentially in float32 FMA; a
+// transpose-reduce (31 shuffles per 32 values) then leaves lane L holding the
+// complete logit of (token, expert) = divmod(i * 32 + L, EB) for each of its
+// NV / 32 values. Top-k selection, softmax and the outputs are computed
+// lane-parallel over segments of EB lanes with shuffles.
+//
+// Exactness of the decision. The same pass accumulates |x|^2; with the
+// per-expert |w_e| this bounds sum_i |x_i w_ie| <= |x| |w_e| (Cauchy-Schwarz),
+// hence the float32 rounding error of each logit by gamma_n |x| |w_e| (+ the
+// bias add), n being the longest accumulation chain and
+// gamma_n = n u / (1 - n u). If a gap that decides S_t or its slot order is
+// not larger than the two bounds, the warp recomputes that token's logits in
+// float64 and decides on those. The selection is then the one exact
+// arithmetic would make, except for gaps below the float64 rounding level.
+// Equal logits go to the lower expert index.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -25,31 +32,40 @@
 namespace rom {
 namespace {
 
-constexpr int kRouterThreads = 256;
+constexpr int kRouterThreads = 512;
 constexpr int kRouterWarps = kRouterThreads / 32;
 
 template <typename InT>
-struct Vec;
+struct Elem;
 template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int V = 8;
+struct Elem<__nv_bfloat16> {
+  static constexpr int V = 8;        // elements per lane per step (two groups of 4)
+  static constexpr int STEP = 256;   // elements per warp per step
 };
 template <>
-struct Vec<float> {
-  static constexpr int V = 4;
+struct Elem<float> {
+  static constexpr int V = 4;        // one group of 4
+  static constexpr int STEP = 128;
 };
 
-// 16 bytes of x (8 bf16 or 4 float) -> float.
-__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&f)[8]) {
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+template <int EB>
+struct Geo {
+  static constexpr int NV = EB <= 8 ? 32 : 64;     // partial logits per lane
+  static constexpr int TPW = NV / EB;              // tokens per warp per pass
+  static constexpr int VPL = NV / 32;              // complete logits per lane
+  static constexpr int W = EB < 32 ? EB : 32;      // lanes per token segment
+  static constexpr int VPT = EB > 32 ? EB / 32 : 1;  // logits per lane per token
+};
+
+// 4 consecutive elements of x -> float.
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float* f) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+  f[0] = __uint_as_float(v.x << 16);
+  f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(v.y << 16);
+  f[3] = __uint_as_float(v.y & 0xFFFF0000u);
 }
-__device__ __forceinline__ void load16(const float* p, float (&f)[4]) {
+__device__ __forceinline__ void load4(const float* p, float* f) {
   const float4 v = __ldg(reinterpret_cast<const float4*>(p));
   f[0] = v.x;
   f[1] = v.y;
@@ -57,70 +73,103 @@ __device__ __forceinline__ void load16(const float* p, float (&f)[4]) {
   f[3] = v.w;
 }
 
-// W_r value of expert e at feature d: from the transposed shared copy
-// [EB][Dm] or from the global [Dm][E] array.
-template <bool SMEM_W>
-__device__ __forceinline__ float wval(const float* sW, const float* w_r, int Dm, int E, int e,
-                                      int d) {
-  return SMEM_W ? sW[e * Dm + d] : __ldg(w_r + static_cast<int64_t>(d) * E + e);
+// Element offset (within a step) of the lane's group g of 4 elements.
+template <typename InT>
+__device__ __forceinline__ int group_off(int g, int lane) {
+  return g * 128 + 4 * lane;
 }
 
-// Top-(k+1) scan over EB values: slot j gets the j-th largest (equal values:
-// lower index first); idx[k] is the best unselected expert (or -1).
-template <int EB, typename VT>
-__device__ __forceinline__ void select_topk(const VT (&l)[EB], int E, int k,
-                                            int (&idx)[kMaxTopK + 1]) {
-  uint64_t used = 0;
+// Argmax over the W lanes of each aligned segment: larger value wins, equal
+// values go to the lower expert index. Every lane of the segment receives
+// the winner.
+template <int W, typename VT>
+__device__ __forceinline__ void seg_argmax(VT& v, int& e) {
 #pragma unroll
-  for (int j = 0; j <= kMaxTopK; ++j) {
-    idx[j] = -1;
-    if (j <= k) {
-      int bi = -1;
-      VT bv = 0;
-#pragma unroll
-      for (int e = 0; e < EB; ++e) {
-        if (e < E && !((used >> e) & 1ull) && (bi < 0 || l[e] > bv)) {
-          bi = e;
-          bv = l[e];
-        }
-      }
-      idx[j] = bi;
-      if (bi >= 0) used |= 1ull << bi;
+  for (int o = W / 2; o > 0; o >>= 1) {
+    const VT ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oe = __shfl_xor_sync(0xffffffffu, e, o);
+    if (ov > v || (ov == v && oe < e)) {
+      v = ov;
+      e = oe;
     }
   }
 }
 
-template <int EB>
-__device__ __forceinline__ float pick(const float (&a)[EB], int e) {
-  float r = 0.f;
+template <int W>
+__device__ __forceinline__ float seg_sum(float v) {
 #pragma unroll
-  for (int i = 0; i < EB; ++i) r = (i == e) ? a[i] : r;
-  return r;
+  for (int o = W / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
-// float64 logits of one token, computed by the whole warp; written to out[0..E).
-template <typename InT, int EB, bool SMEM_W>
+// Selection for one token segment. Each lane holds VPT candidate logits
+// `lv` of experts `le` (le >= E: padding, value -inf). Produces, uniform
+// over the segment, the experts sel[0..k] (sel[k] = the best unselected one,
+// or -1) and their logits selv[]; `slot[v]` = slot of the lane's own
+// candidate v (or -1).
+template <int W, int VPT, typename VT>
+__device__ __forceinline__ void seg_select(const VT (&lv)[VPT], const int (&le)[VPT], int E, int k,
+                                           int (&sel)[kMaxTopK + 1], VT (&selv)[kMaxTopK + 1],
+                                           int (&slot)[VPT]) {
+  bool used[VPT];
+#pragma unroll
+  for (int v = 0; v < VPT; ++v) {
+    used[v] = false;
+    slot[v] = -1;
+  }
+#pragma unroll
+  for (int j = 0; j <= kMaxTopK; ++j) {
+    sel[j] = -1;
+    selv[j] = -INFINITY;
+    if (j <= k) {
+      VT cv = -INFINITY;
+      int ce = 1 << 20;
+#pragma unroll
+      for (int v = 0; v < VPT; ++v) {
+        if (!used[v] && le[v] < E && (lv[v] > cv || (lv[v] == cv && le[v] < ce))) {
+          cv = lv[v];
+          ce = le[v];
+        }
+      }
+      seg_argmax<W, VT>(cv, ce);
+      if (ce < E) {
+        sel[j] = ce;
+        selv[j] = cv;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v)
+          if (le[v] == ce) {
+            used[v] = true;
+            if (j < k) slot[v] = j;
+          }
+      }
+    }
+  }
+}
+
+// float64 logits of one token, computed by the whole warp; lane 0 writes
+// out[0..E).
+template <typename InT, int EB>
 __device__ __noinline__ void refine_logits_f64(const InT* __restrict__ xrow, int Dm,
                                                const float* sW, const float* w_r,
-                                               const float* bias, int E, double* out,
-                                               int lane) {
-  constexpr int V = Vec<InT>::V;
+                                               const float* bias, int E, bool smem_w,
+                                               double* out, int lane) {
   constexpr int G = EB < 16 ? EB : 16;
   for (int e0 = 0; e0 < EB; e0 += G) {
     double a[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) a[g] = 0.0;
-    for (int d0 = lane * V; d0 < Dm; d0 += 32 * V) {
-      float xv[V];
-      load16(xrow + d0, xv);
+    for (int d = 4 * lane; d < Dm; d += 128) {
+      float xv[4];
+      load4(xrow + d, xv);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int e = e0 + g;
         if (e < E) {
 #pragma unroll
-          for (int v = 0; v < V; ++v)
-            a[g] = fma(static_cast<double>(xv[v]),
-                       static_cast<double>(wval<SMEM_W>(sW, w_r, Dm, E, e, d0 + v)), a[g]);
+          for (int j = 0; j < 4; ++j) {
+            const float w = smem_w ? sW[e * Dm + d + j] : __ldg(w_r + static_cast<int64_t>(d + j) * E + e);
+            a[g] = fma(static_cast<double>(xv[j]), static_cast<double>(w), a[g]);
+          }
         }
       }
     }
@@ -140,18 +189,28 @@ __device__ __noinline__ void refine_logits_f64(const InT* __restrict__ xrow, int
   __syncwarp();
 }
 
-template <typename InT, int EB, int TPW, bool SMEM_W>
+template <int N>
+__device__ __forceinline__ float pickf(const float (&a)[N], int i) {
+  float r = a[0];
+#pragma unroll
+  for (int q = 1; q < N; ++q) r = (q == i) ? a[q] : r;
+  return r;
+}
+
+template <typename InT, int EB, bool SMEM_W>
 __global__ void __launch_bounds__(kRouterThreads)
     router_kernel(const InT* __restrict__ x, int64_t T, int Dm, const float* __restrict__ w_r,
                   const float* __restrict__ bias, int E, int k, int renorm,
                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   int32_t* __restrict__ counts, int32_t* __restrict__ chunk_hist,
                   int64_t nchunks, float gamma) {
-  constexpr int V = Vec<InT>::V;
+  using G = Geo<EB>;
+  constexpr int NV = G::NV, TPW = G::TPW, VPL = G::VPL, W = G::W, VPT = G::VPT;
+  constexpr int V = Elem<InT>::V, STEP = Elem<InT>::STEP;
   constexpr int kPasses = kChunkTokens / (kRouterWarps * TPW);
   static_assert(kPasses * kRouterWarps * TPW == kChunkTokens, "chunk geometry");
   extern __shared__ float4 router_smem[];
-  float* sW = reinterpret_cast<float*>(router_smem);  // [EB][Dm] when SMEM_W
+  float* sW = reinterpret_cast<float*>(router_smem);  // [EB][Dm] + STEP pad, when SMEM_W
   __shared__ float s_wnorm[EB];
   __shared__ int s_hist[EB];
   __shared__ double s_l64[kRouterWarps][EB];
@@ -159,14 +218,14 @@ __global__ void __launch_bounds__(kRouterThreads)
 
   if (SMEM_W) {
     for (int i = tid; i < Dm * E; i += kRouterThreads) sW[(i % E) * Dm + i / E] = w_r[i];
-    for (int i = tid; i < Dm * (EB - E); i += kRouterThreads) sW[E * Dm + i] = 0.f;
+    for (int i = tid; i < Dm * (EB - E) + STEP; i += kRouterThreads) sW[E * Dm + i] = 0.f;
     __syncthreads();
   }
   for (int e = warp; e < EB; e += kRouterWarps) {
     float s = 0.f;
     if (e < E)
       for (int d = lane; d < Dm; d += 32) {
-        const float w = wval<SMEM_W>(sW, w_r, Dm, E, e, d);
+        const float w = SMEM_W ? sW[e * Dm + d] : __ldg(w_r + static_cast<int64_t>(d) * E + e);
         s = fmaf(w, w, s);
       }
 #pragma unroll
@@ -178,24 +237,28 @@ __global__ void __launch_bounds__(kRouterThreads)
     for (int e = tid; e < EB; e += kRouterThreads) s_hist[e] = 0;
     __syncthreads();
     for (int pass = 0; pass < kPasses; ++pass) {
-      const int64_t t0 = c * kChunkTokens + static_cast<int64_t>(pass * kRouterWarps + warp) * TPW;
-      float acc[TPW][EB];
+      const int64_t t0 =
+          c * kChunkTokens + static_cast<int64_t>(pass * kRouterWarps + warp) * TPW;
+      float acc[NV];
       float sq[TPW];
 #pragma unroll
-      for (int t = 0; t < TPW; ++t) {
-        sq[t] = 0.f;
+      for (int i = 0; i < NV; ++i) acc[i] = 0.f;
 #pragma unroll
-        for (int e = 0; e < EB; ++e) acc[t][e] = 0.f;
-      }
-      for (int d0 = lane * V; d0 < Dm; d0 += 32 * V) {
+      for (int t = 0; t < TPW; ++t) sq[t] = 0.f;
+
+      for (int d0 = 0; d0 < Dm; d0 += STEP) {
         float xv[TPW][V];
 #pragma unroll
         for (int t = 0; t < TPW; ++t) {
-          if (t0 + t < T) {
-            load16(x + (t0 + t) * static_cast<int64_t>(Dm) + d0, xv[t]);
-          } else {
 #pragma unroll
-            for (int v = 0; v < V; ++v) xv[t][v] = 0.f;
+          for (int g = 0; g < V / 4; ++g) {
+            const int d = d0 + group_off<InT>(g, lane);
+            if (t0 + t < T && d < Dm) {
+              load4(x + (t0 + t) * static_cast<int64_t>(Dm) + d, &xv[t][4 * g]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) xv[t][4 * g + j] = 0.f;
+            }
           }
 #pragma unroll
           for (int v = 0; v < V; ++v) sq[t] = fmaf(xv[t][v], xv[t][v], sq[t]);
@@ -203,95 +266,134 @@ __global__ void __launch_bounds__(kRouterThreads)
 #pragma unroll
         for (int e = 0; e < EB; ++e) {
           float wv[V];
-          if (SMEM_W) {
 #pragma unroll
-            for (int v4 = 0; v4 < V / 4; ++v4) {
-              const float4 q = *reinterpret_cast<const float4*>(sW + e * Dm + d0 + 4 * v4);
-              wv[4 * v4] = q.x;
-              wv[4 * v4 + 1] = q.y;
-              wv[4 * v4 + 2] = q.z;
-              wv[4 * v4 + 3] = q.w;
+          for (int g = 0; g < V / 4; ++g) {
+            const int d = d0 + group_off<InT>(g, lane);
+            if (SMEM_W) {
+              const float4 q = *reinterpret_cast<const float4*>(sW + e * Dm + d);
+              wv[4 * g] = q.x;
+              wv[4 * g + 1] = q.y;
+              wv[4 * g + 2] = q.z;
+              wv[4 * g + 3] = q.w;
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                wv[4 * g + j] = (e < E && d + j < Dm)
+                                    ? __ldg(w_r + static_cast<int64_t>(d + j) * E + e)
+                                    : 0.f;
             }
-          } else {
-#pragma unroll
-            for (int v = 0; v < V; ++v) wv[v] = (e < E) ? wval<false>(sW, w_r, Dm, E, e, d0 + v) : 0.f;
           }
 #pragma unroll
           for (int t = 0; t < TPW; ++t) {
 #pragma unroll
-            for (int v = 0; v < V; ++v) acc[t][e] = fmaf(xv[t][v], wv[v], acc[t][e]);
+            for (int v = 0; v < V; ++v) acc[t * EB + e] = fmaf(xv[t][v], wv[v], acc[t * EB + e]);
           }
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < TPW; ++t) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          sq[t] += __shfl_xor_sync(0xffffffffu, sq[t], off);
-#pragma unroll
-          for (int e = 0; e < EB; ++e) acc[t][e] += __shfl_xor_sync(0xffffffffu, acc[t][e], off);
         }
       }
 
-      // Decisions: warp-uniform, one token at a time.
+      // |x|^2 of every token of the pass, on every lane.
 #pragma unroll
       for (int t = 0; t < TPW; ++t) {
-        const int64_t tok = t0 + t;
-        if (tok >= T) continue;
-        float l[EB], err[EB];
-        const float xn = sqrtf(sq[t]);
 #pragma unroll
-        for (int e = 0; e < EB; ++e) {
-          if (e < E) {
-            l[e] = acc[t][e] + (bias ? __ldg(bias + e) : 0.f);
-            err[e] = gamma * xn * s_wnorm[e] + 1.2e-7f * fabsf(l[e]);
-          } else {
-            l[e] = -INFINITY;
-            err[e] = 0.f;
+        for (int off = 16; off > 0; off >>= 1) sq[t] += __shfl_xor_sync(0xffffffffu, sq[t], off);
+      }
+      // Transpose-reduce: lane L ends with the sum of flat index i*32 + L.
+#pragma unroll
+      for (int blk = 0; blk < VPL; ++blk) {
+        float* a = acc + blk * 32;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const bool up = (lane & o) != 0;
+#pragma unroll
+          for (int j = 0; j < o; ++j) {
+            const float send = up ? a[j] : a[j + o];
+            const float keep = up ? a[j + o] : a[j];
+            a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
           }
         }
+      }
+
+      // Lane-parallel decisions: a token occupies W lanes x VPT values.
+      constexpr int NSEG = VPL / VPT;  // token groups per lane
+#pragma unroll
+      for (int sg = 0; sg < NSEG; ++sg) {
+        float lv[VPT];
+        int le[VPT];
+        int tl = 0;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) {
+          const int f = (sg * VPT + v) * 32 + lane;  // flat index of acc[sg*VPT+v]'s block
+          tl = f / EB;
+          le[v] = f % EB;
+          const float b = (bias && le[v] < E) ? __ldg(bias + le[v]) : 0.f;
+          lv[v] = (le[v] < E) ? acc[(sg * VPT + v) * 32] + b : -INFINITY;
+        }
+        const int64_t tok = t0 + tl;
+        const bool tok_ok = tok < T;
+        const float xn = sqrtf(pickf<TPW>(sq, tl));
         int sel[kMaxTopK + 1];
-        select_topk<EB, float>(l, E, k, sel);
+        float selv[kMaxTopK + 1];
+        int slot[VPT];
+        seg_select<W, VPT, float>(lv, le, E, k, sel, selv, slot);
         bool certain = true;
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) {
           if (j < k && sel[j + 1] >= 0) {
-            const int a = sel[j], b = sel[j + 1];
-            if (!(pick<EB>(l, a) - pick<EB>(l, b) > pick<EB>(err, a) + pick<EB>(err, b)))
-              certain = false;
+            const float ea = gamma * xn * s_wnorm[sel[j]] + 1.2e-7f * fabsf(selv[j]);
+            const float eb = gamma * xn * s_wnorm[sel[j + 1]] + 1.2e-7f * fabsf(selv[j + 1]);
+            if (!(selv[j] - selv[j + 1] > ea + eb)) certain = false;
           }
         }
-        if (!certain) {
-          refine_logits_f64<InT, EB, SMEM_W>(x + tok * static_cast<int64_t>(Dm), Dm, sW, w_r,
-                                             bias, E, s_l64[warp], lane);
-          double l64[EB];
+        // Tokens whose float32 decision is not certain: float64 logits.
+        unsigned todo = __ballot_sync(0xffffffffu, tok_ok && !certain);
+        while (todo) {
+          const int src = __ffs(todo) - 1;
+          const int tl_r = __shfl_sync(0xffffffffu, tl, src);
+          todo &= ~(((W == 32) ? 0xffffffffu : ((1u << W) - 1u)) << (src & ~(W - 1)));
+          refine_logits_f64<InT, EB>(x + (t0 + tl_r) * static_cast<int64_t>(Dm), Dm, sW, w_r,
+                                     bias, E, SMEM_W, s_l64[warp], lane);
+          double lv64[VPT];
 #pragma unroll
-          for (int e = 0; e < EB; ++e) l64[e] = (e < E) ? s_l64[warp][e] : -INFINITY;
-          select_topk<EB, double>(l64, E, k, sel);
+          for (int v = 0; v < VPT; ++v)
+            lv64[v] = (le[v] < E) ? s_l64[warp][le[v] < E ? le[v] : 0] : -INFINITY;
+          int sel2[kMaxTopK + 1];
+          double selv2[kMaxTopK + 1];
+          int slot2[VPT];
+          seg_select<W, VPT, double>(lv64, le, E, k, sel2, selv2, slot2);
+          if (tl == tl_r) {
 #pragma unroll
-          for (int e = 0; e < EB; ++e) l[e] = (e < E) ? static_cast<float>(l64[e]) : -INFINITY;
+            for (int j = 0; j <= kMaxTopK; ++j) {
+              sel[j] = sel2[j];
+              selv[j] = static_cast<float>(selv2[j]);
+            }
+#pragma unroll
+            for (int v = 0; v < VPT; ++v) {
+              slot[v] = slot2[v];
+              lv[v] = static_cast<float>(lv64[v]);
+            }
+          }
           __syncwarp();
         }
-        // Softmax in float32 (exp of the shifted logits).
-        const float m = pick<EB>(l, sel[0]);
+        // Softmax (float32) and outputs.
+        const float m = selv[0];
         float den = 0.f;
         if (renorm) {
 #pragma unroll
           for (int j = 0; j < kMaxTopK; ++j)
-            if (j < k) den += expf(pick<EB>(l, sel[j]) - m);
+            if (j < k) den += expf(selv[j] - m);
         } else {
+          float part = 0.f;
 #pragma unroll
-          for (int e = 0; e < EB; ++e)
-            if (e < E) den += expf(l[e] - m);
+          for (int v = 0; v < VPT; ++v)
+            if (le[v] < E) part += expf(lv[v] - m);
+          den = seg_sum<W>(part);
         }
-        if (lane == 0) {
 #pragma unroll
-          for (int j = 0; j < kMaxTopK; ++j) {
-            if (j < k) {
-              topk_idx[tok * k + j] = sel[j];
-              topk_w[tok * k + j] = expf(pick<EB>(l, sel[j]) - m) / den;
-              atomicAdd(&s_hist[sel[j]], 1);
-            }
+        for (int v = 0; v < VPT; ++v) {
+          if (tok_ok && slot[v] >= 0) {
+            topk_idx[tok * k + slot[v]] = le[v];
+            topk_w[tok * k + slot[v]] = expf(lv[v] - m) / den;
+            atomicAdd(&s_hist[le[v]], 1);
           }
         }
       }
@@ -305,22 +407,23 @@ __global__ void __launch_bounds__(kRouterThreads)
   }
 }
 
-template <typename InT, int EB, int TPW>
+template <typename InT, int EB>
 cudaError_t launch_eb(const InT* x, int64_t T, int Dm, const float* w_r, const float* bias,
                       int E, int k, int renorm, int32_t* topk_idx, float* topk_w,
                       int32_t* counts, int32_t* chunk_hist, cudaStream_t stream) {
-  constexpr int V = Vec<InT>::V;
+  constexpr int V = Elem<InT>::V, STEP = Elem<InT>::STEP;
   const int64_t nchunks = num_chunks(T);
   if (nchunks == 0) return cudaSuccess;
   // Longest float32 accumulation chain: the lane's sequential slice, the
-  // 5-level butterfly and the bias add (+1 spare); 1 % slack for the norms.
-  const double n = static_cast<double>(((Dm + 32 * V - 1) / (32 * V)) * V + 5 + 2);
+  // 5-level reduction tree and the bias add (+1 spare); 1 % slack covers the
+  // rounding of the two norms.
+  const double n = static_cast<double>(((Dm + STEP - 1) / STEP) * V + 5 + 2);
   const double u = 1.0 / 16777216.0;
   const float gamma = static_cast<float>(1.01 * n * u / (1.0 - n * u));
-  const size_t smem_w = static_cast<size_t>(EB) * Dm * sizeof(float);
+  const size_t smem_w = (static_cast<size_t>(EB) * Dm + STEP) * sizeof(float);
   const int sms = device_sm_count();
   if (smem_w <= 160 * 1024) {
-    auto kern = router_kernel<InT, EB, TPW, true>;
+    auto kern = router_kernel<InT, EB, true>;
     cudaError_t err =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
     if (err != cudaSuccess) return err;
@@ -331,8 +434,8 @@ cudaError_t launch_eb(const InT* x, int64_t T, int Dm, const float* w_r, const f
     kern<<<static_cast<unsigned>(grid), kRouterThreads, smem_w, stream>>>(
         x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist, nchunks, gamma);
   } else {
-    auto kern = router_kernel<InT, EB, TPW, false>;
-    const int64_t grid = std::min<int64_t>(nchunks, static_cast<int64_t>(sms) * 4);
+    auto kern = router_kernel<InT, EB, false>;
+    const int64_t grid = std::min<int64_t>(nchunks, static_cast<int64_t>(sms) * 2);
     kern<<<static_cast<unsigned>(grid), kRouterThreads, 0, stream>>>(
         x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist, nchunks, gamma);
   }
@@ -343,20 +446,17 @@ template <typename InT>
 cudaError_t launch_typed(const InT* x, int64_t T, int Dm, const float* w_r, const float* bias,
                          int E, int k, int renorm, int32_t* topk_idx, float* topk_w,
                          int32_t* counts, int32_t* chunk_hist, cudaStream_t stream) {
-  if (E <= 4)
-    return launch_eb<InT, 4, 4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts,
-                                chunk_hist, stream);
-  if (E <= 8)
-    return launch_eb<InT, 8, 4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts,
-                                chunk_hist, stream);
-  if (E <= 16)
-    return launch_eb<InT, 16, 4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts,
-                                 chunk_hist, stream);
-  if (E <= 32)
-    return launch_eb<InT, 32, 2>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts,
-                                 chunk_hist, stream);
-  return launch_eb<InT, 64, 1>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts,
+#define ROM_ROUTER_CASE(EBV)                                                                 \
+  if (E <= EBV)                                                                              \
+    return launch_eb<InT, EBV>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, \
                                chunk_hist, stream);
+  ROM_ROUTER_CASE(4)
+  ROM_ROUTER_CASE(8)
+  ROM_ROUTER_CASE(16)
+  ROM_ROUTER_CASE(32)
+  ROM_ROUTER_CASE(64)
+#undef ROM_ROUTER_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
