@@ -149,7 +149,7 @@ __device__ __forceinline__ void seg_select(const VT (&lv)[VPT], const int (&le)[
 // float64 logits of one token, computed by the whole warp; lane 0 writes
 // out[0..E).
 template <typename InT, int EB>
-__device__ __noinline__ void refine_logits_f64(const InT* __restrict__ xrow, int Dm,
+__device__ __noinline__ void refine_logits_f64(const InT* __restrict__ xrow, int Dm, int DS,
                                                const float* sW, const float* w_r,
                                                const float* bias, int E, bool smem_w,
                                                double* out, int lane) {
@@ -167,7 +167,7 @@ __device__ __noinline__ void refine_logits_f64(const InT* __restrict__ xrow, int
         if (e < E) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const float w = smem_w ? sW[e * Dm + d + j] : __ldg(w_r + static_cast<int64_t>(d + j) * E + e);
+            const float w = smem_w ? sW[e * DS + d + j] : __ldg(w_r + static_cast<int64_t>(d + j) * E + e);
             a[g] = fma(static_cast<double>(xv[j]), static_cast<double>(w), a[g]);
           }
         }
@@ -197,40 +197,53 @@ __device__ __forceinline__ float pickf(const float (&a)[N], int i) {
   return r;
 }
 
-template <typename InT, int EB, bool SMEM_W>
+// Loads W_r^T[e][D0 .. D0+DS) into sW[e][0 .. DS) (zero beyond Dm and for
+// padding experts e >= E). The global reads walk w_r in memory order.
+__device__ __forceinline__ void load_w_slice(float* sW, const float* __restrict__ w_r, int Dm,
+                                             int E, int EB, int D0, int DS, int tid) {
+  const int dn = min(DS, Dm - D0);  // features of this slice that exist
+  const float* src = w_r + static_cast<int64_t>(D0) * E;
+  for (int i = tid; i < dn * E; i += kRouterThreads) {
+    const int d = i / E, e = i - d * E;
+    sW[e * DS + d] = __ldg(src + i);
+  }
+  for (int i = tid; i < DS * EB; i += kRouterThreads) {
+    const int e = i / DS, d = i - e * DS;
+    if (e >= E || d >= dn) sW[i] = 0.f;
+  }
+}
+
+template <typename InT, int EB>
 __global__ void __launch_bounds__(kRouterThreads)
     router_kernel(const InT* __restrict__ x, int64_t T, int Dm, const float* __restrict__ w_r,
                   const float* __restrict__ bias, int E, int k, int renorm,
                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                   int32_t* __restrict__ counts, int32_t* __restrict__ chunk_hist,
-                  int64_t nchunks, float gamma) {
+                  int64_t nchunks, float gamma, int DS) {
   using G = Geo<EB>;
   constexpr int NV = G::NV, TPW = G::TPW, VPL = G::VPL, W = G::W, VPT = G::VPT;
   constexpr int V = Elem<InT>::V, STEP = Elem<InT>::STEP;
   constexpr int kPasses = kChunkTokens / (kRouterWarps * TPW);
   static_assert(kPasses * kRouterWarps * TPW == kChunkTokens, "chunk geometry");
   extern __shared__ float4 router_smem[];
-  float* sW = reinterpret_cast<float*>(router_smem);  // [EB][Dm] + STEP pad, when SMEM_W
+  // W_r^T slice [EB][DS] (+ STEP zero pad): the whole of d_model when it fits
+  // (loaded once per CTA), otherwise d_model slices reloaded per pass.
+  float* sW = reinterpret_cast<float*>(router_smem);
+  __shared__ float s_wsq[EB];
   __shared__ float s_wnorm[EB];
   __shared__ int s_hist[EB];
   __shared__ double s_l64[kRouterWarps][EB];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nslices = (Dm + DS - 1) / DS;
+  const bool resident = nslices == 1;
 
-  if (SMEM_W) {
-    for (int i = tid; i < Dm * E; i += kRouterThreads) sW[(i % E) * Dm + i / E] = w_r[i];
-    for (int i = tid; i < Dm * (EB - E) + STEP; i += kRouterThreads) sW[E * Dm + i] = 0.f;
+  for (int i = tid; i < EB * DS + STEP; i += kRouterThreads)
+    if (i >= EB * DS) sW[i] = 0.f;  // pad read by the last lanes of a step
+  for (int e = tid; e < EB; e += kRouterThreads) s_wsq[e] = 0.f;
+  bool norms_ready = false;
+  if (resident) {
+    load_w_slice(sW, w_r, Dm, E, EB, 0, DS, tid);
     __syncthreads();
-  }
-  for (int e = warp; e < EB; e += kRouterWarps) {
-    float s = 0.f;
-    if (e < E)
-      for (int d = lane; d < Dm; d += 32) {
-        const float w = SMEM_W ? sW[e * Dm + d] : __ldg(w_r + static_cast<int64_t>(d) * E + e);
-        s = fmaf(w, w, s);
-      }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) s_wnorm[e] = sqrtf(s);
   }
 
   for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
@@ -246,49 +259,67 @@ __global__ void __launch_bounds__(kRouterThreads)
 #pragma unroll
       for (int t = 0; t < TPW; ++t) sq[t] = 0.f;
 
-      for (int d0 = 0; d0 < Dm; d0 += STEP) {
-        float xv[TPW][V];
+      for (int s = 0; s < nslices; ++s) {
+        const int D0 = s * DS;
+        if (!resident) {
+          __syncthreads();  // every warp is done with the previous slice
+          load_w_slice(sW, w_r, Dm, E, EB, D0, DS, tid);
+          __syncthreads();
+        }
+        if (!norms_ready) {
+          // |w_e|^2 over this slice, accumulated per expert in slice order.
+          for (int e = warp; e < EB; e += kRouterWarps) {
+            float q = 0.f;
+            for (int d = lane; d < DS; d += 32) q = fmaf(sW[e * DS + d], sW[e * DS + d], q);
 #pragma unroll
-        for (int t = 0; t < TPW; ++t) {
+            for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+            if (lane == 0) s_wsq[e] += q;
+          }
+        }
+        const int dend = min(Dm, D0 + DS);
+        for (int d0 = D0; d0 < dend; d0 += STEP) {
+          float xv[TPW][V];
 #pragma unroll
-          for (int g = 0; g < V / 4; ++g) {
-            const int d = d0 + group_off<InT>(g, lane);
-            if (t0 + t < T && d < Dm) {
-              load4(x + (t0 + t) * static_cast<int64_t>(Dm) + d, &xv[t][4 * g]);
-            } else {
+          for (int t = 0; t < TPW; ++t) {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) xv[t][4 * g + j] = 0.f;
+            for (int g = 0; g < V / 4; ++g) {
+              const int d = d0 + group_off<InT>(g, lane);
+              if (t0 + t < T && d < Dm) {
+                load4(x + (t0 + t) * static_cast<int64_t>(Dm) + d, &xv[t][4 * g]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) xv[t][4 * g + j] = 0.f;
+              }
             }
+#pragma unroll
+            for (int v = 0; v < V; ++v) sq[t] = fmaf(xv[t][v], xv[t][v], sq[t]);
           }
 #pragma unroll
-          for (int v = 0; v < V; ++v) sq[t] = fmaf(xv[t][v], xv[t][v], sq[t]);
-        }
+          for (int e = 0; e < EB; ++e) {
+            float wv[V];
 #pragma unroll
-        for (int e = 0; e < EB; ++e) {
-          float wv[V];
-#pragma unroll
-          for (int g = 0; g < V / 4; ++g) {
-            const int d = d0 + group_off<InT>(g, lane);
-            if (SMEM_W) {
-              const float4 q = *reinterpret_cast<const float4*>(sW + e * Dm + d);
+            for (int g = 0; g < V / 4; ++g) {
+              const float4 q = *reinterpret_cast<const float4*>(
+                  sW + e * DS + (d0 - D0) + group_off<InT>(g, lane));
               wv[4 * g] = q.x;
               wv[4 * g + 1] = q.y;
               wv[4 * g + 2] = q.z;
               wv[4 * g + 3] = q.w;
-            } else {
+            }
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                wv[4 * g + j] = (e < E && d + j < Dm)
-                                    ? __ldg(w_r + static_cast<int64_t>(d + j) * E + e)
-                                    : 0.f;
+            for (int t = 0; t < TPW; ++t) {
+#pragma unroll
+              for (int v = 0; v < V; ++v)
+                acc[t * EB + e] = fmaf(xv[t][v], wv[v], acc[t * EB + e]);
             }
           }
-#pragma unroll
-          for (int t = 0; t < TPW; ++t) {
-#pragma unroll
-            for (int v = 0; v < V; ++v) acc[t * EB + e] = fmaf(xv[t][v], wv[v], acc[t * EB + e]);
-          }
         }
+      }
+      if (!norms_ready) {
+        __syncthreads();
+        for (int e = tid; e < EB; e += kRouterThreads) s_wnorm[e] = sqrtf(s_wsq[e]);
+        __syncthreads();
+        norms_ready = true;
       }
 
       // |x|^2 of every token of the pass, on every lane.
@@ -350,8 +381,8 @@ __global__ void __launch_bounds__(kRouterThreads)
           const int src = __ffs(todo) - 1;
           const int tl_r = __shfl_sync(0xffffffffu, tl, src);
           todo &= ~(((W == 32) ? 0xffffffffu : ((1u << W) - 1u)) << (src & ~(W - 1)));
-          refine_logits_f64<InT, EB>(x + (t0 + tl_r) * static_cast<int64_t>(Dm), Dm, sW, w_r,
-                                     bias, E, SMEM_W, s_l64[warp], lane);
+          refine_logits_f64<InT, EB>(x + (t0 + tl_r) * static_cast<int64_t>(Dm), Dm, DS, sW, w_r,
+                                     bias, E, resident, s_l64[warp], lane);
           double lv64[VPT];
 #pragma unroll
           for (int v = 0; v < VPT; ++v)
@@ -420,25 +451,23 @@ cudaError_t launch_eb(const InT* x, int64_t T, int Dm, const float* w_r, const f
   const double n = static_cast<double>(((Dm + STEP - 1) / STEP) * V + 5 + 2);
   const double u = 1.0 / 16777216.0;
   const float gamma = static_cast<float>(1.01 * n * u / (1.0 - n * u));
-  const size_t smem_w = (static_cast<size_t>(EB) * Dm + STEP) * sizeof(float);
+  // d_model slice held in shared memory: all of it when it fits in 160 KB.
+  const int dm_pad = (Dm + STEP - 1) / STEP * STEP;
+  const int ds_max = ((160 * 1024 / 4 - STEP) / EB) / STEP * STEP;
+  const int DS = std::min(dm_pad, ds_max);
+  const size_t smem_w = (static_cast<size_t>(EB) * DS + STEP) * sizeof(float);
   const int sms = device_sm_count();
-  if (smem_w <= 160 * 1024) {
-    auto kern = router_kernel<InT, EB, true>;
-    cudaError_t err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
-    if (err != cudaSuccess) return err;
-    int per_sm = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRouterThreads, smem_w);
-    if (per_sm < 1) per_sm = 1;
-    const int64_t grid = std::min<int64_t>(nchunks, static_cast<int64_t>(sms) * per_sm);
-    kern<<<static_cast<unsigned>(grid), kRouterThreads, smem_w, stream>>>(
-        x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist, nchunks, gamma);
-  } else {
-    auto kern = router_kernel<InT, EB, false>;
-    const int64_t grid = std::min<int64_t>(nchunks, static_cast<int64_t>(sms) * 2);
-    kern<<<static_cast<unsigned>(grid), kRouterThreads, 0, stream>>>(
-        x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist, nchunks, gamma);
-  }
+  auto kern = router_kernel<InT, EB>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
+  if (err != cudaSuccess) return err;
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRouterThreads, smem_w);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t grid = std::min<int64_t>(nchunks, static_cast<int64_t>(sms) * per_sm);
+  kern<<<static_cast<unsigned>(grid), kRouterThreads, smem_w, stream>>>(
+      x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist, nchunks, gamma,
+      DS);
   return cudaGetLastError();
 }
 
