@@ -177,6 +177,46 @@ int rom_get_status(void* stream, int32_t* host_status);
  */
 int rom_debug_wait_timeout(uint64_t limit_ns, void* stream);
 
+/*
+ * rom_route_dispatch_noalloc -- rom_route() followed by rom_dispatch(), for
+ * callers that cannot allocate device memory. The paper has no counterpart:
+ * this is a deployment variant of the two calls above.
+ *
+ * Who needs it: code that may not call cudaMalloc or any allocator (for
+ * example a plugin that only receives the host framework's buffers, or a
+ * process whose memory is fully reserved by its own pool) cannot provide the
+ * workspace that rom_route() and rom_dispatch() exchange. This entry point
+ * keeps that scratch (the router's per-chunk expert histograms) in a fixed
+ * array of ROM_NOALLOC_SCRATCH_WORDS int32 in the library's own device
+ * memory, which every GPU that loads the library holds until the process
+ * exits. It allocates nothing and calls no allocating routine; the caller
+ * still passes every input and output.
+ *
+ * Arguments, layouts and outputs are those of rom_route() (x, dtype, T, Dm,
+ * w_r, bias, E, k, renorm, topk_idx, topk_w, counts) and rom_dispatch()
+ * (offsets, sorted_slot, slot_pos, x_sorted), without the workspace.
+ *
+ * Limits and errors: ceil(T / 128) * E must not exceed
+ * ROM_NOALLOC_SCRATCH_WORDS (e.g. T <= 1,048,576 tokens at E = 8), else the
+ * call returns ROM_ERR_WORKSPACE and enqueues nothing. Other argument errors
+ * are those of rom_route() and rom_dispatch().
+ *
+ * Sharing: every call on a device uses the same array. Calls that can
+ * overlap on the GPU (unordered streams) race on it and must not be issued;
+ * calls on one stream are safe. The array keeps the last call's contents,
+ * which is harmless: the router rewrites every entry the dispatch reads.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (with that device current) and caches it; make that first call before
+ * any stream capture on the device.
+ */
+#define ROM_NOALLOC_SCRATCH_WORDS 65536
+int rom_route_dispatch_noalloc(const void* x, int dtype, int64_t T, int Dm, const float* w_r,
+                               const float* bias, int E, int k, int renorm, int32_t* topk_idx,
+                               float* topk_w, int32_t* counts, int32_t* offsets,
+                               int32_t* sorted_slot, int32_t* slot_pos, void* x_sorted,
+                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,6 +38,8 @@ SIGNATURES = {
     "rom_combine": (_I, [_I, _I, _P, _L, _I, _I, _P, _P, _P]),
     "rom_get_status": (_I, [_P, ctypes.POINTER(ctypes.c_int32)]),
     "rom_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+    "rom_route_dispatch_noalloc": (_I, [_P, _I, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
+                                        _P, _P, _P]),
 }
 
 _lib = None
@@ -141,6 +143,18 @@ def rom_get_status(stream=None) -> int:
 def rom_debug_wait_timeout(limit_ns: int, stream=None):
     _check(load_library().rom_debug_wait_timeout(limit_ns, _stream(stream)),
            "rom_debug_wait_timeout")
+
+
+def rom_route_dispatch_noalloc(x, w_r, bias, k, renorm, topk_idx, topk_w, counts, offsets,
+                               sorted_slot, slot_pos, x_sorted, stream=None):
+    """Routing + dispatch without a caller workspace (the library's own fixed
+    device scratch; see include/rom.h)."""
+    T, Dm = x.shape
+    E = w_r.shape[1]
+    _check(load_library().rom_route_dispatch_noalloc(
+        _ptr(x), _dtype_code(x), T, Dm, _ptr(w_r), _ptr(bias), E, k, int(renorm),
+        _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets), _ptr(sorted_slot),
+        _ptr(slot_pos), _ptr(x_sorted), _stream(stream)), "rom_route_dispatch_noalloc")
 
 
 # ------------------------------------------------------------------ block helpers
