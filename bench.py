@@ -55,7 +55,10 @@ def block_flops(wl):
     R = wl.T * wl.k
     if wl.kind == "inproj":
         return {"inproj": 2.0 * R * wl.Dm * wl.De}
-    return {"conv_gate": 4.0 * R * wl.Dm * wl.De, "out": 2.0 * R * wl.De * wl.Dm}
+    f = {"conv_gate": 4.0 * R * wl.Dm * wl.De, "out": 2.0 * R * wl.De * wl.Dm}
+    if wl.backward:  # dgrad (Out, In+Gate) and wgrad (Out, In+Gate): twice the forward
+        f["backward"] = 2.0 * (f["conv_gate"] + f["out"])
+    return f
 
 
 def inproj_bytes(wl, n_experts_hit):
@@ -245,6 +248,14 @@ def run_ours(args, rank, world, local_rank):
         out_t = bufs.out
         counts_t = rb.counts
     phases = [ph_route, ph_p0, ph_p1]
+    if wl.backward:
+        dout = to_dev(torch, inp["dout"], bf16)
+        bwd_bufs = rom.BackwardBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.device)
+
+        def ph_bwd():
+            rom.block_backward(bufs, dout, w_r, ws["w_conv"], ws["w_gate"], ws["w_out"],
+                               renorm=wl.renorm, bufs=bwd_bufs)
+        phases.append(ph_bwd)
 
     def step():
         for ph in phases:
@@ -256,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     if wl.kind == "inproj":
         launches_per_step = 3 + (1 if wl.k > 1 else 0)
     else:
-        launches_per_step = 4 + (2 if wl.k > 1 else 0)
+        launches_per_step = 4 + (2 if wl.k > 1 else 0) + (7 if wl.backward else 0)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -304,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     eager_ms = timed_loop(lambda j: phases[j](), args.steps)
     t_total_ms = float(ph_ms.sum())
-    part_names = ["route_dispatch", "proj0", "proj1"]
+    part_names = ["route_dispatch", "proj0", "proj1", "backward"][:len(phases)]
     part_ms = {n: float(ph_ms[:, j].mean()) for j, n in enumerate(part_names)}
 
     # ---------------------------------------------- e2e through host buffers
@@ -356,7 +367,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = WORKLOADS[args.workload]
     flops = block_flops(wl)
-    metric = "tokens/s for RoM projection block fwd"
+    metric = ("tokens/s for RoM projection block fwd+bwd" if wl.backward
+              else "tokens/s for RoM projection block fwd")
     config = {"workload": wl.name, "tokens": wl.T, "d_model": wl.Dm,
               ("d_out" if wl.kind == "inproj" else "d_inner"): wl.De, "experts": wl.E,
               "top_k": wl.k, "renorm": wl.renorm, "parallelism": f"replicas x{world}",
@@ -427,6 +439,7 @@ def main():
                 "block_tflops": tot_flops / step_s / 1e12,
                 "block_frac_of_bf16_peak": tot_flops / step_s / 1e12 / peaks["bf16_tflops"],
                 "kernels_ms": res["part_ms"], "eager_ms_per_step": res["eager_ms"],
+                "step": "forward + backward" if wl.backward else "forward",
                 "timing": "each phase replayed as a CUDA graph; CUDA events on the launching "
                           "stream between phases",
                 "e2e": {"value": wl.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",

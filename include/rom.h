@@ -177,6 +177,81 @@ int rom_get_status(void* stream, int32_t* host_status);
  */
 int rom_debug_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Backward of the block (bf16), for the loss L = sum_t <O_t, dO_t> with the
+ * selection S_t held fixed (RoM page, Knowl 1, differentiated). With
+ * g_{t,j} = dO_t W_out,S_j^T:
+ *   dr_{t,j} = <Y_t (.) G_t, g_{t,j}>,   d(Y(.)G)_t = sum_j r_{t,j} g_{t,j},
+ *   dH = d(Y(.)G) (.) G,   dZ = d(Y(.)G) (.) H (.) SiLU'(Z)   (Z: the gate sum),
+ *   dlogit_{t,j} = r_j (dr_j - sum_i r_i dr_i)   (renormalised top-k weights),
+ *   dX_t = sum_j (dH W_in,S_j^T + dZ W_g,S_j^T) + sum_j dlogit_j W_r[:, S_j],
+ *   dW_in,e = sum_{t->e} x_t^T dH_t,   dW_g,e = sum_{t->e} x_t^T dZ_t,
+ *   dW_out,e = sum_{(t,j)->e} r_{t,j} (Y(.)G)_t^T dO_t.
+ * Call order: rom_bwd_gather, rom_bwd_dgrad_out, rom_bwd_gate,
+ * rom_bwd_dgrad_in, rom_route_bwd, rom_bwd_wgrad (twice). Every buffer is a
+ * caller-owned device buffer; the sorted arrays use the forward's offsets,
+ * sorted_slot and slot_pos. R = T*k, Dm = d_model, De = d_inner.
+ * ------------------------------------------------------------------------ */
+
+/* rdo_sorted[p] = r_s * dO[s / k] (bf16), s = sorted_slot[p]; dout [T][N]
+ * bf16. Requires N % 8 == 0. */
+int rom_bwd_gather(const void* dout, int64_t T, int k, int N, const int32_t* sorted_slot,
+                   const float* topk_w, void* rdo_sorted, void* stream);
+
+/*
+ * Out dgrad: g'_s = rdo_sorted_s W_out,e^T (= r_s g_s) for the rows of each
+ * expert. w_out [E][Dm][De] (forward layout); h_sorted [R][De] bf16 (the
+ * forward's Y(.)G rows). Outputs: g_slots float32 [R][De] in slot order, and
+ * dr_part float32 [R][De/256], the partial dots <h_s, g'_s> of each
+ * 256-column tile. Requires Dm % 64 == 0 and De % 256 == 0.
+ */
+int rom_bwd_dgrad_out(const void* rdo_sorted, int64_t R, int Dm, const void* w_out, int De, int E,
+                      int k, const int32_t* offsets, const int32_t* sorted_slot,
+                      const void* h_sorted, float* g_slots, float* dr_part, void* stream);
+
+/*
+ * Gate backward. uz: float32 [2][R][De], the u and z of every slot in slot
+ * order (the forward's rom_expert_proj(ROM_PROJ_CONV_GATE) output for k > 1);
+ * g_slots from rom_bwd_dgrad_out. Writes dhz_sorted bf16 [R][2*De]: row
+ * slot_pos[s] = [dH_t | dZ_t] of the slot's token t. Requires De % 4 == 0.
+ */
+int rom_bwd_gate(const float* uz, const float* g_slots, int64_t T, int k, int De,
+                 const int32_t* slot_pos, void* dhz_sorted, void* stream);
+
+/*
+ * In/Gate dgrad: dx_slots_s = dhz_sorted_s [W_in,e ; W_g,e]^T (K = 2*De);
+ * w_in, w_g [E][De][Dm] (forward layout). Output float32 [R][Dm], slot order.
+ * Requires De % 64 == 0 and Dm % 256 == 0.
+ */
+int rom_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const void* w_in,
+                     const void* w_g, int Dm, int E, int k, const int32_t* offsets,
+                     const int32_t* sorted_slot, float* dx_slots, void* stream);
+
+/*
+ * Router backward and dX: dr_{t,j} = (sum of dr_part[s][0 .. n_parts)) / r_s;
+ * dlogits [T][E] float32 (may be NULL; zero off S_t);
+ * dx [T][Dm] bf16 = sum_j dx_slots[t*k+j] + sum_j dlogit_{t,j} w_r[:, S_j].
+ * The weights must be renormalised (renorm = 1): r = p without
+ * renormalisation would need every expert's probability (ROM_ERR_UNSUPPORTED).
+ * Requires Dm % 4 == 0.
+ */
+int rom_route_bwd(int64_t T, int k, int E, int Dm, int renorm, const int32_t* topk_idx,
+                  const float* topk_w, const float* dr_part, int n_parts,
+                  const float* dx_slots, const float* w_r, float* dlogits, void* dx,
+                  void* stream);
+
+/*
+ * Weight gradients of every expert: out[e] = A_e^T B_e, A_e and B_e the rows
+ * offsets[e] .. offsets[e+1]-1 of a_sorted [R][M] and b_sorted [R][N]
+ * (bf16). float32 result rows m < m_split go to out0 [E][m_split][N], the
+ * others to out1 [E][M - m_split][N] (out1 may be NULL when m_split == M).
+ * Experts without rows get zeros. dW_out = wgrad(rdo_sorted, h_sorted);
+ * [dW_in ; dW_g] = wgrad(dhz_sorted, x_sorted, m_split = De).
+ * Requires M % 128 == 0, N % 256 == 0 and m_split % 128 == 0.
+ */
+int rom_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int64_t R, int E,
+                  const int32_t* offsets, int m_split, float* out0, float* out1, void* stream);
+
 /*
  * rom_route_dispatch_noalloc -- rom_route() followed by rom_dispatch(), for
  * callers that cannot allocate device memory. The paper has no counterpart:

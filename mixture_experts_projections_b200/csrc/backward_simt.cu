@@ -1,0 +1,225 @@
+// Bandwidth-bound pieces of the RoM block backward ("Routing Mamba ..."
+// chapterpal summary page, Knowl 1, differentiated with S_t held fixed):
+//
+//  scale_gather  rdO_sorted[p] = r_s * dO[s / k]   (s = sorted_slot[p]); the A
+//                operand of the Out dgrad (giving g'_s = r_s g_s) and of dW_out.
+//  gate_bwd      per token t and column c, with H = sum_j u_{t,j},
+//                Z = sum_j z_{t,j} (the forward's float32 slot partials) and
+//                dYG = sum_j g'_{t,j} = sum_j r_j g_j:
+//                  dH = dYG * SiLU(Z),  dZ = dYG * H * SiLU'(Z),
+//                  SiLU'(Z) = s (1 + Z (1 - s)), s = sigmoid(Z);
+//                written as [dH | dZ] rows in expert-sorted order for every
+//                slot of the token (A operand of dX and of dW_in / dW_g).
+//  route_bwd     per token: dr_j = <Y(.)G, g_j> = (sum of the Out dgrad's
+//                partial dots) / r_j; with renormalised top-k weights
+//                r = softmax over the selected logits,
+//                  dlogit_j = r_j (dr_j - sum_i r_i dr_i)   (0 off S_t);
+//                dX_t = sum_j dX_{t,j} + sum_j dlogit_j W_r[:, S_j].
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <algorithm>
+
+#include "rom_internal.cuh"
+
+namespace rom {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// One warp per sorted row; 8 bf16 (16 bytes) per lane per step.
+__global__ void __launch_bounds__(kThreads)
+    scale_gather_kernel(const __nv_bfloat16* __restrict__ dout, int64_t R, int k, int N,
+                        const int32_t* __restrict__ sorted_slot,
+                        const float* __restrict__ topk_w, __nv_bfloat16* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+  const int nv = N / 8;
+  for (int64_t p = warp; p < R; p += nwarps) {
+    const int64_t s = sorted_slot[p];
+    const float r = topk_w[s];
+    const uint4* src = reinterpret_cast<const uint4*>(dout + (s / k) * N);
+    uint4* d = reinterpret_cast<uint4*>(dst + p * N);
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o[q] = pack2(r * __uint_as_float(w[q] << 16), r * __uint_as_float(w[q] & 0xFFFF0000u));
+      d[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// One thread per (token, 4 columns).
+__global__ void __launch_bounds__(kThreads)
+    gate_bwd_kernel(const float* __restrict__ uz, const float* __restrict__ gp, int64_t T, int k,
+                    int De, const int32_t* __restrict__ slot_pos, __nv_bfloat16* __restrict__ dhz) {
+  const int nq = De / 4;
+  const int64_t total = T * nq;
+  const int64_t R = T * k;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t t = i / nq;
+    const int c = static_cast<int>(i - t * nq) * 4;
+    float h[4] = {0.f, 0.f, 0.f, 0.f}, z[4] = {0.f, 0.f, 0.f, 0.f}, g[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int64_t s = t * k + j;
+      const float4 a = __ldg(reinterpret_cast<const float4*>(uz + s * De + c));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(uz + (R + s) * De + c));
+      const float4 d = __ldg(reinterpret_cast<const float4*>(gp + s * De + c));
+      h[0] += a.x; h[1] += a.y; h[2] += a.z; h[3] += a.w;
+      z[0] += b.x; z[1] += b.y; z[2] += b.z; z[3] += b.w;
+      g[0] += d.x; g[1] += d.y; g[2] += d.z; g[3] += d.w;
+    }
+    float dh[4], dz[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float s = 1.0f / (1.0f + expf(-z[q]));
+      dh[q] = g[q] * (z[q] * s);
+      dz[q] = g[q] * h[q] * (s * (1.0f + z[q] * (1.0f - s)));
+    }
+    const uint2 wh = make_uint2(pack2(dh[0], dh[1]), pack2(dh[2], dh[3]));
+    const uint2 wz = make_uint2(pack2(dz[0], dz[1]), pack2(dz[2], dz[3]));
+    for (int j = 0; j < k; ++j) {
+      const int64_t row = slot_pos[t * k + j];
+      *reinterpret_cast<uint2*>(dhz + row * (2 * De) + c) = wh;
+      *reinterpret_cast<uint2*>(dhz + row * (2 * De) + De + c) = wz;
+    }
+  }
+}
+
+// One warp per token; W_r^T slice [E][DS] staged in shared memory.
+__global__ void __launch_bounds__(kThreads)
+    route_bwd_kernel(int64_t T, int k, int E, int Dm, const int32_t* __restrict__ topk_idx,
+                     const float* __restrict__ topk_w, const float* __restrict__ dr_part,
+                     int n_parts, const float* __restrict__ dx_slots,
+                     const float* __restrict__ w_r, float* __restrict__ dlogits,
+                     __nv_bfloat16* __restrict__ dx, int DS) {
+  extern __shared__ float sWt[];  // [E][DS]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = kThreads / 32;
+  for (int D0 = 0; D0 < Dm; D0 += DS) {
+    const int dn = min(DS, Dm - D0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < dn * E; i += kThreads) {
+      const int d = i / E, e = i - d * E;
+      sWt[e * DS + d] = __ldg(w_r + static_cast<int64_t>(D0) * E + i);
+    }
+    __syncthreads();
+    for (int64_t t = blockIdx.x * static_cast<int64_t>(nw) + warp; t < T;
+         t += static_cast<int64_t>(gridDim.x) * nw) {
+      // dr_j and dlogit_j (recomputed per slice; a few dozen flops)
+      float dl[kMaxTopK];
+      int sel[kMaxTopK];
+      float s = 0.f;
+      float dr[kMaxTopK], rw[kMaxTopK];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        dl[j] = 0.f;
+        sel[j] = 0;
+        dr[j] = 0.f;
+        rw[j] = 0.f;
+        if (j < k) {
+          const int64_t slot = t * k + j;
+          float acc = 0.f;
+          for (int q = lane; q < n_parts; q += 32) acc += dr_part[slot * n_parts + q];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          rw[j] = topk_w[slot];
+          sel[j] = topk_idx[slot];
+          dr[j] = acc / rw[j];
+          s += rw[j] * dr[j];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k) dl[j] = rw[j] * (dr[j] - s);
+      if (D0 == 0 && dlogits) {
+        for (int e = lane; e < E; e += 32) {
+          float v = 0.f;
+#pragma unroll
+          for (int j = 0; j < kMaxTopK; ++j)
+            if (j < k && sel[j] == e) v = dl[j];
+          dlogits[t * E + e] = v;
+        }
+      }
+      for (int d = lane * 4; d < dn; d += 128) {
+        float4 acc = __ldg(reinterpret_cast<const float4*>(dx_slots + (t * k) * Dm + D0 + d));
+        for (int j = 1; j < k; ++j) {
+          const float4 v =
+              __ldg(reinterpret_cast<const float4*>(dx_slots + (t * k + j) * Dm + D0 + d));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+          if (j < k) {
+            const float4 w = *reinterpret_cast<const float4*>(sWt + sel[j] * DS + d);
+            acc.x = fmaf(dl[j], w.x, acc.x);
+            acc.y = fmaf(dl[j], w.y, acc.y);
+            acc.z = fmaf(dl[j], w.z, acc.z);
+            acc.w = fmaf(dl[j], w.w, acc.w);
+          }
+        }
+        *reinterpret_cast<uint2*>(dx + t * Dm + D0 + d) =
+            make_uint2(pack2(acc.x, acc.y), pack2(acc.z, acc.w));
+      }
+    }
+  }
+}
+
+unsigned grid_for(int64_t work_items, int per_block) {
+  const int64_t g = (work_items + per_block - 1) / per_block;
+  return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(g, device_sm_count() * 16)));
+}
+
+}  // namespace
+
+cudaError_t launch_scale_gather(const void* dout, int64_t R, int k, int N,
+                                const int32_t* sorted_slot, const float* topk_w, void* dst,
+                                cudaStream_t stream) {
+  if (R == 0) return cudaSuccess;
+  scale_gather_kernel<<<grid_for(R, kThreads / 32), kThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(dout), R, k, N, sorted_slot, topk_w,
+      static_cast<__nv_bfloat16*>(dst));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_bwd(const float* uz, const float* gp, int64_t T, int k, int De,
+                            const int32_t* slot_pos, void* dhz, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  gate_bwd_kernel<<<grid_for(T * (De / 4), kThreads), kThreads, 0, stream>>>(
+      uz, gp, T, k, De, slot_pos, static_cast<__nv_bfloat16*>(dhz));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_bwd(int64_t T, int k, int E, int Dm, const int32_t* topk_idx,
+                             const float* topk_w, const float* dr_part, int n_parts,
+                             const float* dx_slots, const float* w_r, float* dlogits, void* dx,
+                             cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  // W_r^T slice: all of d_model when E * Dm floats fit in 160 KB.
+  const int ds_max = (160 * 1024 / 4 / E) / 128 * 128;
+  const int DS = std::min((Dm + 127) / 128 * 128, std::max(128, ds_max));
+  const size_t smem = static_cast<size_t>(E) * DS * sizeof(float);
+  cudaError_t err = cudaFuncSetAttribute(route_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((T + 7) / 8, device_sm_count()));
+  route_bwd_kernel<<<grid, kThreads, smem, stream>>>(T, k, E, Dm, topk_idx, topk_w, dr_part,
+                                                     n_parts, dx_slots, w_r, dlogits,
+                                                     static_cast<__nv_bfloat16*>(dx), DS);
+  return cudaGetLastError();
+}
+
+}  // namespace rom

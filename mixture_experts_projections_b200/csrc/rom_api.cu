@@ -217,6 +217,99 @@ int rom_get_status(void* stream, int32_t* host_status) {
   return ROM_OK;
 }
 
+int rom_bwd_gather(const void* dout, int64_t T, int k, int N, const int32_t* sorted_slot,
+                   const float* topk_w, void* rdo_sorted, void* stream) {
+  if (T < 0 || k < 1 || k > rom::kMaxTopK || N <= 0) return ROM_ERR_INVALID_ARG;
+  if (N % 8 != 0 || T * k >= (int64_t(1) << 31)) return ROM_ERR_UNSUPPORTED;
+  if (T == 0) return ROM_OK;
+  if (!dout || !sorted_slot || !topk_w || !rdo_sorted) return ROM_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(rdo_sorted)) return ROM_ERR_UNSUPPORTED;
+  return rom::to_status(rom::launch_scale_gather(dout, T * k, k, N, sorted_slot, topk_w,
+                                                 rdo_sorted, static_cast<cudaStream_t>(stream)));
+}
+
+int rom_bwd_dgrad_out(const void* rdo_sorted, int64_t R, int Dm, const void* w_out, int De, int E,
+                      int k, const int32_t* offsets, const int32_t* sorted_slot,
+                      const void* h_sorted, float* g_slots, float* dr_part, void* stream) {
+  if (R < 0 || Dm <= 0 || De <= 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E ||
+      k > rom::kMaxTopK || R % k != 0)
+    return ROM_ERR_INVALID_ARG;
+  if (Dm % 64 != 0 || De % 256 != 0 || R >= (int64_t(1) << 31)) return ROM_ERR_UNSUPPORTED;
+  if (!offsets || !w_out || !sorted_slot || !h_sorted || !g_slots || !dr_part ||
+      (R > 0 && !rdo_sorted))
+    return ROM_ERR_INVALID_ARG;
+  if (!aligned16(rdo_sorted) || !aligned16(w_out) || !aligned16(h_sorted) || !aligned16(g_slots))
+    return ROM_ERR_UNSUPPORTED;
+  int* st = rom::status_ptr();
+  if (!st) return ROM_ERR_CUDA;
+  return rom::to_status(rom::launch_bwd_dgrad_out(rdo_sorted, R, Dm, w_out, De, E, k, offsets,
+                                                  sorted_slot, h_sorted, g_slots, dr_part, st,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int rom_bwd_gate(const float* uz, const float* g_slots, int64_t T, int k, int De,
+                 const int32_t* slot_pos, void* dhz_sorted, void* stream) {
+  if (T < 0 || k < 1 || k > rom::kMaxTopK || De <= 0) return ROM_ERR_INVALID_ARG;
+  if (De % 4 != 0) return ROM_ERR_UNSUPPORTED;
+  if (T == 0) return ROM_OK;
+  if (!uz || !g_slots || !slot_pos || !dhz_sorted) return ROM_ERR_INVALID_ARG;
+  if (!aligned16(uz) || !aligned16(g_slots) || !aligned16(dhz_sorted)) return ROM_ERR_UNSUPPORTED;
+  return rom::to_status(rom::launch_gate_bwd(uz, g_slots, T, k, De, slot_pos, dhz_sorted,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int rom_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const void* w_in,
+                     const void* w_g, int Dm, int E, int k, const int32_t* offsets,
+                     const int32_t* sorted_slot, float* dx_slots, void* stream) {
+  if (R < 0 || Dm <= 0 || De <= 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E ||
+      k > rom::kMaxTopK || R % k != 0)
+    return ROM_ERR_INVALID_ARG;
+  if (De % 64 != 0 || Dm % 256 != 0 || R >= (int64_t(1) << 31)) return ROM_ERR_UNSUPPORTED;
+  if (!offsets || !w_in || !w_g || !sorted_slot || !dx_slots || (R > 0 && !dhz_sorted))
+    return ROM_ERR_INVALID_ARG;
+  if (!aligned16(dhz_sorted) || !aligned16(w_in) || !aligned16(w_g) || !aligned16(dx_slots))
+    return ROM_ERR_UNSUPPORTED;
+  int* st = rom::status_ptr();
+  if (!st) return ROM_ERR_CUDA;
+  return rom::to_status(rom::launch_bwd_dgrad_in(dhz_sorted, R, De, w_in, w_g, Dm, E, k, offsets,
+                                                 sorted_slot, dx_slots, st,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+int rom_route_bwd(int64_t T, int k, int E, int Dm, int renorm, const int32_t* topk_idx,
+                  const float* topk_w, const float* dr_part, int n_parts,
+                  const float* dx_slots, const float* w_r, float* dlogits, void* dx,
+                  void* stream) {
+  if (T < 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E || k > rom::kMaxTopK || Dm <= 0 ||
+      n_parts < 1 || (renorm != 0 && renorm != 1))
+    return ROM_ERR_INVALID_ARG;
+  if (renorm != 1 || Dm % 4 != 0) return ROM_ERR_UNSUPPORTED;
+  if (T == 0) return ROM_OK;
+  if (!topk_idx || !topk_w || !dr_part || !dx_slots || !w_r || !dx) return ROM_ERR_INVALID_ARG;
+  if (!aligned16(dx_slots) || !aligned16(w_r) || (reinterpret_cast<uintptr_t>(dx) & 7u))
+    return ROM_ERR_UNSUPPORTED;
+  return rom::to_status(rom::launch_route_bwd(T, k, E, Dm, topk_idx, topk_w, dr_part, n_parts,
+                                              dx_slots, w_r, dlogits, dx,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int rom_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int64_t R, int E,
+                  const int32_t* offsets, int m_split, float* out0, float* out1, void* stream) {
+  if (M <= 0 || N <= 0 || R < 0 || E < 1 || E > rom::kMaxExperts || m_split < 0 || m_split > M)
+    return ROM_ERR_INVALID_ARG;
+  if (M % 128 != 0 || N % 256 != 0 || m_split % 128 != 0 || R >= (int64_t(1) << 31))
+    return ROM_ERR_UNSUPPORTED;
+  if (!a_sorted || !b_sorted || !offsets || !out0 || (m_split < M && !out1))
+    return ROM_ERR_INVALID_ARG;
+  if (!aligned16(a_sorted) || !aligned16(b_sorted) || !aligned16(out0) ||
+      (out1 && !aligned16(out1)))
+    return ROM_ERR_UNSUPPORTED;
+  int* st = rom::status_ptr();
+  if (!st) return ROM_ERR_CUDA;
+  return rom::to_status(rom::launch_bwd_wgrad(a_sorted, M, b_sorted, N, R, E, offsets, m_split,
+                                              out0, out1, st, static_cast<cudaStream_t>(stream)));
+}
+
 int rom_debug_wait_timeout(uint64_t limit_ns, void* stream) {
   if (limit_ns < 1000ull || limit_ns > 10000000000ull) return ROM_ERR_INVALID_ARG;
   int* st = rom::status_ptr();

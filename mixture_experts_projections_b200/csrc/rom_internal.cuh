@@ -54,4 +54,28 @@ cudaError_t launch_combine(int mode, bool bf16, const float* in, int64_t T, int 
 
 cudaError_t launch_debug_wait(uint64_t limit_ns, int* status, cudaStream_t stream);
 
+// ---- backward (grouped_gemm_bwd.cu, backward_simt.cu)
+enum BwdMode : int { kBwdDgradOut = 0, kBwdDgradIn = 1, kBwdWgrad = 2 };
+
+cudaError_t launch_bwd_dgrad_out(const void* rdo_sorted, int64_t R, int Dm, const void* w_out,
+                                 int De, int E, int k, const int32_t* offsets,
+                                 const int32_t* sorted_slot, const void* h_sorted, float* g_slots,
+                                 float* dr_part, int* status, cudaStream_t stream);
+cudaError_t launch_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const void* w_in,
+                                const void* w_g, int Dm, int E, int k, const int32_t* offsets,
+                                const int32_t* sorted_slot, float* dx_slots, int* status,
+                                cudaStream_t stream);
+cudaError_t launch_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int64_t R,
+                             int E, const int32_t* offsets, int m_split, float* out0, float* out1,
+                             int* status, cudaStream_t stream);
+cudaError_t launch_scale_gather(const void* dout, int64_t R, int k, int N,
+                                const int32_t* sorted_slot, const float* topk_w, void* dst,
+                                cudaStream_t stream);
+cudaError_t launch_gate_bwd(const float* uz, const float* gp, int64_t T, int k, int De,
+                            const int32_t* slot_pos, void* dhz, cudaStream_t stream);
+cudaError_t launch_route_bwd(int64_t T, int k, int E, int Dm, const int32_t* topk_idx,
+                             const float* topk_w, const float* dr_part, int n_parts,
+                             const float* dx_slots, const float* w_r, float* dlogits, void* dx,
+                             cudaStream_t stream);
+
 }  // namespace rom

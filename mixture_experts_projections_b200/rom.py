@@ -40,6 +40,12 @@ SIGNATURES = {
     "rom_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "rom_route_dispatch_noalloc": (_I, [_P, _I, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
                                         _P, _P, _P]),
+    "rom_bwd_gather": (_I, [_P, _L, _I, _I, _P, _P, _P, _P]),
+    "rom_bwd_dgrad_out": (_I, [_P, _L, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "rom_bwd_gate": (_I, [_P, _P, _L, _I, _I, _P, _P, _P]),
+    "rom_bwd_dgrad_in": (_I, [_P, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P]),
+    "rom_route_bwd": (_I, [_L, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
+    "rom_bwd_wgrad": (_I, [_P, _I, _P, _I, _L, _I, _P, _I, _P, _P, _P]),
 }
 
 _lib = None
@@ -256,3 +262,99 @@ def inproj_forward(x, w_r, w, k=1, renorm=False, bias=None, bufs=None, out=None,
                         rb.sorted_slot, rb.topk_w, slots, stream)
         rom_combine(ROM_COMBINE_SUM, _dtype_code(x), slots, T, k, N, None, out, stream)
     return out, rb
+
+
+# ------------------------------------------------------------------ backward
+
+
+def rom_bwd_gather(dout, k, sorted_slot, topk_w, rdo_sorted, stream=None):
+    T, N = dout.shape
+    _check(load_library().rom_bwd_gather(_ptr(dout), T, k, N, _ptr(sorted_slot), _ptr(topk_w),
+                                         _ptr(rdo_sorted), _stream(stream)), "rom_bwd_gather")
+
+
+def rom_bwd_dgrad_out(rdo_sorted, w_out, E, k, offsets, sorted_slot, h_sorted, g_slots, dr_part,
+                      stream=None):
+    R, Dm = rdo_sorted.shape
+    De = w_out.shape[2]
+    _check(load_library().rom_bwd_dgrad_out(
+        _ptr(rdo_sorted), R, Dm, _ptr(w_out), De, E, k, _ptr(offsets), _ptr(sorted_slot),
+        _ptr(h_sorted), _ptr(g_slots), _ptr(dr_part), _stream(stream)), "rom_bwd_dgrad_out")
+
+
+def rom_bwd_gate(uz, g_slots, T, k, De, slot_pos, dhz_sorted, stream=None):
+    _check(load_library().rom_bwd_gate(_ptr(uz), _ptr(g_slots), T, k, De, _ptr(slot_pos),
+                                       _ptr(dhz_sorted), _stream(stream)), "rom_bwd_gate")
+
+
+def rom_bwd_dgrad_in(dhz_sorted, w_in, w_g, E, k, offsets, sorted_slot, dx_slots, stream=None):
+    R = dhz_sorted.shape[0]
+    De = dhz_sorted.shape[1] // 2
+    Dm = w_in.shape[2]
+    _check(load_library().rom_bwd_dgrad_in(
+        _ptr(dhz_sorted), R, De, _ptr(w_in), _ptr(w_g), Dm, E, k, _ptr(offsets),
+        _ptr(sorted_slot), _ptr(dx_slots), _stream(stream)), "rom_bwd_dgrad_in")
+
+
+def rom_route_bwd(T, k, E, Dm, renorm, topk_idx, topk_w, dr_part, dx_slots, w_r, dlogits, dx,
+                  stream=None):
+    _check(load_library().rom_route_bwd(
+        T, k, E, Dm, int(renorm), _ptr(topk_idx), _ptr(topk_w), _ptr(dr_part), dr_part.shape[1],
+        _ptr(dx_slots), _ptr(w_r), _ptr(dlogits), _ptr(dx), _stream(stream)), "rom_route_bwd")
+
+
+def rom_bwd_wgrad(a_sorted, b_sorted, E, offsets, m_split, out0, out1, stream=None):
+    R, M = a_sorted.shape
+    N = b_sorted.shape[1]
+    _check(load_library().rom_bwd_wgrad(
+        _ptr(a_sorted), M, _ptr(b_sorted), N, R, E, _ptr(offsets), m_split, _ptr(out0),
+        _ptr(out1), _stream(stream)), "rom_bwd_wgrad")
+
+
+class BackwardBuffers:
+    """Device buffers of one backward pass (allocated by torch)."""
+
+    def __init__(self, T, Dm, De, E, k, device):
+        R = T * k
+        bf = torch.bfloat16
+        self.rdo_sorted = torch.empty((R, Dm), dtype=bf, device=device)
+        self.g_slots = torch.empty((R, De), dtype=torch.float32, device=device)
+        self.dr_part = torch.empty((R, De // 256), dtype=torch.float32, device=device)
+        self.dhz_sorted = torch.empty((R, 2 * De), dtype=bf, device=device)
+        self.dx_slots = torch.empty((R, Dm), dtype=torch.float32, device=device)
+        self.dx = torch.empty((T, Dm), dtype=bf, device=device)
+        self.dlogits = torch.empty((T, E), dtype=torch.float32, device=device)
+        self.dw_out = torch.empty((E, Dm, De), dtype=torch.float32, device=device)
+        self.dw_conv = torch.empty((E, De, Dm), dtype=torch.float32, device=device)
+        self.dw_gate = torch.empty((E, De, Dm), dtype=torch.float32, device=device)
+
+
+def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None, stream=None):
+    """Backward of the RoM block for top-k > 1 (renormalised weights).
+
+    fwd: the BlockBuffers of the forward (routing, h_sorted, u/z slot partials);
+    dout [T, Dm] bf16; weights in the library layout. Returns BackwardBuffers
+    with dx [T, Dm] bf16, dlogits [T, E] and dw_conv / dw_gate [E, De, Dm],
+    dw_out [E, Dm, De] (float32, the weights' layout).
+    """
+    rb = fwd.routing
+    T, Dm = dout.shape
+    E, De, _ = w_conv.shape
+    k = rb.k
+    if k < 2:
+        raise RomError("block_backward needs the forward's per-slot u/z partials (top-k > 1)")
+    R = T * k
+    if bufs is None:
+        bufs = BackwardBuffers(T, Dm, De, E, k, dout.device)
+    rom_bwd_gather(dout, k, rb.sorted_slot, rb.topk_w, bufs.rdo_sorted, stream)
+    rom_bwd_dgrad_out(bufs.rdo_sorted, w_out, E, k, rb.offsets, rb.sorted_slot,
+                      fwd.h_sorted[:R], bufs.g_slots, bufs.dr_part, stream)
+    rom_bwd_gate(fwd.uz, bufs.g_slots, T, k, De, rb.slot_pos, bufs.dhz_sorted, stream)
+    rom_bwd_dgrad_in(bufs.dhz_sorted, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
+                     bufs.dx_slots, stream)
+    rom_route_bwd(T, k, E, Dm, renorm, rb.topk_idx, rb.topk_w, bufs.dr_part, bufs.dx_slots, w_r,
+                  bufs.dlogits, bufs.dx, stream)
+    rom_bwd_wgrad(bufs.rdo_sorted, fwd.h_sorted[:R], E, rb.offsets, Dm, bufs.dw_out, None, stream)
+    rom_bwd_wgrad(bufs.dhz_sorted, rb.x_sorted[:R], E, rb.offsets, De, bufs.dw_conv, bufs.dw_gate,
+                  stream)
+    return bufs
