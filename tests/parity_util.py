@@ -3,7 +3,11 @@ layout and compare CUDA results with the CPU oracle.
 
 Tolerances (the floating-point bar of the parity tests):
   * routing indices, counts, offsets and the permutation: bit-exact;
-  * routing weights r: relative 2e-6 (float32 softmax of float32 logits);
+  * routing weights r: relative 2e-5. r = exp(l_e - m) / sum, so its
+    relative error is about twice the absolute error of the logits; the bf16
+    router accumulates each logit (d_model products) in float32 inside the
+    tensor cores, whose rounding reaches ~1e-5 at d_model = 2048 -- the
+    selection itself stays exact (near ties are re-decided in float64);
   * bf16 outputs: max abs error <= 2e-2 and relative Frobenius error <= 5e-3
     against the float64 oracle. The full-size workloads are held to exactly
     that. The synthetic test shapes and the bf16 intermediate h can reach
@@ -24,7 +28,7 @@ from mixture_experts_projections_b200.inputs import bf16_bits
 BF16_MAX_ABS = 2e-2
 BF16_REL_FRO = 5e-3
 F32_REL = 1e-5
-TOPK_W_RTOL = 2e-6
+TOPK_W_RTOL = 2e-5
 
 
 def to_dev(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
