@@ -143,12 +143,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // -------------------------------------------------- producer warp
+    // Lane L owns features d0 + L and d0 + L + 32 of each K block: it loads
+    // their E router weights (contiguous in w_r) and writes the three bf16
+    // parts into the B tile. For E <= 16 the next block's weights are loaded
+    // while the current block is converted.
+    constexpr bool kPrefetch = EP <= 16;
+    float wcur[2][EP], wnext[2][EP];
+    const bool vec4 = (E % 4) == 0;
+    auto load_w = [&](int kb, float (&dst)[2][EP]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int d = kb * BK + lane + 32 * h;
+        const float* src = w_r + static_cast<int64_t>(d) * E;
+        if (d < Dm && vec4) {
+#pragma unroll
+          for (int e4 = 0; e4 < EP / 4; ++e4) {
+            if (4 * e4 < E) {
+              const float4 v = __ldg(reinterpret_cast<const float4*>(src) + e4);
+              dst[h][4 * e4] = v.x;
+              dst[h][4 * e4 + 1] = v.y;
+              dst[h][4 * e4 + 2] = v.z;
+              dst[h][4 * e4 + 3] = v.w;
+            } else {
+              dst[h][4 * e4] = dst[h][4 * e4 + 1] = dst[h][4 * e4 + 2] = dst[h][4 * e4 + 3] = 0.f;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < EP; ++e) dst[h][e] = (d < Dm && e < E) ? __ldg(src + e) : 0.f;
+        }
+      }
+    };
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0, last_par = 0;
     bool ok = true;
+    bool have_next = false;
     for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb) {
+        if constexpr (kPrefetch) {
+          if (have_next) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int e = 0; e < EP; ++e) wcur[h][e] = wnext[h][e];
+          } else {
+            load_w(kb, wcur);
+          }
+          const int nkb = (kb + 1 < KB) ? kb + 1 : 0;  // the next tile restarts at block 0
+          load_w(nkb, wnext);
+          have_next = true;
+        } else {
+          load_w(kb, wcur);
+        }
         // every lane waits (and acquires); the outcome is made warp-uniform
         const bool got = mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, status);
         if (!__all_sync(0xffffffffu, got)) {
@@ -161,18 +208,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&ctl.full[stage], A_BYTES);
           tma_load_2d(sa, &tmX, &ctl.full[stage], kb * BK, static_cast<int>(tile * BM));
         }
-        // B tile: rows part * EP + e, columns d = 0..63 of this K block.
-        const int d0 = kb * BK;
-        for (int i = lane; i < BK * E; i += 32) {
-          const int d = i / E, e = i - d * E;
-          const float w = (d0 + d < Dm) ? __ldg(w_r + static_cast<int64_t>(d0) * E + i) : 0.f;
-          const uint16_t hi = bf16_bits_rn(w);
-          const float r1 = w - bf16_to_f(hi);
-          const uint16_t lo = bf16_bits_rn(r1);
-          const uint16_t lo2 = bf16_bits_rn(r1 - bf16_to_f(lo));
-          *reinterpret_cast<uint16_t*>(sb + sw128_off(e, d)) = hi;
-          *reinterpret_cast<uint16_t*>(sb + sw128_off(EP + e, d)) = lo;
-          *reinterpret_cast<uint16_t*>(sb + sw128_off(2 * EP + e, d)) = lo2;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int d = lane + 32 * h;
+#pragma unroll
+          for (int e = 0; e < EP; ++e) {
+            if (e < E) {
+              const float w = wcur[h][e];
+              const uint16_t hi = bf16_bits_rn(w);
+              const float r1 = w - bf16_to_f(hi);
+              const uint16_t lo = bf16_bits_rn(r1);
+              const uint16_t lo2 = bf16_bits_rn(r1 - bf16_to_f(lo));
+              *reinterpret_cast<uint16_t*>(sb + sw128_off(e, d)) = hi;
+              *reinterpret_cast<uint16_t*>(sb + sw128_off(EP + e, d)) = lo;
+              *reinterpret_cast<uint16_t*>(sb + sw128_off(2 * EP + e, d)) = lo2;
+            }
+          }
         }
         fence_async_shared();
         __syncwarp();
