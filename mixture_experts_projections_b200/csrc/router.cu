@@ -494,11 +494,9 @@ cudaError_t launch_router(const void* x, bool bf16, int64_t T, int Dm, const flo
                           const float* bias, int E, int k, int renorm, int32_t* topk_idx,
                           float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                           cudaStream_t stream) {
-  // bf16 activations: the tensor-core router (router_tc.cu); float32
-  // activations: the CUDA-core router below.
   if (bf16)
-    return launch_router_tc(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts,
-                            chunk_hist, status, stream);
+    return launch_typed(static_cast<const __nv_bfloat16*>(x), T, Dm, w_r, bias, E, k, renorm,
+                        topk_idx, topk_w, counts, chunk_hist, stream);
   return launch_typed(static_cast<const float*>(x), T, Dm, w_r, bias, E, k, renorm, topk_idx,
                       topk_w, counts, chunk_hist, stream);
 }
