@@ -22,6 +22,12 @@ cudaError_t launch_router(const void* x, bool bf16, int64_t T, int Dm, const flo
                           float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                           cudaStream_t stream);
 
+// Returns cudaErrorNotSupported when W_r does not fit in shared memory.
+cudaError_t launch_router_stream(const void* x, int64_t T, int Dm, const float* w_r,
+                                 const float* bias, int E, int k, int renorm, int32_t* topk_idx,
+                                 float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
+                                 cudaStream_t stream);
+
 cudaError_t launch_dispatch(const void* x, bool bf16, int64_t T, int Dm, int E, int k,
                             const int32_t* topk_idx, const int32_t* chunk_hist,
                             int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,

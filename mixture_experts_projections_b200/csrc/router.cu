@@ -494,9 +494,15 @@ cudaError_t launch_router(const void* x, bool bf16, int64_t T, int Dm, const flo
                           const float* bias, int E, int k, int renorm, int32_t* topk_idx,
                           float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                           cudaStream_t stream) {
-  if (bf16)
+  if (bf16) {
+    // The streaming router (router_stream.cu) when W_r stays resident in
+    // shared memory; the register-tiled kernel below otherwise.
+    const cudaError_t e = launch_router_stream(x, T, Dm, w_r, bias, E, k, renorm, topk_idx,
+                                               topk_w, counts, chunk_hist, status, stream);
+    if (e != cudaErrorNotSupported) return e;
     return launch_typed(static_cast<const __nv_bfloat16*>(x), T, Dm, w_r, bias, E, k, renorm,
                         topk_idx, topk_w, counts, chunk_hist, stream);
+  }
   return launch_typed(static_cast<const float*>(x), T, Dm, w_r, bias, E, k, renorm, topk_idx,
                       topk_w, counts, chunk_hist, stream);
 }
