@@ -45,6 +45,9 @@ constexpr int B_BYTES = UMMA_N * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * UMMA_N;
 constexpr int kThreads = 192;
+// Out / in-projection calls with at most this many routed rows use the
+// swap-AB kernel (weights on the MMA's M side).
+constexpr int64_t kSwapMaxRows = 1024;
 
 struct Params {
   const int32_t* offsets;
@@ -339,6 +342,214 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Swap-AB variant for few tokens per expert (decode): the weight rows are the
+// MMA's M side (128 per tile) and the expert's tokens its N side (64 per
+// tile), so a tile streams 128 x K of weights once and the tile count is
+// E x N/128 x ceil(n_e / 64) -- enough tiles to cover the SMs even when every
+// expert has only a handful of tokens. Same output as the Out / in-projection
+// epilogue: out[token][n] = r * acc (bf16, k == 1) or per slot in float32.
+constexpr int SW_BN = 64;                      // tokens per tile (MMA N)
+constexpr int SW_STAGES = 8;
+constexpr int SW_A_BYTES = BM * BK * 2;        // 16 KB of weights
+constexpr int SW_B_BYTES = SW_BN * BK * 2;     // 8 KB of tokens
+constexpr int SW_STAGE_BYTES = SW_A_BYTES + SW_B_BYTES;
+constexpr uint32_t SW_TMEM_COLS = 2 * SW_BN;
+
+struct SwapCtl {
+  uint64_t full[SW_STAGES];
+  uint64_t empty[SW_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int tile_start[kMaxExperts + 1];
+  int off[kMaxExperts + 1];
+  int tt[kMaxExperts];  // token tiles per expert
+};
+
+constexpr size_t kSwapSmemBytes = SW_STAGES * SW_STAGE_BYTES + sizeof(SwapCtl) + 1024;
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_swap_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmX, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  SwapCtl& ctl = *reinterpret_cast<SwapCtl*>(smem + SW_STAGES * SW_STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+  const int n_wt = p.N / BM;  // weight-row tiles per expert
+
+  for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = p.offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      const int tt = (ctl.off[e + 1] - ctl.off[e] + SW_BN - 1) / SW_BN;
+      ctl.tt[e] = tt;
+      ctl.tile_start[e] = run;
+      run += tt * n_wt;
+    }
+    ctl.tile_start[E] = run;
+    for (int s = 0; s < SW_STAGES; ++s) {
+      mbar_init(&ctl.full[s], 1);
+      mbar_init(&ctl.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&ctl.tfull[a], 1);
+      mbar_init(&ctl.tempty[a], 4);
+    }
+    mbar_init(&ctl.drain, 1);
+    ctl.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl.tmem_base, SW_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl.tmem_base;
+  const int total = ctl.tile_start[E];
+  const int KB = (p.K + BK - 1) / BK;
+  volatile int* abort_flag = &ctl.abort;
+  // tile -> (expert, weight-row block, token block); weight-row blocks vary
+  // fastest so that CTAs running together share the expert's token rows.
+  auto coords = [&](int tile, int& e, int& w_blk, int& t_blk) {
+    e = 0;
+    while (tile >= ctl.tile_start[e + 1]) ++e;
+    const int local = tile - ctl.tile_start[e];
+    t_blk = local / n_wt;
+    w_blk = local - t_blk * n_wt;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, w_blk, t_blk;
+        coords(tile, e, w_blk, t_blk);
+        const int n0 = w_blk * BM;
+        const int r0 = ctl.off[e] + t_blk * SW_BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * SW_STAGE_BYTES;
+          mbar_arrive_expect_tx(&ctl.full[stage], SW_STAGE_BYTES);
+          tma_load_3d(sa, &tmW, &ctl.full[stage], kb * BK, n0, e);
+          tma_load_2d(sa + SW_A_BYTES, &tmX, &ctl.full[stage], kb * BK, r0);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == SW_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      int never = 0;
+      for (int s = 0; s < SW_STAGES; ++s)
+        if ((issued >> s) & 1u) mbar_wait(&ctl.full[s], (last_par >> s) & 1u, &never, p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, SW_BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        if (!mbar_wait(&ctl.tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * SW_BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&ctl.full[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * SW_STAGE_BYTES);
+          const uint32_t b_addr = a_addr + SW_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                        sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0);
+          mma_commit(&ctl.empty[stage]);
+          if (++stage == SW_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&ctl.tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      mma_commit(&ctl.drain);
+      int never = 0;
+      mbar_wait(&ctl.drain, 0, &never, p.status);
+    }
+  } else {
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int e, w_blk, t_blk;
+      coords(tile, e, w_blk, t_blk);
+      if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * SW_BN);
+      const int n = w_blk * BM + q * 32 + lane;  // this thread's output column
+      const int n_e = ctl.off[e + 1] - ctl.off[e];
+#pragma unroll 1
+      for (int c = 0; c < SW_BN / 32; ++c) {
+        const int j0 = t_blk * SW_BN + c * 32;  // first token of this column chunk
+        if (j0 >= n_e) break;
+        uint32_t a[32];
+        tmem_ld32(t_row + c * 32, a);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j0 + j >= n_e) continue;
+          const int64_t prow = ctl.off[e] + j0 + j;
+          const int64_t slot = p.sorted_slot[prow];
+          const float v = p.topk_w[slot] * __uint_as_float(a[j]);
+          if (MODE == kEpiScaleToken)
+            static_cast<__nv_bfloat16*>(p.out)[(slot / p.k) * p.N + n] = __float2bfloat16_rn(v);
+          else
+            static_cast<float*>(p.out)[slot * p.N + n] = v;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, SW_TMEM_COLS);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -391,6 +602,33 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
                                    cudaStream_t stream) {
   const bool gate = (mode == kEpiGateH || mode == kEpiGateSlots);
   const int tile_n = gate ? 128 : 256;
+  // Few tokens (decode): the swap-AB kernel streams every weight tile once.
+  if (!gate && R <= kSwapMaxRows && N % BM == 0 && K % 8 == 0 && E <= kMaxExperts) {
+    if (R == 0) return cudaSuccess;
+    CUtensorMap tw, tx;
+    if (!make_map(&tw, w0, K, N, E, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tx, a_sorted, K, R, 0, SW_BN)) return cudaErrorInvalidValue;
+    Params p{};
+    p.offsets = offsets;
+    p.sorted_slot = sorted_slot;
+    p.topk_w = topk_w;
+    p.out = out;
+    p.R = R;
+    p.K = K;
+    p.N = N;
+    p.E = E;
+    p.k = k;
+    p.status = status;
+    const int64_t max_tiles = ((R + SW_BN - 1) / SW_BN + E) * static_cast<int64_t>(N / BM);
+    const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
+    auto kern = (mode == kEpiScaleToken) ? tc_swap_gemm_kernel<kEpiScaleToken>
+                                         : tc_swap_gemm_kernel<kEpiScaleSlots>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kSwapSmemBytes));
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, kSwapSmemBytes, stream>>>(tw, tx, p);
+    return cudaGetLastError();
+  }
   if (K % 8 != 0 || N % 128 != 0 || E > kMaxExperts || R >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
   if (R == 0) return cudaSuccess;

@@ -77,15 +77,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KB = (Dm + BK - 1) / BK;
 
-  // W_r^T, zero-padded to EB experts and DW features; |w_e|.
-  for (int i = tid; i < Dm * E; i += kThreads) {
-    const int d = i / E, e = i - d * E;
-    sW[e * DW + d] = __ldg(w_r + i);
+  // W_r^T, zero-padded to EB experts and DW features. Thread t loads whole
+  // feature rows w_r[d][0..E) (contiguous), eight rows in flight at a time.
+  for (int d0 = tid; d0 < Dm; d0 += 8 * kThreads) {
+    float v[8][EB];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int d = d0 + r * kThreads;
+#pragma unroll
+      for (int e = 0; e < EB; ++e)
+        v[r][e] = (d < Dm && e < E) ? __ldg(w_r + static_cast<int64_t>(d) * E + e) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int d = d0 + r * kThreads;
+      if (d < Dm)
+#pragma unroll
+        for (int e = 0; e < EB; ++e) sW[e * DW + d] = v[r][e];
+    }
   }
-  for (int i = tid; i < EB * DW; i += kThreads) {
-    const int e = i / DW, d = i - e * DW;
-    if (e >= E || d >= Dm) sW[i] = 0.f;
-  }
+  for (int e = 0; e < EB; ++e)
+    for (int d = (e < E ? Dm : 0) + tid; d < DW; d += kThreads) sW[e * DW + d] = 0.f;
   for (int i = tid; i < 2 * EB; i += kThreads) (&ctl.hist[0][0])[i] = 0;
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
