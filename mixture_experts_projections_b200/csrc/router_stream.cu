@@ -45,6 +45,7 @@ struct SCtl {
   uint64_t empty[kMaxStages];
   uint64_t part_ready[4][2];
   uint64_t part_free[4][2];
+  uint64_t wload;
   int abort;
   int done[2];
   int hist[2][EB];
@@ -73,31 +74,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + stages * A_BYTES);
   float* sW = reinterpret_cast<float*>(smem + stages * A_BYTES +
-                                       ((sizeof(Ctl) + 15) / 16) * 16);  // [EB][DW]
+                                       ((sizeof(Ctl) + 15) / 16) * 16);  // [DW][EB]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KB = (Dm + BK - 1) / BK;
 
-  // W_r^T, zero-padded to EB experts and DW features. Thread t loads whole
-  // feature rows w_r[d][0..E) (contiguous), eight rows in flight at a time.
-  for (int d0 = tid; d0 < Dm; d0 += 8 * kThreads) {
-    float v[8][EB];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int d = d0 + r * kThreads;
-#pragma unroll
-      for (int e = 0; e < EB; ++e)
-        v[r][e] = (d < Dm && e < E) ? __ldg(w_r + static_cast<int64_t>(d) * E + e) : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int d = d0 + r * kThreads;
-      if (d < Dm)
-#pragma unroll
-        for (int e = 0; e < EB; ++e) sW[e * DW + d] = v[r][e];
-    }
-  }
-  for (int e = 0; e < EB; ++e)
-    for (int d = (e < E ? Dm : 0) + tid; d < DW; d += kThreads) sW[e * DW + d] = 0.f;
+  // W_r as stored, [d_model][E] float32 (E == EB here), copied by the bulk
+  // copy engine; rows d_model .. DW-1 are zero.
+  for (int i = tid; i < (DW - Dm) * EB; i += kThreads) sW[Dm * EB + i] = 0.f;
   for (int i = tid; i < 2 * EB; i += kThreads) (&ctl.hist[0][0])[i] = 0;
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -109,20 +92,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&ctl.part_ready[g][p], 1);
         mbar_init(&ctl.part_free[g][p], 1);
       }
+    mbar_init(&ctl.wload, 1);
     ctl.abort = 0;
     ctl.done[0] = ctl.done[1] = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  volatile int* abort_flag = &ctl.abort;
+  if (tid == 0) {
+    const uint32_t bytes = static_cast<uint32_t>(Dm) * EB * 4u;
+    mbar_arrive_expect_tx(&ctl.wload, bytes);
+    for (uint32_t off = 0; off < bytes; off += 32768u) {
+      const uint32_t n = (bytes - off < 32768u) ? bytes - off : 32768u;
+      bulk_load(reinterpret_cast<uint8_t*>(sW) + off,
+                reinterpret_cast<const uint8_t*>(w_r) + off, n, &ctl.wload);
+    }
+  }
+  {
+    int never = 0;
+    mbar_wait(&ctl.wload, 0, &never, status);
+  }
   for (int e = warp; e < EB; e += kThreads / 32) {
     float q = 0.f;
-    for (int d = lane; d < Dm; d += 32) q = fmaf(sW[e * DW + d], sW[e * DW + d], q);
+    for (int d = lane; d < Dm; d += 32) q = fmaf(sW[d * EB + e], sW[d * EB + e], q);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
     if (lane == 0) ctl.wnorm[e] = sqrtf(q);
   }
   __syncthreads();
-  volatile int* abort_flag = &ctl.abort;
 
   if (warp == 0) {
     // -------------------------------------------------- TMA producer
@@ -193,22 +190,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         stage = 0;
         phase ^= 1u;
       }
-      const int d0 = kb * BK + 32 * h;
+      const float* wrow = sW + static_cast<int64_t>(kb * BK + 32 * h) * EB;
 #pragma unroll
       for (int i = 0; i < 32; ++i) sq = fmaf(xs[i], xs[i], sq);
+      // block partials, two experts per packed FMA; per expert the 32
+      // features are accumulated in order
+      float2 p2[EB / 2];
 #pragma unroll
-      for (int e = 0; e < EB; ++e) {
-        const float4* wp = reinterpret_cast<const float4*>(sW + e * DW + d0);
-        float p = 0.f;
+      for (int e2 = 0; e2 < EB / 2; ++e2) p2[e2] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 wv = wp[i4];
-          p = fmaf(xs[4 * i4], wv.x, p);
-          p = fmaf(xs[4 * i4 + 1], wv.y, p);
-          p = fmaf(xs[4 * i4 + 2], wv.z, p);
-          p = fmaf(xs[4 * i4 + 3], wv.w, p);
+      for (int i = 0; i < 32; ++i) {
+        const float2 xx = make_float2(xs[i], xs[i]);
+        const float4* wv = reinterpret_cast<const float4*>(wrow + i * EB);
+#pragma unroll
+        for (int e4 = 0; e4 < EB / 4; ++e4) {
+          const float4 w4 = wv[e4];
+          p2[2 * e4] = __ffma2_rn(xx, make_float2(w4.x, w4.y), p2[2 * e4]);
+          p2[2 * e4 + 1] = __ffma2_rn(xx, make_float2(w4.z, w4.w), p2[2 * e4 + 1]);
         }
-        acc[e] += p;
+      }
+#pragma unroll
+      for (int e2 = 0; e2 < EB / 2; ++e2) {
+        const float2 a2 = __fadd2_rn(make_float2(acc[2 * e2], acc[2 * e2 + 1]), p2[e2]);
+        acc[2 * e2] = a2.x;
+        acc[2 * e2 + 1] = a2.y;
       }
     }
     if (!ok) break;
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const double xv = static_cast<double>(__bfloat162float(xr[d]));
 #pragma unroll
             for (int q = 0; q < 16; ++q)
-              if (e0 + q < E) a[q] = fma(xv, static_cast<double>(sW[(e0 + q) * DW + d]), a[q]);
+              if (e0 + q < E) a[q] = fma(xv, static_cast<double>(sW[d * EB + e0 + q]), a[q]);
           }
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
@@ -429,16 +434,18 @@ cudaError_t launch_router_stream(const void* x, int64_t T, int Dm, const float* 
                                  const float* bias, int E, int k, int renorm, int32_t* topk_idx,
                                  float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                                  cudaStream_t stream) {
-  if (E <= 4)
+  // W_r is staged as stored ([d_model][E], 16-byte rows): E in {4, 8, 16}.
+  if (reinterpret_cast<uintptr_t>(w_r) & 15u) return cudaErrorNotSupported;
+  if (E == 4)
     return launch_eb<4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                         status, stream);
-  if (E <= 8)
+  if (E == 8)
     return launch_eb<8>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                         status, stream);
-  if (E <= 16)
+  if (E == 16)
     return launch_eb<16>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                          status, stream);
-  return cudaErrorNotSupported;  // wider routers use the register-tiled kernel
+  return cudaErrorNotSupported;  // other expert counts use the register-tiled kernel
 }
 
 }  // namespace rom
