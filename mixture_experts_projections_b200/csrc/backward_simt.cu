@@ -26,6 +26,7 @@ namespace rom {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kRouteBwdThreads = 1024;  // one warp per token, many tokens in flight
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // One warp per token; W_r^T slice [E][DS] staged in shared memory.
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kRouteBwdThreads)
     route_bwd_kernel(int64_t T, int k, int E, int Dm, const int32_t* __restrict__ topk_idx,
                      const float* __restrict__ topk_w, const float* __restrict__ dr_part,
                      int n_parts, const float* __restrict__ dx_slots,
@@ -105,11 +106,11 @@ __global__ void __launch_bounds__(kThreads)
                      __nv_bfloat16* __restrict__ dx, int DS) {
   extern __shared__ float sWt[];  // [E][DS]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = kThreads / 32;
+  const int nw = kRouteBwdThreads / 32;
   for (int D0 = 0; D0 < Dm; D0 += DS) {
     const int dn = min(DS, Dm - D0);
     __syncthreads();
-    for (int i = threadIdx.x; i < dn * E; i += kThreads) {
+    for (int i = threadIdx.x; i < dn * E; i += kRouteBwdThreads) {
       const int d = i / E, e = i - d * E;
       sWt[e * DS + d] = __ldg(w_r + static_cast<int64_t>(D0) * E + i);
     }
@@ -215,8 +216,9 @@ cudaError_t launch_route_bwd(int64_t T, int k, int E, int Dm, const int32_t* top
   cudaError_t err = cudaFuncSetAttribute(route_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((T + 7) / 8, device_sm_count()));
-  route_bwd_kernel<<<grid, kThreads, smem, stream>>>(T, k, E, Dm, topk_idx, topk_w, dr_part,
+  const unsigned grid =
+      static_cast<unsigned>(std::min<int64_t>((T + 31) / 32, device_sm_count()));
+  route_bwd_kernel<<<grid, kRouteBwdThreads, smem, stream>>>(T, k, E, Dm, topk_idx, topk_w, dr_part,
                                                      n_parts, dx_slots, w_r, dlogits,
                                                      static_cast<__nv_bfloat16*>(dx), DS);
   return cudaGetLastError();

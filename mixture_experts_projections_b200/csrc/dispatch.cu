@@ -19,7 +19,7 @@
 namespace rom {
 namespace {
 
-constexpr int kDispatchThreads = 256;
+constexpr int kDispatchThreads = 512;
 constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kMaxGroups = kChunkTokens * kMaxTopK / 32;  // 32-slot groups per chunk
 
