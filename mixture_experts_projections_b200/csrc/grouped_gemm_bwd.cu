@@ -130,8 +130,9 @@ __global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tmB1, const BwdParams p) {
   constexpr bool kW = Mode<MODE>::kWgrad;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
+  // the shared array, not an integer round-trip) so accesses stay LDS/STS.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   SmemCtl& ctl = *reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;

@@ -104,8 +104,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kGate = (MODE == kEpiGateH || MODE == kEpiGateSlots);
   constexpr int kTileN = kGate ? 128 : 256;  // output columns per tile
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
+  // the shared array, not an integer round-trip) so accesses stay LDS/STS.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   SmemCtl& ctl = *reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
@@ -376,8 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_swap_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmX, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
+  // the shared array, not an integer round-trip) so accesses stay LDS/STS.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   SwapCtl& ctl = *reinterpret_cast<SwapCtl*>(smem + SW_STAGES * SW_STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;

@@ -70,8 +70,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                          int DW, float gamma, int* status) {
   using Ctl = SCtl<EB>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
+  // the shared array, not an integer round-trip) so accesses stay LDS/STS.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + stages * A_BYTES);
   float* sW = reinterpret_cast<float*>(smem + stages * A_BYTES +
                                        ((sizeof(Ctl) + 15) / 16) * 16);  // [DW][EB]
