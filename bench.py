@@ -51,6 +51,34 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def csrc_digest():
+    """sha256 over the CUDA sources and the C header (identifies the kernels)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "mixture_experts_projections_b200", "csrc", "*.cu*")))
+    files.append(os.path.join(ROOT, "include", "rom.h"))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from profiles/traffic.json,
+    if that ncu capture was taken on exactly these kernel sources, else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = t.get(workload)
+    if not ent or ent.get("csrc_sha256") != csrc_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
 def block_flops(wl):
     R = wl.T * wl.k
     if wl.kind == "inproj":
@@ -428,15 +456,17 @@ def main():
             ach = inproj_bytes(wl, n_hit) / t_k / 1e9
             roof = {"bound": "hbm", "kernel": "rom_expert_proj(INPROJ)", "achieved": ach,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
-                    "traffic": None, "peak_source": f"{src} hbm_gbs"}
+                    "traffic": profiled_traffic(wl.name), "peak_source": f"{src} hbm_gbs"}
         else:
             t_k = res["part_ms"]["proj0"] / 1e3
             ach = flops["conv_gate"] / t_k / 1e12
             pk = peaks["bf16_tflops"]
             roof = {"bound": "tensor", "kernel": "rom_expert_proj(CONV_GATE)", "achieved": ach,
-                    "peak": pk, "unit": "TFLOP/s", "frac": ach / pk, "traffic": None,
+                    "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                    "traffic": profiled_traffic(wl.name),
                     "peak_source": f"{src} bf16_tflops (burst)"}
         line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "csrc_sha256": csrc_digest(),
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["step_ms"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
