@@ -350,18 +350,36 @@ def run_ours(args, rank, world, local_rank):
     part_ms_eager = {n: float(eager_ms[:, j].mean()) for j, n in enumerate(part_names)}
 
     # ---------------------------------------------- e2e through host buffers
+    # The public host-buffer call: inputs in pinned host memory, result copied
+    # back, copies inside the timed region. Forward-only workloads go through
+    # rom.HostPipeline (chunks over 3 streams: copies overlap the kernels);
+    # the forward + backward step copies x in and O out around one step.
     h_x = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
     h_x.copy_(x)
     h_out = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
+    pipe = None
+    if not wl.backward:
+        pipe = rom.HostPipeline(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device,
+                                De=None if wl.kind == "inproj" else wl.De)
+
+    def e2e_call():
+        if pipe is None:
+            x.copy_(h_x, non_blocking=True)
+            o = step()
+            h_out.copy_(o, non_blocking=True)
+        elif wl.kind == "inproj":
+            pipe.inproj_forward(h_x, w_r, w, h_out, renorm=wl.renorm, bias=bias)
+        else:
+            pipe.block_forward(h_x, w_r, bias, ws["w_conv"], ws["w_gate"], ws["w_out"], h_out,
+                               renorm=wl.renorm)
+
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         flush.zero_()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
         s0.record(stream)
-        x.copy_(h_x, non_blocking=True)
-        o = step()
-        h_out.copy_(o, non_blocking=True)
+        e2e_call()
         s1.record(stream)
         s1.synchronize()
         if i >= args.warmup:

@@ -358,3 +358,89 @@ def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None
     rom_bwd_wgrad(bufs.dhz_sorted, rb.x_sorted[:R], E, rb.offsets, De, bufs.dw_conv, bufs.dw_gate,
                   stream)
     return bufs
+
+
+# ------------------------------------------------------------------ host buffers, pipelined
+
+
+class HostPipeline:
+    """Forward of the block (or the Swimba in-projection) on HOST tensors.
+
+    Tokens are independent, so the batch is cut into chunks (multiples of the
+    128-token routing chunk) that cycle over `nstreams` CUDA streams: the
+    host-to-device copy of one chunk, the kernels of another and the
+    device-to-host copy of a third run at the same time. Each token's result
+    is the one a single call on the whole batch gives. Device buffers are
+    allocated once per stream (torch); the kernels are the library's.
+    """
+
+    def __init__(self, T, Dm, N_out, E, k, dtype, device="cuda", chunks=8, nstreams=3,
+                 De=None):
+        self.T, self.Dm, self.E, self.k = T, Dm, E, k
+        per = -(-T // chunks)
+        self.chunk = max(128, -(-per // 128) * 128)
+        self.streams = [torch.cuda.Stream(device=device) for _ in range(nstreams)]
+        self.x = [torch.empty((self.chunk, Dm), dtype=dtype, device=device) for _ in range(nstreams)]
+        if De is not None:  # RoM block
+            self.bufs = [BlockBuffers(self.chunk, Dm, De, E, k, dtype, device) for _ in range(nstreams)]
+        else:  # in-projection
+            self.bufs = [RoutingBuffers(self.chunk, Dm, E, k, dtype, device) for _ in range(nstreams)]
+            self.out = [torch.empty((self.chunk, N_out), dtype=dtype, device=device)
+                        for _ in range(nstreams)]
+            self.slots = ([torch.empty((self.chunk * k, N_out), dtype=torch.float32, device=device)
+                           for _ in range(nstreams)] if k > 1 else [None] * nstreams)
+
+    def _chunks(self, T):
+        return [(i, min(T, i + self.chunk)) for i in range(0, T, self.chunk)]
+
+    def block_forward(self, x_host, w_r, bias, w_conv, w_gate, w_out, out_host, renorm=False):
+        """x_host [T, Dm] and out_host [T, Dm]: pinned host tensors."""
+        T = x_host.shape[0]
+        cur = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record(cur)
+        for n, (a, b) in enumerate(self._chunks(T)):
+            j = n % len(self.streams)
+            s = self.streams[j]
+            s.wait_event(start)
+            with torch.cuda.stream(s):
+                xd = self.x[j][: b - a]
+                xd.copy_(x_host[a:b], non_blocking=True)
+                bufs = self.bufs[j]
+                if b - a != self.chunk:
+                    bufs = BlockBuffers(b - a, self.Dm, w_conv.shape[1], self.E, self.k, xd.dtype,
+                                        xd.device)
+                blk = block_forward(xd, w_r, bias, w_conv, w_gate, w_out, self.k, renorm, bufs,
+                                    stream=s)
+                out_host[a:b].copy_(blk.out, non_blocking=True)
+        for s in self.streams:
+            ev = torch.cuda.Event()
+            ev.record(s)
+            cur.wait_event(ev)
+        return out_host
+
+    def inproj_forward(self, x_host, w_r, w, out_host, renorm=False, bias=None):
+        """x_host [T, Dm], out_host [T, N_out]: pinned host tensors."""
+        T = x_host.shape[0]
+        cur = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record(cur)
+        for n, (a, b) in enumerate(self._chunks(T)):
+            j = n % len(self.streams)
+            s = self.streams[j]
+            s.wait_event(start)
+            with torch.cuda.stream(s):
+                xd = self.x[j][: b - a]
+                xd.copy_(x_host[a:b], non_blocking=True)
+                bufs = self.bufs[j]
+                if b - a != self.chunk:
+                    bufs = RoutingBuffers(b - a, self.Dm, self.E, self.k, xd.dtype, xd.device)
+                od = self.out[j][: b - a]
+                sl = None if self.slots[j] is None else self.slots[j][: (b - a) * self.k]
+                inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s)
+                out_host[a:b].copy_(od, non_blocking=True)
+        for s in self.streams:
+            ev = torch.cuda.Event()
+            ev.record(s)
+            cur.wait_event(ev)
+        return out_host

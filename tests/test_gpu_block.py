@@ -99,3 +99,25 @@ def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
                            ref)
     assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
+
+
+@pytest.mark.parametrize("T,Dm,De,E,k,renorm", [(5000, 256, 256, 8, 1, False),
+                                                (3000, 256, 384, 8, 2, True)])
+def test_host_pipeline_matches_single_call(T, Dm, De, E, k, renorm):
+    """Chunked, multi-stream forward on pinned host buffers gives every
+    token's routing exactly and its output within the forward's bar."""
+    inp = make_block_inputs(T, Dm, De, E, seed=T, router_std=0.05)
+    d = block_to_dev(inp, "bf16")
+    ref = rom.block_forward(d["x"], d["w_r"], None, d["w_conv"], d["w_gate"], d["w_out"], k=k,
+                            renorm=renorm).out
+    x_h = d["x"].cpu().pin_memory()
+    out_h = torch.empty((T, Dm), dtype=torch.bfloat16, pin_memory=True)
+    pipe = rom.HostPipeline(T, Dm, None, E, k, torch.bfloat16, "cuda", chunks=5, De=De)
+    pipe.block_forward(x_h, d["w_r"], None, d["w_conv"], d["w_gate"], d["w_out"], out_h,
+                       renorm=renorm)
+    torch.cuda.synchronize()
+    assert_close(out_h.float().numpy(), to_np(ref), "bf16", "O (pipelined vs single call)",
+                 magnitude_scaled_abs=True)
+    orc_ref = oracle_block(inp, k, renorm)
+    assert_close(out_h.float().numpy().astype(np.float64), orc_ref["O"], "bf16", "O (pipelined)",
+                 magnitude_scaled_abs=True)
