@@ -378,7 +378,9 @@ class HostPipeline:
                  De=None):
         self.T, self.Dm, self.E, self.k = T, Dm, E, k
         per = -(-T // chunks)
-        self.chunk = max(128, -(-per // 128) * 128)
+        # Chunks of at least 2048 tokens (smaller ones cost more in launches
+        # and stream switches than the overlap saves), at most the batch.
+        self.chunk = min(max(2048, -(-per // 128) * 128), max(128, -(-T // 128) * 128))
         self.streams = [torch.cuda.Stream(device=device) for _ in range(nstreams)]
         self.x = [torch.empty((self.chunk, Dm), dtype=dtype, device=device) for _ in range(nstreams)]
         if De is not None:  # RoM block
@@ -393,54 +395,59 @@ class HostPipeline:
     def _chunks(self, T):
         return [(i, min(T, i + self.chunk)) for i in range(0, T, self.chunk)]
 
-    def block_forward(self, x_host, w_r, bias, w_conv, w_gate, w_out, out_host, renorm=False):
-        """x_host [T, Dm] and out_host [T, Dm]: pinned host tensors."""
-        T = x_host.shape[0]
+    def _run(self, T, body):
+        """body(j, a, b, stream) for every chunk [a, b); one chunk runs on
+        the current stream, several cycle over the pipeline's streams."""
         cur = torch.cuda.current_stream()
+        chunks = self._chunks(T)
+        if len(chunks) == 1:
+            body(0, 0, T, cur)
+            return
         start = torch.cuda.Event()
         start.record(cur)
-        for n, (a, b) in enumerate(self._chunks(T)):
+        for n, (a, b) in enumerate(chunks):
             j = n % len(self.streams)
             s = self.streams[j]
             s.wait_event(start)
             with torch.cuda.stream(s):
-                xd = self.x[j][: b - a]
-                xd.copy_(x_host[a:b], non_blocking=True)
-                bufs = self.bufs[j]
-                if b - a != self.chunk:
-                    bufs = BlockBuffers(b - a, self.Dm, w_conv.shape[1], self.E, self.k, xd.dtype,
-                                        xd.device)
-                blk = block_forward(xd, w_r, bias, w_conv, w_gate, w_out, self.k, renorm, bufs,
-                                    stream=s)
-                out_host[a:b].copy_(blk.out, non_blocking=True)
+                body(j, a, b, s)
         for s in self.streams:
             ev = torch.cuda.Event()
             ev.record(s)
             cur.wait_event(ev)
+
+    def block_forward(self, x_host, w_r, bias, w_conv, w_gate, w_out, out_host, renorm=False):
+        """x_host [T, Dm] and out_host [T, Dm]: pinned host tensors."""
+        T = x_host.shape[0]
+
+        def body(j, a, b, s):
+            xd = self.x[j][: b - a]
+            xd.copy_(x_host[a:b], non_blocking=True)
+            bufs = self.bufs[j]
+            if b - a != self.chunk:
+                bufs = BlockBuffers(b - a, self.Dm, w_conv.shape[1], self.E, self.k, xd.dtype,
+                                    xd.device)
+            blk = block_forward(xd, w_r, bias, w_conv, w_gate, w_out, self.k, renorm, bufs,
+                                stream=s)
+            out_host[a:b].copy_(blk.out, non_blocking=True)
+
+        self._run(T, body)
         return out_host
 
     def inproj_forward(self, x_host, w_r, w, out_host, renorm=False, bias=None):
         """x_host [T, Dm], out_host [T, N_out]: pinned host tensors."""
         T = x_host.shape[0]
-        cur = torch.cuda.current_stream()
-        start = torch.cuda.Event()
-        start.record(cur)
-        for n, (a, b) in enumerate(self._chunks(T)):
-            j = n % len(self.streams)
-            s = self.streams[j]
-            s.wait_event(start)
-            with torch.cuda.stream(s):
-                xd = self.x[j][: b - a]
-                xd.copy_(x_host[a:b], non_blocking=True)
-                bufs = self.bufs[j]
-                if b - a != self.chunk:
-                    bufs = RoutingBuffers(b - a, self.Dm, self.E, self.k, xd.dtype, xd.device)
-                od = self.out[j][: b - a]
-                sl = None if self.slots[j] is None else self.slots[j][: (b - a) * self.k]
-                inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s)
-                out_host[a:b].copy_(od, non_blocking=True)
-        for s in self.streams:
-            ev = torch.cuda.Event()
-            ev.record(s)
-            cur.wait_event(ev)
+
+        def body(j, a, b, s):
+            xd = self.x[j][: b - a]
+            xd.copy_(x_host[a:b], non_blocking=True)
+            bufs = self.bufs[j]
+            if b - a != self.chunk:
+                bufs = RoutingBuffers(b - a, self.Dm, self.E, self.k, xd.dtype, xd.device)
+            od = self.out[j][: b - a]
+            sl = None if self.slots[j] is None else self.slots[j][: (b - a) * self.k]
+            inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s)
+            out_host[a:b].copy_(od, non_blocking=True)
+
+        self._run(T, body)
         return out_host

@@ -102,7 +102,8 @@ def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
 
 
 @pytest.mark.parametrize("T,Dm,De,E,k,renorm", [(5000, 256, 256, 8, 1, False),
-                                                (3000, 256, 384, 8, 2, True)])
+                                                (3000, 256, 384, 8, 2, True),
+                                                (900, 256, 256, 4, 1, False)])
 def test_host_pipeline_matches_single_call(T, Dm, De, E, k, renorm):
     """Chunked, multi-stream forward on pinned host buffers gives every
     token's routing exactly and its output within the forward's bar."""
