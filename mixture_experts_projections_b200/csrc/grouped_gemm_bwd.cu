@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "rom_internal.cuh"
@@ -121,6 +122,73 @@ __device__ __forceinline__ void bwd_tile(const SmemCtl& c, const BwdParams& p, i
     const int local = tile - c.tile_start[e];
     n_blk = local / c.mt[e];
     m_blk = local - n_blk * c.mt[e];
+  }
+}
+
+// Epilogue of one accumulator tile for one warp: thread i reads TMEM lane
+// t_row.lane + i, which holds output row `row` (wgrad: row m of dW_e; dgrad:
+// row `row` of expert e's rows e_begin .. e_end - 1), columns
+// n_blk * 256 .. + 255.
+template <int MODE>
+__device__ __forceinline__ void bwd_epilogue_rows(const BwdParams& p, uint32_t t_row, int e,
+                                                  int e_begin, int e_end, int row, int n_blk) {
+  const int n0 = n_blk * BN;
+  if (MODE == kBwdWgrad) {
+    const bool has_k = e_end > e_begin;
+    const int m = row;
+    float* dst_row = (m < p.m_split)
+                         ? p.out0 + (static_cast<int64_t>(e) * p.m_split + m) * p.N
+                         : p.out1 + (static_cast<int64_t>(e) * (p.M - p.m_split) + (m - p.m_split)) * p.N;
+    const bool valid = m < p.M;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      if (n0 + c * 32 >= p.N) break;
+      uint32_t a[32];
+      tmem_ld32(t_row + c * 32, a);
+      tmem_ld_wait();
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(dst_row + n0 + c * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = has_k ? make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                                       __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  } else {
+    const int row_local = row;
+    const bool valid = row_local < e_end - e_begin;
+    const int64_t prow = static_cast<int64_t>(e_begin) + row_local;
+    const int64_t slot = valid ? p.sorted_slot[prow] : 0;
+    float dot = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      if (n0 + c * 32 >= p.N) break;
+      uint32_t a[32];
+      tmem_ld32(t_row + c * 32, a);
+      tmem_ld_wait();
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(p.out0 + slot * p.N + n0 + c * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                               __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
+        if (MODE == kBwdDgradOut) {
+          const uint4* hp = reinterpret_cast<const uint4*>(p.h_sorted + prow * p.N + n0 + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 hv = __ldg(hp + v);
+            const uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dot = fmaf(__uint_as_float(w[i] << 16), __uint_as_float(a[8 * v + 2 * i]), dot);
+              dot = fmaf(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(a[8 * v + 2 * i + 1]), dot);
+            }
+          }
+        }
+      }
+    }
+    if (MODE == kBwdDgradOut && valid) p.dr_part[slot * p.n_tiles_n + n_blk] = dot;
   }
 }
 
@@ -327,64 +395,8 @@ __global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
       tc_fence_after();
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const int n0 = n_blk * BN;
-      if (kW) {
-        const bool has_k = ctl.off[e + 1] > ctl.off[e];
-        const int m = m_blk * BM + q * 32 + lane;
-        float* dst_row = (m < p.m_split)
-                             ? p.out0 + (static_cast<int64_t>(e) * p.m_split + m) * p.N
-                             : p.out1 + (static_cast<int64_t>(e) * (p.M - p.m_split) + (m - p.m_split)) * p.N;
-        const bool valid = m < p.M;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          if (n0 + c * 32 >= p.N) break;
-          uint32_t a[32];
-          tmem_ld32(t_row + c * 32, a);
-          tmem_ld_wait();
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>(dst_row + n0 + c * 32);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = has_k ? make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                           __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-      } else {
-        const int row_local = m_blk * BM + q * 32 + lane;
-        const bool valid = row_local < ctl.off[e + 1] - ctl.off[e];
-        const int64_t prow = static_cast<int64_t>(ctl.off[e]) + row_local;
-        const int64_t slot = valid ? p.sorted_slot[prow] : 0;
-        float dot = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          if (n0 + c * 32 >= p.N) break;
-          uint32_t a[32];
-          tmem_ld32(t_row + c * 32, a);
-          tmem_ld_wait();
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>(p.out0 + slot * p.N + n0 + c * 32);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                   __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
-            if (MODE == kBwdDgradOut) {
-              const uint4* hp = reinterpret_cast<const uint4*>(p.h_sorted + prow * p.N + n0 + c * 32);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const uint4 hv = __ldg(hp + v);
-                const uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  dot = fmaf(__uint_as_float(w[i] << 16), __uint_as_float(a[8 * v + 2 * i]), dot);
-                  dot = fmaf(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(a[8 * v + 2 * i + 1]), dot);
-                }
-              }
-            }
-          }
-        }
-        if (MODE == kBwdDgradOut && valid) p.dr_part[slot * p.n_tiles_n + n_blk] = dot;
-      }
+      const int row = m_blk * BM + q * 32 + lane;  // output row (wgrad) / expert-local row
+      bwd_epilogue_rows<MODE>(p, t_row, e, ctl.off[e], ctl.off[e + 1], row, n_blk);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.tempty[acc]);
@@ -398,6 +410,357 @@ __global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// SM-pair variant (cluster of two CTAs, tcgen05.mma.cta_group::2, M = 256):
+// CTA v of the pair loads rows 128v .. 128v+127 of the pair tile's A rows
+// (dgrad: 128 sorted rows; wgrad: 128 output rows m, as two 64-wide MN
+// chunks) and B columns n0 + 128v .. + 127 (two 64-wide MN chunks), 32 KB
+// per K step instead of 48 KB, and receives the 128 x 256 accumulator of its
+// own rows in its own TMEM.
+//  Full K blocks: both CTAs' TMA loads complete on CTA 0's full[s], which
+//         CTA 0's producer arms with the bytes of both.
+//  The ragged last K block of an expert (wgrad): each CTA's loads complete
+//         on its own own[s]; its fix-up warp zeroes the K rows past the
+//         expert's end in its own shared memory and then arrives on CTA 0's
+//         ready[s] (two arrivals per phase), on which the MMA issuer waits
+//         with cluster-scope acquire.
+//  full[s], own[s] and ready[s] each advance only on the uses that arm them,
+//  and every waiter tracks a per-stage parity of exactly those uses: a wait
+//  can then never see a barrier one phase behind (which a parity wait would
+//  take for complete).
+// empty[s] and tfull[a] are armed in both CTAs by multicast commits; CTA 0's
+// tempty[a] takes the arrivals of all 8 epilogue warps. Both CTAs end at a
+// cluster barrier that every path reaches after bounded waits.
+constexpr int PM = 256;
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int P_B_BYTES = 128 * BK * 2;  // 16 KB: two 64-wide MN chunks
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+
+struct PairCtl {
+  uint64_t full[P_STAGES];
+  uint64_t own[P_STAGES];
+  uint64_t ready[P_STAGES];
+  uint64_t empty[P_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int tile_start[kMaxExperts + 1];
+  int off[kMaxExperts + 1];
+  int mt[kMaxExperts];
+};
+
+constexpr size_t kPairSmemBytes = P_STAGES * P_STAGE_BYTES + sizeof(PairCtl) + 1024;
+
+template <int MODE>
+__global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
+    tc_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB0,
+                       const __grid_constant__ CUtensorMap tmB1, const BwdParams p) {
+  constexpr bool kW = Mode<MODE>::kWgrad;
+  extern __shared__ uint8_t smem_raw[];
+  // Same 1024-byte aligned offset in both CTAs: the pair MMA reads the peer's
+  // operands at the leader's offsets.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  PairCtl& ctl = *reinterpret_cast<PairCtl*>(smem + P_STAGES * P_STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+
+  for (int i = threadIdx.x; i <= E; i += Mode<MODE>::kThreads) ctl.off[i] = p.offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      const int mt = (ctl.off[e + 1] - ctl.off[e] + PM - 1) / PM;
+      ctl.mt[e] = mt;
+      ctl.tile_start[e] = run;
+      run += kW ? p.m_tiles * p.n_tiles_n : mt * p.n_tiles_n;
+    }
+    ctl.tile_start[E] = run;
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&ctl.full[s], 1);
+      mbar_init(&ctl.own[s], 1);
+      mbar_init(&ctl.ready[s], 2);
+      mbar_init(&ctl.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&ctl.tfull[a], 1);
+      mbar_init(&ctl.tempty[a], 8);
+    }
+    mbar_init(&ctl.drain, 1);
+    ctl.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&ctl.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised in both CTAs before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = ctl.tmem_base;
+  const int total = ctl.tile_start[E];
+  volatile int* abort_flag = &ctl.abort;
+
+  auto tile_of = [&](int tile, int& e, int& m_blk, int& n_blk) {
+    if (kW) {
+      const int per_e = p.m_tiles * p.n_tiles_n;
+      e = tile / per_e;
+      const int rem = tile - e * per_e;
+      n_blk = rem / p.m_tiles;
+      m_blk = rem - n_blk * p.m_tiles;
+    } else {
+      e = 0;
+      while (tile >= ctl.tile_start[e + 1]) ++e;
+      const int local = tile - ctl.tile_start[e];
+      n_blk = local / ctl.mt[e];
+      m_blk = local - n_blk * ctl.mt[e];
+    }
+  };
+  auto tile_kb = [&](int e) -> int {
+    if (kW) return (ctl.off[e + 1] - ctl.off[e] + BK - 1) / BK;
+    return (p.K + BK - 1) / BK;
+  };
+  const int half = static_cast<int>(rank) * 128;
+
+  // wgrad: is K block kb of expert e the expert's ragged last block?
+  auto ragged = [&](int e, int kb) -> bool {
+    return kW && (ctl.off[e + 1] - ctl.off[e] - kb * BK) < BK;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      const uint32_t full0 = mapa_shared(smem_u32(&ctl.full[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      // Per-stage parities: full[s] advances on full-block uses only, own[s]
+      // on ragged-block uses only (so no waiter can be a phase behind).
+      uint32_t full_par = 0, own_par = 0;
+      uint32_t full_used = 0, own_used = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        int e, m_blk, n_blk;
+        tile_of(tile, e, m_blk, n_blk);
+        const int KB = tile_kb(e);
+        const int nb = n_blk * BN + half;  // this CTA's first B column
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * P_STAGE_BYTES;
+          uint8_t* sb = sa + P_A_BYTES;
+          const uint32_t fb = full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
+          const bool own = ragged(e, kb);  // loads complete on this CTA's own[s]
+          if (own) {
+            mbar_arrive_expect_tx(&ctl.own[stage], P_STAGE_BYTES);
+          } else if (leader) {
+            mbar_arrive_expect_tx(&ctl.full[stage], 2 * P_STAGE_BYTES);
+          }
+          if (kW) {
+            const int r0 = ctl.off[e] + kb * BK;
+            const int m0 = m_blk * PM + half;
+            if (own) {
+              uint64_t* bar = &ctl.own[stage];
+              tma_load_2d(sa, &tmA, bar, m0, r0);
+              tma_load_2d(sa + CHUNK_BYTES, &tmA, bar, m0 + 64, r0);
+              tma_load_2d(sb, &tmB0, bar, nb, r0);
+              tma_load_2d(sb + CHUNK_BYTES, &tmB0, bar, nb + 64, r0);
+            } else {
+              tma_load_2d_pair(sa, &tmA, fb, m0, r0);
+              tma_load_2d_pair(sa + CHUNK_BYTES, &tmA, fb, m0 + 64, r0);
+              tma_load_2d_pair(sb, &tmB0, fb, nb, r0);
+              tma_load_2d_pair(sb + CHUNK_BYTES, &tmB0, fb, nb + 64, r0);
+            }
+          } else {
+            const int row0 = ctl.off[e] + m_blk * PM + half;
+            tma_load_2d_pair(sa, &tmA, fb, kb * BK, row0);
+            const bool second = (MODE == kBwdDgradIn) && kb >= p.kb_split;
+            const CUtensorMap* mb = second ? &tmB1 : &tmB0;
+            const int kk = second ? kb - p.kb_split : kb;
+            tma_load_3d_pair(sb, mb, fb, nb, kk * BK, e);
+            tma_load_3d_pair(sb + CHUNK_BYTES, mb, fb, nb + 64, kk * BK, e);
+          }
+          if (own) {
+            own_used |= 1u << stage;
+            own_par ^= 1u << stage;
+          } else if (leader) {
+            full_used |= 1u << stage;
+            full_par ^= 1u << stage;
+          }
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Loads that complete on this CTA's barriers have all landed (the last
+      // armed phase of a barrier has the parity before its last toggle).
+      int never = 0;
+      for (int s = 0; s < P_STAGES; ++s) {
+        if ((full_used >> s) & 1u)
+          mbar_wait(&ctl.full[s], ((full_par >> s) & 1u) ^ 1u, &never, p.status);
+        if ((own_used >> s) & 1u)
+          mbar_wait(&ctl.own[s], ((own_par >> s) & 1u) ^ 1u, &never, p.status);
+      }
+      if (!leader && !ok) {
+        // Aborted: this CTA's other loads complete on the leader's barriers,
+        // which it cannot wait on; give copies in flight a fixed time to land.
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (CTA 0)
+      const uint32_t idesc = idesc_bf16(PM, BN, kW, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t ready_par = 0;  // per-stage parity of ready[s] (ragged uses only)
+      uint32_t full_par = 0;   // per-stage parity of full[s] (full-block uses only)
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        int e, m_blk, n_blk;
+        tile_of(tile, e, m_blk, n_blk);
+        const int KB = tile_kb(e);
+        if (!mbar_wait(&ctl.tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          bool got;
+          if (ragged(e, kb)) {
+            // both CTAs' fix-up warps have zeroed the rows past the expert
+            got = mbar_wait_cluster(&ctl.ready[stage], (ready_par >> stage) & 1u, abort_flag,
+                                    p.status);
+            ready_par ^= 1u << stage;
+          } else {
+            got = mbar_wait(&ctl.full[stage], (full_par >> stage) & 1u, abort_flag, p.status);
+            full_par ^= 1u << stage;
+          }
+          if (!got) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * P_STAGE_BYTES);
+          const uint32_t b_addr = a_addr + P_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = kW ? sw128_mn_desc(a_addr + kk * 2048, CHUNK_BYTES)
+                                   : sw128_kmajor_desc(a_addr + kk * 32);
+            const uint64_t bd = sw128_mn_desc(b_addr + kk * 2048, CHUNK_BYTES);
+            mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          mma_commit_pair_mc(&ctl.empty[stage], 0x3);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&ctl.tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      mma_commit_pair(&ctl.drain);
+      int never = 0;
+      mbar_wait(&ctl.drain, 0, &never, p.status);
+    }
+  } else if (warp == 6) {
+    // -------------------------------------------------- fix-up warp (wgrad, both CTAs)
+    // Only the ragged last K block of an expert passes through here: after
+    // this CTA's own loads land, zero its rows past the expert's end, then
+    // report to CTA 0's ready[s].
+    const uint32_t ready0 = mapa_shared(smem_u32(&ctl.ready[0]), 0);
+    int stage = 0;
+    uint32_t own_par = 0;  // per-stage parity of own[s]
+    bool ok = true;
+    for (int tile = pair; tile < total && ok; tile += npairs) {
+      int e, m_blk, n_blk;
+      tile_of(tile, e, m_blk, n_blk);
+      const int n_e = ctl.off[e + 1] - ctl.off[e];
+      const int KB = tile_kb(e);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (ragged(e, kb)) {
+          const uint32_t par = (own_par >> stage) & 1u;
+          own_par ^= 1u << stage;
+          if (!mbar_wait(&ctl.own[stage], par, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          // zero lines valid..63 of the 4 chunks (2 of A, 2 of B)
+          const int valid = n_e - kb * BK;
+          uint8_t* base = smem + stage * P_STAGE_BYTES;
+          const int per_chunk = (BK - valid) * 8;  // 16-byte pieces
+          for (int i = lane; i < 4 * per_chunk; i += 32) {
+            const int c = i / per_chunk, q = i - c * per_chunk;
+            uint4* dst = reinterpret_cast<uint4*>(base + c * CHUNK_BYTES + valid * 128) + q;
+            *dst = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader)
+              mbar_arrive(&ctl.ready[stage]);
+            else
+              mbar_arrive_remote(ready0 + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+          }
+        }
+        if (++stage == P_STAGES) stage = 0;
+      }
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      int e, m_blk, n_blk;
+      tile_of(tile, e, m_blk, n_blk);
+      if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int row = m_blk * PM + half + q * 32 + lane;
+      bwd_epilogue_rows<MODE>(p, t_row, e, ctl.off[e], ctl.off[e + 1], row, n_blk);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&ctl.tempty[acc]);
+        else
+          mbar_arrive_remote(tempty0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA releases TMEM or exits while the other works
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -445,6 +808,52 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   return cudaGetLastError();
 }
 
+template <int MODE>
+cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                             const BwdParams& p, int64_t max_tiles, cudaStream_t stream) {
+  auto kern = tc_bwd_pair_kernel<MODE>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kPairSmemBytes));
+  if (err != cudaSuccess) return err;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(Mode<MODE>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Co-resident pairs on this device (one CTA per SM), cached per device and mode.
+  static int pairs_cache[64] = {0};
+  int dev = 0;
+  err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int pairs = (dev < 64) ? pairs_cache[dev] : 0;
+  if (pairs == 0) {
+    cfg.gridDim = dim3(2 * 64, 1, 1);
+    err = cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg);
+    if (err != cudaSuccess) return err;
+    if (pairs <= 0) return cudaErrorNotSupported;
+    if (dev < 64) pairs_cache[dev] = pairs;
+  }
+  const int64_t n = std::min<int64_t>(pairs, max_tiles);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * n), 1, 1);
+  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, p);
+}
+
+// The SM-pair kernels serve the backward GEMMs unless ROM_TC_PAIR=0.
+bool use_pair_kernel() {
+  static int v = -1;
+  if (v < 0) {
+    const char* s = getenv("ROM_TC_PAIR");
+    v = (s && s[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 BwdParams base_params(const int32_t* offsets, int64_t R, int E, int k, int* status) {
   BwdParams p{};
   p.offsets = offsets;
@@ -475,6 +884,9 @@ cudaError_t launch_bwd_dgrad_out(const void* rdo_sorted, int64_t R, int Dm, cons
   p.K = Dm;
   p.N = De;
   p.n_tiles_n = De / BN;
+  if (use_pair_kernel())
+    return launch_pair_mode<kBwdDgradOut>(
+        ta, tb, tb, p, ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n), stream);
   const int64_t max_tiles = ((R + BM - 1) / BM + E) * static_cast<int64_t>(p.n_tiles_n);
   const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
   return launch_mode<kBwdDgradOut>(ta, tb, tb, p, grid, stream);
@@ -499,6 +911,9 @@ cudaError_t launch_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const
   p.N = Dm;
   p.kb_split = De / BK;
   p.n_tiles_n = Dm / BN;
+  if (use_pair_kernel())
+    return launch_pair_mode<kBwdDgradIn>(
+        ta, tb0, tb1, p, ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n), stream);
   const int64_t max_tiles = ((R + BM - 1) / BM + E) * static_cast<int64_t>(p.n_tiles_n);
   const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
   return launch_mode<kBwdDgradIn>(ta, tb0, tb1, p, grid, stream);
@@ -518,8 +933,13 @@ cudaError_t launch_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, 
   p.M = M;
   p.N = N;
   p.m_split = m_split;
-  p.m_tiles = M / BM;
   p.n_tiles_n = N / BN;
+  if (use_pair_kernel()) {
+    p.m_tiles = (M + PM - 1) / PM;
+    return launch_pair_mode<kBwdWgrad>(
+        ta, tb, tb, p, static_cast<int64_t>(E) * p.m_tiles * p.n_tiles_n, stream);
+  }
+  p.m_tiles = M / BM;
   const int64_t tiles = static_cast<int64_t>(E) * p.m_tiles * p.n_tiles_n;
   const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), tiles));
   return launch_mode<kBwdWgrad>(ta, tb, tb, p, grid, stream);

@@ -10,19 +10,24 @@
 // from `offsets` (no host synchronisation). Tiles never straddle experts;
 // rows past an expert's end are computed and discarded at the store.
 //
-// Tile: 128 rows x 256 accumulator columns x 64-element K steps.
-//   Conv+Gate: the 256 columns are 128 columns of W_in next to the same 128
-//   columns of W_g, so one MMA of N = 256 yields u and z side by side, and the
-//   epilogue forms h = u * SiLU(z) (top-1) or stores u and z per slot (top-k).
+// Tile: 256 rows x 256 accumulator columns x 64-element K steps, computed
+// by a pair of CTAs on two SMs (a 2-CTA cluster, tcgen05.mma.cta_group::2):
+// each CTA holds 128 of the rows and half of the 256 B columns in its shared
+// memory and receives its rows' 128 x 256 fp32 accumulator in its own TMEM.
+//   Conv+Gate: the 256 columns are 128 columns of W_in (held by CTA 0) next
+//   to the same 128 columns of W_g (CTA 1), so one MMA of N = 256 yields u
+//   and z side by side, and the epilogue forms h = u * SiLU(z) (top-1) or
+//   stores u and z per slot (top-k).
 //   Out / in-projection: 256 output columns, scaled by r in the epilogue (a
 //   last tile of 128 columns when N % 256 == 128: the weight rows past N are
 //   zero-filled by TMA and those columns are not stored).
-// CTA: persistent (one per SM), 6 warps:
-//   warp 0  TMA producer (one thread), 4-stage shared-memory ring (48 KB/stage)
-//   warp 1  TMEM allocator and MMA issuer (one thread)
+// CTA: persistent (one pair of CTAs per pair of SMs), 6 warps:
+//   warp 0  TMA producer (one thread), 6-stage ring (32 KB/stage per CTA)
+//   warp 1  TMEM allocator; in CTA 0 also the MMA issuer (one thread)
 //   warps 2-5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile run
 // while the MMAs of the next tile proceed. Every wait is bounded.
+// Few routed rows (decode) take a swap-AB kernel instead (below).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -39,10 +44,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int UMMA_N = 256;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;      // 16 KB
-constexpr int B_BYTES = UMMA_N * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * UMMA_N;
 constexpr int kThreads = 192;
 // Out / in-projection calls with at most this many routed rows use the
@@ -63,9 +64,130 @@ struct Params {
   int* status;
 };
 
-struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+// u * SiLU(z) = u * z / (1 + e^-z), with the fast exp and divide intrinsics:
+// their relative error (~1e-6) is far below the bf16 rounding of h (2^-9),
+// and for z < -88 (e^-z = inf) the quotient is 0 as SiLU's limit.
+__device__ __forceinline__ float silu_gate(float u, float z) {
+  return u * __fdividef(z, 1.0f + __expf(-z));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Epilogue of one accumulator tile for one warp: thread i reads TMEM lane
+// t_row.lane + i, i.e. sorted row `prow` (stored only when `valid`), output
+// columns n0 .. n0 + (128 for the gate modes, 256 otherwise) - 1.
+template <int MODE>
+__device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, bool valid,
+                                              int64_t prow, int n0) {
+  if (MODE == kEpiGateH) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32], z[32];
+      tmem_ld32(t_row + c * 32, u);
+      tmem_ld32(t_row + 128 + c * 32, z);
+      tmem_ld_wait();
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + prow * p.N + n0 + c * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 w;
+          w.x = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 0]), __uint_as_float(z[8 * v + 0])),
+                          silu_gate(__uint_as_float(u[8 * v + 1]), __uint_as_float(z[8 * v + 1])));
+          w.y = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 2]), __uint_as_float(z[8 * v + 2])),
+                          silu_gate(__uint_as_float(u[8 * v + 3]), __uint_as_float(z[8 * v + 3])));
+          w.z = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 4]), __uint_as_float(z[8 * v + 4])),
+                          silu_gate(__uint_as_float(u[8 * v + 5]), __uint_as_float(z[8 * v + 5])));
+          w.w = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 6]), __uint_as_float(z[8 * v + 6])),
+                          silu_gate(__uint_as_float(u[8 * v + 7]), __uint_as_float(z[8 * v + 7])));
+          dst[v] = w;
+        }
+      }
+    }
+  } else if (MODE == kEpiGateSlots) {
+    float* out = static_cast<float*>(p.out);
+    const int64_t slot = valid ? p.sorted_slot[prow] : 0;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32], z[32];
+      tmem_ld32(t_row + c * 32, u);
+      tmem_ld32(t_row + 128 + c * 32, z);
+      tmem_ld_wait();
+      if (valid) {
+        uint4* du = reinterpret_cast<uint4*>(out + slot * p.N + n0 + c * 32);
+        uint4* dz = reinterpret_cast<uint4*>(out + (p.R + slot) * p.N + n0 + c * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          du[v] = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+          dz[v] = make_uint4(z[4 * v], z[4 * v + 1], z[4 * v + 2], z[4 * v + 3]);
+        }
+      }
+    }
+  } else {
+    const int64_t slot = valid ? p.sorted_slot[prow] : 0;
+    const float r = valid ? p.topk_w[slot] : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      if (n0 + c * 32 >= p.N) break;  // partial last tile (N % 256 == 128)
+      uint32_t a[32];
+      tmem_ld32(t_row + c * 32, a);
+      tmem_ld_wait();
+      if (valid) {
+        if (MODE == kEpiScaleToken) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+          uint4* dst = reinterpret_cast<uint4*>(out + (slot / p.k) * p.N + n0 + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16(r * __uint_as_float(a[8 * v + 0]), r * __uint_as_float(a[8 * v + 1]));
+            w.y = pack_bf16(r * __uint_as_float(a[8 * v + 2]), r * __uint_as_float(a[8 * v + 3]));
+            w.z = pack_bf16(r * __uint_as_float(a[8 * v + 4]), r * __uint_as_float(a[8 * v + 5]));
+            w.w = pack_bf16(r * __uint_as_float(a[8 * v + 6]), r * __uint_as_float(a[8 * v + 7]));
+            dst[v] = w;
+          }
+        } else {
+          float* out = static_cast<float*>(p.out);
+          float4* dst = reinterpret_cast<float4*>(out + slot * p.N + n0 + c * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(r * __uint_as_float(a[4 * v]), r * __uint_as_float(a[4 * v + 1]),
+                                 r * __uint_as_float(a[4 * v + 2]), r * __uint_as_float(a[4 * v + 3]));
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// SM-pair variant (cluster of two CTAs, tcgen05.mma.cta_group::2): a pair
+// tile is 256 rows x 256 accumulator columns. CTA v of the pair loads rows
+// 128v .. 128v+127 of the tile's A rows and half of the B rows (Conv+Gate:
+// CTA 0 the 128 W_in columns, CTA 1 the same 128 W_g columns; Out: CTA v
+// the output columns 128v .. 128v+127), so each SM streams 32 KB per K step
+// instead of 48 KB, and the 128 x 256 accumulator of its own rows lands in
+// its own TMEM, where its own epilogue warps read it as in the one-CTA
+// kernel. Protocol:
+//   full[s]   lives in CTA 0: CTA 0's producer arms it with both CTAs'
+//             bytes; both producers' TMA loads complete on it.
+//   empty[s]  one per CTA: the MMA commit arrives on both (multicast).
+//   tfull[a]  one per CTA: the commit after a tile's last MMA, multicast.
+//   tempty[a] lives in CTA 0: the 4 epilogue warps of each CTA arrive
+//             (CTA 1's through the cluster window).
+// A CTA never exits while the other may still touch its shared memory or
+// TMEM: both end at a cluster barrier that every path reaches after bounded
+// waits.
+constexpr int PM = 256;                      // rows per pair tile
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = BM * BK * 2;       // 16 KB: this CTA's 128 rows
+constexpr int P_B_BYTES = 128 * BK * 2;      // 16 KB: this CTA's half of B
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+
+struct PairCtl {
+  uint64_t full[P_STAGES];
+  uint64_t empty[P_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -76,59 +198,45 @@ struct SmemCtl {
   int mt[kMaxExperts];
 };
 
-constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(SmemCtl) + 1024;
-
-__device__ __forceinline__ void tile_coords(const SmemCtl& c, int tile, int& e, int& m_blk,
-                                            int& n_blk) {
-  e = 0;
-  while (tile >= c.tile_start[e + 1]) ++e;
-  const int local = tile - c.tile_start[e];
-  n_blk = local / c.mt[e];
-  m_blk = local - n_blk * c.mt[e];
-}
-
-__device__ __forceinline__ float silu_gate(float u, float z) {
-  return u * (z / (1.0f + expf(-z)));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
+constexpr size_t kPairSmemBytes = P_STAGES * P_STAGE_BYTES + sizeof(PairCtl) + 1024;
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB0,
-                           const __grid_constant__ CUtensorMap tmB1, const Params p) {
+    tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const Params p) {
   constexpr bool kGate = (MODE == kEpiGateH || MODE == kEpiGateSlots);
   constexpr int kTileN = kGate ? 128 : 256;  // output columns per tile
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
-  // the shared array, not an integer round-trip) so accesses stay LDS/STS.
+  // Same 1024-byte aligned offset in both CTAs (same kernel, same static
+  // layout), as the pair MMA reads the peer's operands at the leader's offsets.
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  SmemCtl& ctl = *reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
+  PairCtl& ctl = *reinterpret_cast<PairCtl*>(smem + P_STAGES * P_STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
 
   for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = p.offsets[i];
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = 0;
     for (int e = 0; e < E; ++e) {
-      const int mt = (ctl.off[e + 1] - ctl.off[e] + BM - 1) / BM;
+      const int mt = (ctl.off[e + 1] - ctl.off[e] + PM - 1) / PM;
       ctl.mt[e] = mt;
       ctl.tile_start[e] = run;
       run += mt * p.n_tiles_n;
     }
     ctl.tile_start[E] = run;
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < P_STAGES; ++s) {
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ctl.tfull[a], 1);
-      mbar_init(&ctl.tempty[a], 4);
+      mbar_init(&ctl.tempty[a], 8);
     }
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
@@ -136,72 +244,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB0);
-    if (kGate) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(kGate && !leader ? &tmB1 : &tmB0);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&ctl.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers initialised in both CTAs before any remote use
   tc_fence_after();
   const uint32_t tmem_base = ctl.tmem_base;
   const int total = ctl.tile_start[E];
   const int KB = (p.K + BK - 1) / BK;
   volatile int* abort_flag = &ctl.abort;
 
+  auto coords = [&](int tile, int& e, int& m_blk, int& n_blk) {
+    e = 0;
+    while (tile >= ctl.tile_start[e + 1]) ++e;
+    const int local = tile - ctl.tile_start[e];
+    n_blk = local / ctl.mt[e];
+    m_blk = local - n_blk * ctl.mt[e];
+  };
+
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer (both CTAs)
+      const CUtensorMap* tmB = (kGate && !leader) ? &tmB1 : &tmB0;
+      const uint32_t full0 = mapa_shared(smem_u32(&ctl.full[0]), 0);
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0, last_par = 0;  // per-stage: ever armed, parity of last arming
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      uint32_t issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
         int e, m_blk, n_blk;
-        tile_coords(ctl, tile, e, m_blk, n_blk);
-        const int row0 = ctl.off[e] + m_blk * BM;
-        const int n0 = n_blk * kTileN;
-        bool ok = true;
+        coords(tile, e, m_blk, n_blk);
+        const int row0 = ctl.off[e] + m_blk * PM + static_cast<int>(rank) * BM;
+        const int brow0 = kGate ? n_blk * 128 : n_blk * 256 + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(&ctl.full[stage], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &ctl.full[stage], kb * BK, row0);
-          if (kGate) {
-            tma_load_3d(sb, &tmB0, &ctl.full[stage], kb * BK, n0, e);
-            tma_load_3d(sb + B_BYTES / 2, &tmB1, &ctl.full[stage], kb * BK, n0, e);
-          } else {
-            tma_load_3d(sb, &tmB0, &ctl.full[stage], kb * BK, n0, e);
-          }
+          uint8_t* sa = smem + stage * P_STAGE_BYTES;
+          const uint32_t fb = full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
+          if (leader) mbar_arrive_expect_tx(&ctl.full[stage], 2 * P_STAGE_BYTES);
+          tma_load_2d_pair(sa, &tmA, fb, kb * BK, row0);
+          tma_load_3d_pair(sa + P_A_BYTES, tmB, fb, kb * BK, brow0, e);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (!ok) break;
       }
-      // No TMA write may still be landing when the CTA exits.
-      int never = 0;
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u) mbar_wait(&ctl.full[s], (last_par >> s) & 1u, &never, p.status);
+      if (leader) {
+        // Every load of both CTAs has landed before the pair can exit.
+        int never = 0;
+        for (int s = 0; s < P_STAGES; ++s)
+          if ((issued >> s) & 1u) mbar_wait(&ctl.full[s], (last_par >> s) & 1u, &never, p.status);
+      } else if (!ok) {
+        // Aborted: this CTA's loads complete on the leader's barriers, which
+        // it cannot wait on; give copies in flight a fixed time to land.
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+      }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, UMMA_N);
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (CTA 0)
+      const uint32_t idesc = idesc_bf16_f32(PM, UMMA_N);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = pair; tile < total && ok; tile += npairs) {
         if (!mbar_wait(&ctl.tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * UMMA_N);
@@ -211,125 +330,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
+          const uint32_t a_addr = smem_u32(smem + stage * P_STAGE_BYTES);
+          const uint32_t b_addr = a_addr + P_A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
-                        sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0);
+            mma_bf16_ss_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                             sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0);
           }
-          mma_commit(&ctl.empty[stage]);
-          if (++stage == STAGES) {
+          mma_commit_pair_mc(&ctl.empty[stage], 0x3);
+          if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&ctl.tfull[acc]);
+        mma_commit_pair_mc(&ctl.tfull[acc], 0x3);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // Every issued MMA has completed before TMEM is released.
-      mma_commit(&ctl.drain);
+      mma_commit_pair(&ctl.drain);
       int never = 0;
       mbar_wait(&ctl.drain, 0, &never, p.status);
     }
   } else {
     // -------------------------------------------------- epilogue (warps 2..5)
     const int q = warp & 3;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int tile = pair; tile < total; tile += npairs) {
       int e, m_blk, n_blk;
-      tile_coords(ctl, tile, e, m_blk, n_blk);
+      coords(tile, e, m_blk, n_blk);
       if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
-      const int row_local = m_blk * BM + q * 32 + lane;
+      const int row_local = m_blk * PM + static_cast<int>(rank) * BM + q * 32 + lane;
       const bool valid = row_local < ctl.off[e + 1] - ctl.off[e];
       const int64_t prow = static_cast<int64_t>(ctl.off[e]) + row_local;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * UMMA_N);
-      const int n0 = n_blk * kTileN;
-      if (MODE == kEpiGateH) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t u[32], z[32];
-          tmem_ld32(t_row + c * 32, u);
-          tmem_ld32(t_row + 128 + c * 32, z);
-          tmem_ld_wait();
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + prow * p.N + n0 + c * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 0]), __uint_as_float(z[8 * v + 0])),
-                              silu_gate(__uint_as_float(u[8 * v + 1]), __uint_as_float(z[8 * v + 1])));
-              w.y = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 2]), __uint_as_float(z[8 * v + 2])),
-                              silu_gate(__uint_as_float(u[8 * v + 3]), __uint_as_float(z[8 * v + 3])));
-              w.z = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 4]), __uint_as_float(z[8 * v + 4])),
-                              silu_gate(__uint_as_float(u[8 * v + 5]), __uint_as_float(z[8 * v + 5])));
-              w.w = pack_bf16(silu_gate(__uint_as_float(u[8 * v + 6]), __uint_as_float(z[8 * v + 6])),
-                              silu_gate(__uint_as_float(u[8 * v + 7]), __uint_as_float(z[8 * v + 7])));
-              dst[v] = w;
-            }
-          }
-        }
-      } else if (MODE == kEpiGateSlots) {
-        float* out = static_cast<float*>(p.out);
-        const int64_t slot = valid ? p.sorted_slot[prow] : 0;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t u[32], z[32];
-          tmem_ld32(t_row + c * 32, u);
-          tmem_ld32(t_row + 128 + c * 32, z);
-          tmem_ld_wait();
-          if (valid) {
-            uint4* du = reinterpret_cast<uint4*>(out + slot * p.N + n0 + c * 32);
-            uint4* dz = reinterpret_cast<uint4*>(out + (p.R + slot) * p.N + n0 + c * 32);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              du[v] = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
-              dz[v] = make_uint4(z[4 * v], z[4 * v + 1], z[4 * v + 2], z[4 * v + 3]);
-            }
-          }
-        }
-      } else {
-        const int64_t slot = valid ? p.sorted_slot[prow] : 0;
-        const float r = valid ? p.topk_w[slot] : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          if (n0 + c * 32 >= p.N) break;  // partial last tile (N % 256 == 128)
-          uint32_t a[32];
-          tmem_ld32(t_row + c * 32, a);
-          tmem_ld_wait();
-          if (valid) {
-            if (MODE == kEpiScaleToken) {
-              __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-              uint4* dst = reinterpret_cast<uint4*>(out + (slot / p.k) * p.N + n0 + c * 32);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint4 w;
-                w.x = pack_bf16(r * __uint_as_float(a[8 * v + 0]), r * __uint_as_float(a[8 * v + 1]));
-                w.y = pack_bf16(r * __uint_as_float(a[8 * v + 2]), r * __uint_as_float(a[8 * v + 3]));
-                w.z = pack_bf16(r * __uint_as_float(a[8 * v + 4]), r * __uint_as_float(a[8 * v + 5]));
-                w.w = pack_bf16(r * __uint_as_float(a[8 * v + 6]), r * __uint_as_float(a[8 * v + 7]));
-                dst[v] = w;
-              }
-            } else {
-              float* out = static_cast<float*>(p.out);
-              float4* dst = reinterpret_cast<float4*>(out + slot * p.N + n0 + c * 32);
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(r * __uint_as_float(a[4 * v]), r * __uint_as_float(a[4 * v + 1]),
-                                     r * __uint_as_float(a[4 * v + 2]), r * __uint_as_float(a[4 * v + 3]));
-            }
-          }
-        }
-      }
+      epilogue_rows<MODE>(p, t_row, valid, prow, n_blk * kTileN);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.tempty[acc]);
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&ctl.tempty[acc]);
+        else
+          mbar_arrive_remote(tempty0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -337,9 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // neither CTA releases TMEM or exits while the other works
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -585,14 +634,39 @@ bool make_map(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int exp
 }
 
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const Params& p, int grid, cudaStream_t stream) {
-  auto kern = tc_grouped_gemm_kernel<MODE>;
+cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                             const Params& p, int64_t max_tiles, cudaStream_t stream) {
+  auto kern = tc_pair_gemm_kernel<MODE>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
+                                         static_cast<int>(kPairSmemBytes));
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(a, b0, b1, p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Co-resident pairs on this device (one CTA per SM), cached per device.
+  static int pairs_cache[64] = {0};
+  int dev = 0;
+  err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int pairs = (dev < 64) ? pairs_cache[dev] : 0;
+  if (pairs == 0) {
+    cfg.gridDim = dim3(2 * 64, 1, 1);
+    err = cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg);
+    if (err != cudaSuccess) return err;
+    if (pairs <= 0) return cudaErrorNotSupported;
+    if (dev < 64) pairs_cache[dev] = pairs;
+  }
+  const int64_t n = std::min<int64_t>(pairs, max_tiles);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * n), 1, 1);
+  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, p);
 }
 
 }  // namespace
@@ -635,38 +709,39 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
     return cudaErrorInvalidValue;
   if (R == 0) return cudaSuccess;
   CUtensorMap ta, tb0, tb1;
-  if (!make_map(&ta, a_sorted, K, R, 0, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&tb0, w0, K, N, E, gate ? 128 : 256)) return cudaErrorInvalidValue;
-  if (gate) {
-    if (!make_map(&tb1, w1, K, N, E, 128)) return cudaErrorInvalidValue;
-  } else {
-    tb1 = tb0;
-  }
-  Params p;
-  p.offsets = offsets;
-  p.sorted_slot = sorted_slot;
-  p.topk_w = topk_w;
-  p.out = out;
-  p.R = R;
-  p.K = K;
-  p.N = N;
-  p.E = E;
-  p.k = k;
-  p.n_tiles_n = (N + tile_n - 1) / tile_n;
-  p.status = status;
-  const int64_t max_tiles = ((R + BM - 1) / BM + E) * static_cast<int64_t>(p.n_tiles_n);
-  const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
-  switch (mode) {
-    case kEpiGateH:
-      return launch_mode<kEpiGateH>(ta, tb0, tb1, p, grid, stream);
-    case kEpiGateSlots:
-      return launch_mode<kEpiGateSlots>(ta, tb0, tb1, p, grid, stream);
-    case kEpiScaleToken:
-      return launch_mode<kEpiScaleToken>(ta, tb0, tb1, p, grid, stream);
-    case kEpiScaleSlots:
-      return launch_mode<kEpiScaleSlots>(ta, tb0, tb1, p, grid, stream);
-    default:
-      return cudaErrorInvalidValue;
+  {
+    if (!make_map(&ta, a_sorted, K, R, 0, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tb0, w0, K, N, E, 128)) return cudaErrorInvalidValue;
+    if (gate) {
+      if (!make_map(&tb1, w1, K, N, E, 128)) return cudaErrorInvalidValue;
+    } else {
+      tb1 = tb0;
+    }
+    Params p{};
+    p.offsets = offsets;
+    p.sorted_slot = sorted_slot;
+    p.topk_w = topk_w;
+    p.out = out;
+    p.R = R;
+    p.K = K;
+    p.N = N;
+    p.E = E;
+    p.k = k;
+    p.n_tiles_n = (N + tile_n - 1) / tile_n;
+    p.status = status;
+    const int64_t max_tiles = ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n);
+    switch (mode) {
+      case kEpiGateH:
+        return launch_pair_mode<kEpiGateH>(ta, tb0, tb1, p, max_tiles, stream);
+      case kEpiGateSlots:
+        return launch_pair_mode<kEpiGateSlots>(ta, tb0, tb1, p, max_tiles, stream);
+      case kEpiScaleToken:
+        return launch_pair_mode<kEpiScaleToken>(ta, tb0, tb1, p, max_tiles, stream);
+      case kEpiScaleSlots:
+        return launch_pair_mode<kEpiScaleSlots>(ta, tb0, tb1, p, max_tiles, stream);
+      default:
+        return cudaErrorInvalidValue;
+    }
   }
 }
 

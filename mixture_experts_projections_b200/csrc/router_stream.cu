@@ -6,13 +6,15 @@
 // time. A producer warp streams the tile's X in 64-feature blocks through a
 // TMA ring (128 x 64 bf16, 128-byte swizzle); the router weight W_r^T stays
 // resident in shared memory as float32 [E][d_model].
-// Eight compute warps: warp w owns tokens 32 (w % 4) .. +31 (one token per
-// lane) and feature half h = w / 4 of every block. A lane reads its token's
-// 32 features of the block from shared memory and the weights as broadcast
-// float4 reads, accumulates a block partial per expert sequentially in
-// float32 FMA and adds it to its running sum. The h = 1 warp hands its sums
-// (and |x|^2) to the h = 0 warp of the same tokens, which adds them last.
-// Each logit therefore goes through at most 32 + ceil(d_model / 64) + 2
+// 4 Q compute warps (Q = 4 feature quarters for E <= 8, Q = 2 halves for
+// E = 16, whose larger W_r leaves less shared memory): warp w owns tokens
+// 32 (w % 4) .. +31 (one token per lane) and feature part h = w / 4 (64 / Q
+// features) of every block. A lane reads its token's features of the block
+// from shared memory and the weights as broadcast float4 reads, accumulates
+// a block partial per expert sequentially in float32 FMA and adds it to its
+// running sum. The h > 0 warps hand their sums (and |x|^2) to the h = 0 warp
+// of the same tokens, which adds them in order h = 1 .. Q-1. Each logit
+// therefore goes through at most 64 / Q + ceil(d_model / 64) + (Q - 1) + 1
 // roundings in a fixed order; with |x| and |w_e| this bounds its error by
 // gamma_n |x| |w_e| (Cauchy-Schwarz). A token whose deciding gaps are not
 // larger than the bounds is re-decided on float64 logits (warp-cooperative,
@@ -35,11 +37,16 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB per stage
-constexpr int kCompute = 8;
-constexpr int kThreads = 32 * (1 + kCompute);
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 8;
 
-template <int EB>
+template <int Q>
+struct Geo {
+  static constexpr int kCompute = 4 * Q;               // compute warps
+  static constexpr int kThreads = 32 * (1 + kCompute);  // + the producer warp
+  static constexpr int kFeat = BK / Q;                  // features per warp per block
+};
+
+template <int EB, int Q>
 struct SCtl {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
@@ -50,7 +57,7 @@ struct SCtl {
   int done[2];
   int hist[2][EB];
   float wnorm[EB];
-  float part[2][BM][EB + 1];  // h = 1 sums (+ |x|^2 in the last column)
+  float part[2][Q - 1][BM][EB + 1];  // h > 0 sums (+ |x|^2 in the last column)
   double l64[4][EB];
 };
 
@@ -59,8 +66,8 @@ __device__ __forceinline__ uint32_t sw128_off(int n, int k) {
   return o ^ (((o >> 7) & 7u) << 4);
 }
 
-template <int EB>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int EB, int Q>
+__global__ void __launch_bounds__(Geo<Q>::kThreads, 1)
     router_stream_kernel(const __grid_constant__ CUtensorMap tmX,
                          const __nv_bfloat16* __restrict__ x, int64_t T, int Dm,
                          const float* __restrict__ w_r, const float* __restrict__ bias, int E,
@@ -68,7 +75,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                          float* __restrict__ topk_w, int32_t* __restrict__ counts,
                          int32_t* __restrict__ chunk_hist, int64_t ntiles, int stages,
                          int DW, float gamma, int* status) {
-  using Ctl = SCtl<EB>;
+  using Ctl = SCtl<EB, Q>;
+  constexpr int kThreads = Geo<Q>::kThreads;
+  constexpr int kCompute = Geo<Q>::kCompute;
+  constexpr int FQ = Geo<Q>::kFeat;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
   // the shared array, not an integer round-trip) so accesses stay LDS/STS.
@@ -90,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int g = 0; g < 4; ++g)
       for (int p = 0; p < 2; ++p) {
-        mbar_init(&ctl.part_ready[g][p], 1);
+        mbar_init(&ctl.part_ready[g][p], Q - 1);
         mbar_init(&ctl.part_free[g][p], 1);
       }
     mbar_init(&ctl.wload, 1);
@@ -109,18 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 reinterpret_cast<const uint8_t*>(w_r) + off, n, &ctl.wload);
     }
   }
-  {
-    int never = 0;
-    mbar_wait(&ctl.wload, 0, &never, status);
-  }
-  for (int e = warp; e < EB; e += kThreads / 32) {
-    float q = 0.f;
-    for (int d = lane; d < Dm; d += 32) q = fmaf(sW[d * EB + e], sW[d * EB + e], q);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-    if (lane == 0) ctl.wnorm[e] = sqrtf(q);
-  }
-  __syncthreads();
 
   if (warp == 0) {
     // -------------------------------------------------- TMA producer
@@ -155,9 +153,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------------------------------------------- compute warps
-  const int cw = warp - 1;  // 0..7
+  // (the producer streams X meanwhile)
+  const int cw = warp - 1;  // 0 .. kCompute-1
   const int g = cw & 3, h = cw >> 2;
   const int row = 32 * g + lane;
+  {
+    int never = 0;
+    mbar_wait(&ctl.wload, 0, &never, status);
+  }
+  for (int e = cw; e < EB; e += kCompute) {
+    float q = 0.f;
+    for (int d = lane; d < Dm; d += 32) q = fmaf(sW[d * EB + e], sW[d * EB + e], q);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (lane == 0) ctl.wnorm[e] = sqrtf(q);
+  }
+  // The norms are read by the deciding warps: a barrier over the compute
+  // warps only (every compute warp reaches it; the producer does not take part).
+  named_barrier_sync(1, 32 * kCompute);
   int stage = 0;
   uint32_t phase = 0;
   int tpar = 0;
@@ -174,10 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const uint8_t* sa = smem + stage * A_BYTES;
-      float xs[32];
+      float xs[FQ];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sa + sw128_off(row, 32 * h + 8 * j));
+      for (int j = 0; j < FQ / 8; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sa + sw128_off(row, FQ * h + 8 * j));
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -191,16 +204,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         stage = 0;
         phase ^= 1u;
       }
-      const float* wrow = sW + static_cast<int64_t>(kb * BK + 32 * h) * EB;
+      const float* wrow = sW + static_cast<int64_t>(kb * BK + FQ * h) * EB;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) sq = fmaf(xs[i], xs[i], sq);
-      // block partials, two experts per packed FMA; per expert the 32
+      for (int i = 0; i < FQ; ++i) sq = fmaf(xs[i], xs[i], sq);
+      // block partials, two experts per packed FMA; per expert the FQ
       // features are accumulated in order
       float2 p2[EB / 2];
 #pragma unroll
       for (int e2 = 0; e2 < EB / 2; ++e2) p2[e2] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < FQ; ++i) {
         const float2 xx = make_float2(xs[i], xs[i]);
         const float4* wv = reinterpret_cast<const float4*>(wrow + i * EB);
 #pragma unroll
@@ -218,14 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok) break;
-    if (h == 1) {
-      // hand the half sums to the h = 0 warp of the same tokens
+    if (h > 0) {
+      // hand the part sums to the h = 0 warp of the same tokens
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&ctl.part_free[g][tpar], tphase ^ 1u, abort_flag, status)))
         break;
 #pragma unroll
-      for (int e = 0; e < EB; ++e) ctl.part[tpar][row][e] = acc[e];
-      ctl.part[tpar][row][EB] = sq;
+      for (int e = 0; e < EB; ++e) ctl.part[tpar][h - 1][row][e] = acc[e];
+      ctl.part[tpar][h - 1][row][EB] = sq;
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.part_ready[g][tpar]);
     } else {
@@ -233,8 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                       mbar_wait(&ctl.part_ready[g][tpar], tphase, abort_flag, status)))
         break;
 #pragma unroll
-      for (int e = 0; e < EB; ++e) acc[e] += ctl.part[tpar][row][e];
-      sq += ctl.part[tpar][row][EB];
+      for (int hh = 0; hh < Q - 1; ++hh) {
+#pragma unroll
+        for (int e = 0; e < EB; ++e) acc[e] += ctl.part[tpar][hh][row][e];
+        sq += ctl.part[tpar][hh][row][EB];
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.part_free[g][tpar]);
 
@@ -388,13 +404,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int EB>
+template <int EB, int Q>
 cudaError_t launch_eb(const void* x, int64_t T, int Dm, const float* w_r, const float* bias, int E,
                       int k, int renorm, int32_t* topk_idx, float* topk_w, int32_t* counts,
                       int32_t* chunk_hist, int* status, cudaStream_t stream) {
   const int64_t ntiles = num_chunks(T);
   const int DW = (Dm + BK - 1) / BK * BK;
-  const size_t ctl = (sizeof(SCtl<EB>) + 15) / 16 * 16;
+  const size_t ctl = (sizeof(SCtl<EB, Q>) + 15) / 16 * 16;
   const size_t wbytes = static_cast<size_t>(EB) * DW * sizeof(float);
   const size_t budget = 224 * 1024;
   int stages = kMaxStages;
@@ -412,18 +428,20 @@ cudaError_t launch_eb(const void* x, int64_t T, int Dm, const float* w_r, const 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // Longest rounding chain of a logit: 32 block FMAs, one add per block,
-  // the two halves, the bias (+1 spare); 1 % slack covers the norms.
-  const double n = 32.0 + static_cast<double>((Dm + BK - 1) / BK) + 3.0;
+  // Longest rounding chain of a logit: 64 / Q block FMAs, one add per
+  // block, Q - 1 adds of the parts, the bias (+1 spare); 1 % slack covers
+  // the norms.
+  const double n = static_cast<double>(Geo<Q>::kFeat) +
+                   static_cast<double>((Dm + BK - 1) / BK) + static_cast<double>(Q - 1) + 2.0;
   const double u = 1.0 / 16777216.0;
   const float gamma = static_cast<float>(1.01 * n * u / (1.0 - n * u));
   const size_t smem = stages * A_BYTES + ctl + wbytes + 1024;
-  auto kern = router_stream_kernel<EB>;
+  auto kern = router_stream_kernel<EB, Q>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int grid = static_cast<int>(std::min<int64_t>(ntiles, device_sm_count()));
-  kern<<<grid, kThreads, smem, stream>>>(tm, static_cast<const __nv_bfloat16*>(x), T, Dm, w_r,
+  kern<<<grid, Geo<Q>::kThreads, smem, stream>>>(tm, static_cast<const __nv_bfloat16*>(x), T, Dm, w_r,
                                          bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                                          ntiles, stages, DW, gamma, status);
   return cudaGetLastError();
@@ -438,13 +456,13 @@ cudaError_t launch_router_stream(const void* x, int64_t T, int Dm, const float* 
   // W_r is staged as stored ([d_model][E], 16-byte rows): E in {4, 8, 16}.
   if (reinterpret_cast<uintptr_t>(w_r) & 15u) return cudaErrorNotSupported;
   if (E == 4)
-    return launch_eb<4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
+    return launch_eb<4, 4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                         status, stream);
   if (E == 8)
-    return launch_eb<8>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
+    return launch_eb<8, 4>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                         status, stream);
   if (E == 16)
-    return launch_eb<16>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
+    return launch_eb<16, 2>(x, T, Dm, w_r, bias, E, k, renorm, topk_idx, topk_w, counts, chunk_hist,
                          status, stream);
   return cudaErrorNotSupported;  // other expert counts use the register-tiled kernel
 }
