@@ -305,27 +305,44 @@ __global__ void __launch_bounds__(Geo<Q>::kThreads, 1)
         const int src = __ffs(todo) - 1;
         todo &= todo - 1;
         const int64_t tr = __shfl_sync(0xffffffffu, tok, src);
-        const __nv_bfloat16* xr = x + tr * Dm;
-        for (int e0 = 0; e0 < EB; e0 += 16) {
-          double a[16];
+        // float64 logits of token tr: lane i takes the 16-byte pieces
+        // i, i + 32, ... of the row (8 features each), four loads in flight.
+        const uint4* xr = reinterpret_cast<const uint4*>(x + tr * Dm);
+        const int npc = Dm / 8;
+        double a[EB];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) a[q] = 0.0;
-          for (int d = lane; d < Dm; d += 32) {
-            const double xv = static_cast<double>(__bfloat162float(xr[d]));
+        for (int e = 0; e < EB; ++e) a[e] = 0.0;
+        for (int pc0 = lane; pc0 < npc; pc0 += 4 * 32) {
+          uint4 v[4];
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-              if (e0 + q < E) a[q] = fma(xv, static_cast<double>(sW[d * EB + e0 + q]), a[q]);
+          for (int u = 0; u < 4; ++u) {
+            const int pc = pc0 + 32 * u;
+            v[u] = (pc < npc) ? __ldg(xr + pc) : make_uint4(0u, 0u, 0u, 0u);
           }
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int u = 0; u < 4; ++u) {
+            const int pc = pc0 + 32 * u;
+            if (pc >= npc) break;
+            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a[q] += __shfl_xor_sync(0xffffffffu, a[q], o);
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t bits = (j & 1) ? (w4[j >> 1] & 0xFFFF0000u) : (w4[j >> 1] << 16);
+              const double xv = static_cast<double>(__uint_as_float(bits));
+              const float* wr = sW + static_cast<int64_t>(pc * 8 + j) * EB;
+#pragma unroll
+              for (int e = 0; e < EB; ++e) a[e] = fma(xv, static_cast<double>(wr[e]), a[e]);
+            }
           }
-          if (lane == src)
-#pragma unroll
-            for (int q = 0; q < 16; ++q)
-              if (e0 + q < E) ctl.l64[g][e0 + q] = a[q] + (bias ? static_cast<double>(bias[e0 + q]) : 0.0);
         }
+#pragma unroll
+        for (int e = 0; e < EB; ++e) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a[e] += __shfl_xor_sync(0xffffffffu, a[e], o);
+        }
+        if (lane == src)
+#pragma unroll
+          for (int e = 0; e < EB; ++e)
+            if (e < E) ctl.l64[g][e] = a[e] + (bias ? static_cast<double>(bias[e]) : 0.0);
         __syncwarp();
         if (lane == src) {
           uint64_t u2 = 0;
