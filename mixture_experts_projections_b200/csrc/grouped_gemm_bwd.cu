@@ -1,8 +1,10 @@
 // Backward grouped GEMMs of the RoM block on the tcgen05 tensor cores
 // ("Routing Mamba ..." chapterpal summary page, Knowl 1, differentiated with
 // the selection S_t held fixed). Three modes share one persistent,
-// warp-specialised kernel (TMA producer, single-thread MMA issuer, 4 epilogue
-// warps, 128 x 256 fp32 accumulators double-buffered in TMEM):
+// warp-specialised kernel run by pairs of CTAs on two SMs (2-CTA clusters,
+// tcgen05.mma.cta_group::2, 256 x 256 pair tiles; per CTA a TMA producer,
+// 4 epilogue warps and, in CTA 0, the single-thread MMA issuer; each CTA's
+// 128 x 256 fp32 accumulators double-buffered in its own TMEM):
 //
 //  kBwdDgradOut  g'_s = (r dO)_s W_out,e^T for the rows s of expert e
 //                (rows in expert-sorted order; A = r-scaled dO rows, K-major;
@@ -31,7 +33,6 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <cstdlib>
 #include <mutex>
 
 #include "rom_internal.cuh"
@@ -43,10 +44,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int CHUNK_BYTES = 64 * BK * 2;  // one 64 x 64 MN-major box, 8 KB
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
@@ -70,22 +67,6 @@ struct BwdParams {
   int* status;
 };
 
-struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t ready[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort;
-  int tile_start[kMaxExperts + 1];
-  int off[kMaxExperts + 1];
-  int mt[kMaxExperts];
-};
-
-constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(SmemCtl) + 1024;
-
 __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t smem_addr, uint32_t lbo_bytes) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
@@ -105,25 +86,6 @@ struct Mode {
   static constexpr bool kWgrad = MODE == kBwdWgrad;
   static constexpr int kThreads = kWgrad ? 224 : 192;  // + the fix-up warp
 };
-
-// Tile -> (expert, m block, n block).
-template <int MODE>
-__device__ __forceinline__ void bwd_tile(const SmemCtl& c, const BwdParams& p, int tile, int& e,
-                                         int& m_blk, int& n_blk) {
-  if (MODE == kBwdWgrad) {
-    const int per_e = p.m_tiles * p.n_tiles_n;
-    e = tile / per_e;
-    const int rem = tile - e * per_e;
-    n_blk = rem / p.m_tiles;
-    m_blk = rem - n_blk * p.m_tiles;
-  } else {
-    e = 0;
-    while (tile >= c.tile_start[e + 1]) ++e;
-    const int local = tile - c.tile_start[e];
-    n_blk = local / c.mt[e];
-    m_blk = local - n_blk * c.mt[e];
-  }
-}
 
 // Epilogue of one accumulator tile for one warp: thread i reads TMEM lane
 // t_row.lane + i, which holds output row `row` (wgrad: row m of dW_e; dgrad:
@@ -189,227 +151,6 @@ __device__ __forceinline__ void bwd_epilogue_rows(const BwdParams& p, uint32_t t
       }
     }
     if (MODE == kBwdDgradOut && valid) p.dr_part[slot * p.n_tiles_n + n_blk] = dot;
-  }
-}
-
-template <int MODE>
-__global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
-    tc_bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                  const __grid_constant__ CUtensorMap tmB1, const BwdParams p) {
-  constexpr bool kW = Mode<MODE>::kWgrad;
-  extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base, kept as a shared-memory pointer (an offset into
-  // the shared array, not an integer round-trip) so accesses stay LDS/STS.
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  SmemCtl& ctl = *reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int E = p.E;
-
-  for (int i = threadIdx.x; i <= E; i += Mode<MODE>::kThreads) ctl.off[i] = p.offsets[i];
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) {
-      const int mt = (ctl.off[e + 1] - ctl.off[e] + BM - 1) / BM;
-      ctl.mt[e] = mt;
-      ctl.tile_start[e] = run;
-      run += kW ? p.m_tiles * p.n_tiles_n : mt * p.n_tiles_n;
-    }
-    ctl.tile_start[E] = run;
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ctl.full[s], 1);
-      mbar_init(&ctl.ready[s], 1);
-      mbar_init(&ctl.empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&ctl.tfull[a], 1);
-      mbar_init(&ctl.tempty[a], 4);
-    }
-    mbar_init(&ctl.drain, 1);
-    ctl.abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB0);
-    tma_prefetch_desc(&tmB1);
-  }
-  if (warp == 1) {
-    tmem_alloc(&ctl.tmem_base, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = ctl.tmem_base;
-  const int total = ctl.tile_start[E];
-  volatile int* abort_flag = &ctl.abort;
-
-  // K blocks of a tile.
-  auto tile_kb = [&](int e) -> int {
-    if (kW) return (ctl.off[e + 1] - ctl.off[e] + BK - 1) / BK;
-    return (p.K + BK - 1) / BK;
-  };
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------ TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0, last_par = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int e, m_blk, n_blk;
-        bwd_tile<MODE>(ctl, p, tile, e, m_blk, n_blk);
-        const int KB = tile_kb(e);
-        const int n0 = n_blk * BN;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          uint64_t* bar = &ctl.full[stage];
-          mbar_arrive_expect_tx(bar, STAGE_BYTES);
-          if (kW) {
-            const int r0 = ctl.off[e] + kb * BK;
-            const int m0 = m_blk * BM;
-            tma_load_2d(sa, &tmA, bar, m0, r0);
-            tma_load_2d(sa + CHUNK_BYTES, &tmA, bar, m0 + 64, r0);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d(sb + j * CHUNK_BYTES, &tmB0, bar, n0 + 64 * j, r0);
-          } else {
-            const int row0 = ctl.off[e] + m_blk * BM;
-            tma_load_2d(sa, &tmA, bar, kb * BK, row0);
-            const bool second = (MODE == kBwdDgradIn) && kb >= p.kb_split;
-            const CUtensorMap* mb = second ? &tmB1 : &tmB0;
-            const int kk = second ? kb - p.kb_split : kb;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_3d(sb + j * CHUNK_BYTES, mb, bar, n0 + 64 * j, kk * BK, e);
-          }
-          issued |= 1u << stage;
-          last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      int never = 0;
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u) mbar_wait(&ctl.full[s], (last_par >> s) & 1u, &never, p.status);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16(BM, BN, kW, true);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int e, m_blk, n_blk;
-        bwd_tile<MODE>(ctl, p, tile, e, m_blk, n_blk);
-        const int KB = tile_kb(e);
-        if (!mbar_wait(&ctl.tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < KB; ++kb) {
-          uint64_t* rb = kW ? &ctl.ready[stage] : &ctl.full[stage];
-          if (!mbar_wait(rb, phase, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = kW ? sw128_mn_desc(a_addr + kk * 2048, CHUNK_BYTES)
-                                   : sw128_kmajor_desc(a_addr + kk * 32);
-            const uint64_t bd = sw128_mn_desc(b_addr + kk * 2048, CHUNK_BYTES);
-            mma_bf16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0);
-          }
-          mma_commit(&ctl.empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        mma_commit(&ctl.tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      }
-      mma_commit(&ctl.drain);
-      int never = 0;
-      mbar_wait(&ctl.drain, 0, &never, p.status);
-    }
-  } else if (warp == 6) {
-    // -------------------------------------------------- fix-up warp (wgrad)
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      int e, m_blk, n_blk;
-      bwd_tile<MODE>(ctl, p, tile, e, m_blk, n_blk);
-      const int n_e = ctl.off[e + 1] - ctl.off[e];
-      const int KB = tile_kb(e);
-      for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(&ctl.full[stage], phase, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        const int valid = n_e - kb * BK;
-        if (valid < BK) {
-          // zero lines valid..63 of the 6 chunks (2 of A, 4 of B)
-          uint8_t* base = smem + stage * STAGE_BYTES;
-          const int lines = BK - valid;
-          const int per_chunk = lines * 8;  // 16-byte pieces
-          for (int i = lane; i < 6 * per_chunk; i += 32) {
-            const int c = i / per_chunk, q = i - c * per_chunk;
-            uint4* dst = reinterpret_cast<uint4*>(base + c * CHUNK_BYTES + valid * 128) + q;
-            *dst = make_uint4(0u, 0u, 0u, 0u);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl.ready[stage]);
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-  } else {
-    // -------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      int e, m_blk, n_blk;
-      bwd_tile<MODE>(ctl, p, tile, e, m_blk, n_blk);
-      if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
-      tc_fence_after();
-      const uint32_t t_row =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const int row = m_blk * BM + q * 32 + lane;  // output row (wgrad) / expert-local row
-      bwd_epilogue_rows<MODE>(p, t_row, e, ctl.off[e], ctl.off[e + 1], row, n_blk);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -798,17 +539,6 @@ bool map_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int
 }
 
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const BwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = tc_bwd_kernel<MODE>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-  if (err != cudaSuccess) return err;
-  kern<<<grid, Mode<MODE>::kThreads, kSmemBytes, stream>>>(a, b0, b1, p);
-  return cudaGetLastError();
-}
-
-template <int MODE>
 cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                              const BwdParams& p, int64_t max_tiles, cudaStream_t stream) {
   auto kern = tc_bwd_pair_kernel<MODE>;
@@ -844,16 +574,6 @@ cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const 
   return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, p);
 }
 
-// The SM-pair kernels serve the backward GEMMs unless ROM_TC_PAIR=0.
-bool use_pair_kernel() {
-  static int v = -1;
-  if (v < 0) {
-    const char* s = getenv("ROM_TC_PAIR");
-    v = (s && s[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
-}
-
 BwdParams base_params(const int32_t* offsets, int64_t R, int E, int k, int* status) {
   BwdParams p{};
   p.offsets = offsets;
@@ -884,12 +604,8 @@ cudaError_t launch_bwd_dgrad_out(const void* rdo_sorted, int64_t R, int Dm, cons
   p.K = Dm;
   p.N = De;
   p.n_tiles_n = De / BN;
-  if (use_pair_kernel())
-    return launch_pair_mode<kBwdDgradOut>(
-        ta, tb, tb, p, ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n), stream);
-  const int64_t max_tiles = ((R + BM - 1) / BM + E) * static_cast<int64_t>(p.n_tiles_n);
-  const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
-  return launch_mode<kBwdDgradOut>(ta, tb, tb, p, grid, stream);
+  return launch_pair_mode<kBwdDgradOut>(
+      ta, tb, tb, p, ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n), stream);
 }
 
 cudaError_t launch_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const void* w_in,
@@ -911,12 +627,8 @@ cudaError_t launch_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const
   p.N = Dm;
   p.kb_split = De / BK;
   p.n_tiles_n = Dm / BN;
-  if (use_pair_kernel())
-    return launch_pair_mode<kBwdDgradIn>(
-        ta, tb0, tb1, p, ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n), stream);
-  const int64_t max_tiles = ((R + BM - 1) / BM + E) * static_cast<int64_t>(p.n_tiles_n);
-  const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
-  return launch_mode<kBwdDgradIn>(ta, tb0, tb1, p, grid, stream);
+  return launch_pair_mode<kBwdDgradIn>(
+      ta, tb0, tb1, p, ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n), stream);
 }
 
 cudaError_t launch_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int64_t R,
@@ -934,15 +646,9 @@ cudaError_t launch_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, 
   p.N = N;
   p.m_split = m_split;
   p.n_tiles_n = N / BN;
-  if (use_pair_kernel()) {
-    p.m_tiles = (M + PM - 1) / PM;
-    return launch_pair_mode<kBwdWgrad>(
-        ta, tb, tb, p, static_cast<int64_t>(E) * p.m_tiles * p.n_tiles_n, stream);
-  }
-  p.m_tiles = M / BM;
-  const int64_t tiles = static_cast<int64_t>(E) * p.m_tiles * p.n_tiles_n;
-  const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), tiles));
-  return launch_mode<kBwdWgrad>(ta, tb, tb, p, grid, stream);
+  p.m_tiles = (M + PM - 1) / PM;
+  return launch_pair_mode<kBwdWgrad>(ta, tb, tb, p,
+                                     static_cast<int64_t>(E) * p.m_tiles * p.n_tiles_n, stream);
 }
 
 }  // namespace rom
