@@ -10,6 +10,10 @@
 // ascending slot order: warps rank 32 consecutive slots with __match_any_sync,
 // and a per-expert prefix over the 32-slot groups orders the groups. The
 // result needs no atomics on the global order and is deterministic.
+//
+// Few chunks (small batches, decode): gridDim.y CTAs share a chunk. Each
+// repeats the (cheap) ranking and copies one slice of the row's 16-byte
+// columns; slice 0 writes the index outputs.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -29,6 +33,7 @@ __global__ void __launch_bounds__(kDispatchThreads)
                     int64_t nchunks, int32_t* __restrict__ offsets,
                     int32_t* __restrict__ sorted_slot, int32_t* __restrict__ slot_pos,
                     uint4* __restrict__ x_sorted) {
+  const int slice = blockIdx.y, nslices = gridDim.y;
   __shared__ int s_tot[kMaxExperts];
   __shared__ int s_base[kMaxExperts];
   __shared__ int s_off[kMaxExperts + 1];
@@ -66,7 +71,7 @@ __global__ void __launch_bounds__(kDispatchThreads)
     s_off[E] = run;
   }
   __syncthreads();
-  if (c == 0)
+  if (c == 0 && slice == 0)
     for (int e = tid; e <= E; e += kDispatchThreads) offsets[e] = s_off[e];
 
   // Per-group, per-expert counts and the rank of each slot inside its group.
@@ -104,19 +109,24 @@ __global__ void __launch_bounds__(kDispatchThreads)
       const int ls = g * 32 + lane;
       const int e = my_e[q];
       const int pos = s_off[e] + s_base[e] + s_gcount[g][e] + my_rank[q];
-      sorted_slot[pos] = static_cast<int32_t>(s0 + ls);
-      slot_pos[s0 + ls] = pos;
+      if (slice == 0) {
+        sorted_slot[pos] = static_cast<int32_t>(s0 + ls);
+        slot_pos[s0 + ls] = pos;
+      }
       s_pos[ls] = pos;
     }
   }
   __syncthreads();
-  // Gather: one warp per slot row, 16-byte vectors, 4 in flight per lane.
+  // Gather this CTA's column slice [v0, v1) of every slot row: one warp per
+  // row, 16-byte vectors, 4 in flight per lane.
+  const int v0 = static_cast<int>(static_cast<int64_t>(row_vec16) * slice / nslices);
+  const int v1 = static_cast<int>(static_cast<int64_t>(row_vec16) * (slice + 1) / nslices);
   for (int ls = warp; ls < ns; ls += kDispatchWarps) {
     const int64_t src = (s0 + ls) / k;
     const uint4* srow = x + src * row_vec16;
     uint4* drow = x_sorted + static_cast<int64_t>(s_pos[ls]) * row_vec16;
-    int i = lane;
-    for (; i + 96 < row_vec16; i += 128) {
+    int i = v0 + lane;
+    for (; i + 96 < v1; i += 128) {
       const uint4 a = __ldg(srow + i), b = __ldg(srow + i + 32), cc = __ldg(srow + i + 64),
                   d = __ldg(srow + i + 96);
       drow[i] = a;
@@ -124,7 +134,7 @@ __global__ void __launch_bounds__(kDispatchThreads)
       drow[i + 64] = cc;
       drow[i + 96] = d;
     }
-    for (; i < row_vec16; i += 32) drow[i] = __ldg(srow + i);
+    for (; i < v1; i += 32) drow[i] = __ldg(srow + i);
   }
 }
 
@@ -140,7 +150,13 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int64_t T, int Dm, int E, 
     return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream);
   }
   const int row_bytes = Dm * (bf16 ? 2 : 4);
-  dispatch_kernel<<<static_cast<unsigned>(nchunks), kDispatchThreads, 0, stream>>>(
+  // Slices per chunk: enough CTAs to cover the SMs twice, at most 16, and
+  // at least 32 vectors (512 bytes) of each row per slice.
+  const int64_t want = (2 * static_cast<int64_t>(device_sm_count())) / nchunks;
+  const int nslices = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>({want, 16, (row_bytes / 16) / 32})));
+  dispatch_kernel<<<dim3(static_cast<unsigned>(nchunks), static_cast<unsigned>(nslices)),
+                    kDispatchThreads, 0, stream>>>(
       static_cast<const uint4*>(x), T, row_bytes / 16, E, k, topk_idx, chunk_hist, nchunks,
       offsets, sorted_slot, slot_pos, static_cast<uint4*>(x_sorted));
   return cudaGetLastError();

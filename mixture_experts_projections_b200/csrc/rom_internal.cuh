@@ -22,6 +22,15 @@ cudaError_t launch_router(const void* x, bool bf16, int64_t T, int Dm, const flo
                           float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                           cudaStream_t stream);
 
+// One CTA per token (small batches); cudaErrorNotSupported when T exceeds
+// kSmallRouterMaxTokens, E is not 4, 8 or 16, or the data is not 16-byte
+// aligned.
+constexpr int64_t kSmallRouterMaxTokens = 1024;
+cudaError_t launch_router_small(const void* x, bool bf16, int64_t T, int Dm, const float* w_r,
+                                const float* bias, int E, int k, int renorm, int32_t* topk_idx,
+                                float* topk_w, int32_t* counts, int32_t* chunk_hist,
+                                cudaStream_t stream);
+
 // Returns cudaErrorNotSupported when W_r does not fit in shared memory.
 cudaError_t launch_router_stream(const void* x, int64_t T, int Dm, const float* w_r,
                                  const float* bias, int E, int k, int renorm, int32_t* topk_idx,

@@ -494,6 +494,12 @@ cudaError_t launch_router(const void* x, bool bf16, int64_t T, int Dm, const flo
                           const float* bias, int E, int k, int renorm, int32_t* topk_idx,
                           float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                           cudaStream_t stream) {
+  // Small batches: one CTA per token (router_small.cu).
+  {
+    const cudaError_t e = launch_router_small(x, bf16, T, Dm, w_r, bias, E, k, renorm, topk_idx,
+                                              topk_w, counts, chunk_hist, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if (bf16) {
     // The streaming router (router_stream.cu) when W_r stays resident in
     // shared memory; the register-tiled kernel below otherwise.

@@ -372,11 +372,19 @@ class HostPipeline:
     device-to-host copy of a third run at the same time. Each token's result
     is the one a single call on the whole batch gives. Device buffers are
     allocated once per stream (torch); the kernels are the library's.
+
+    With ``graph=True`` the second call with the same host buffers, weights
+    and size captures the whole multi-stream sequence (copies and kernels)
+    into a CUDA graph, and later such calls replay it: the host then issues
+    one launch per call instead of some ten per chunk. The first call runs
+    eagerly (it also initialises the library's per-device state).
     """
 
     def __init__(self, T, Dm, N_out, E, k, dtype, device="cuda", chunks=8, nstreams=3,
-                 De=None):
+                 De=None, graph=True):
         self.T, self.Dm, self.E, self.k = T, Dm, E, k
+        self.graph = graph
+        self._graphs, self._seen, self._tail = {}, set(), {}
         per = -(-T // chunks)
         # Chunks of at least 2048 tokens (smaller ones cost more in launches
         # and stream switches than the overlap saves), at most the batch.
@@ -405,49 +413,85 @@ class HostPipeline:
             return
         start = torch.cuda.Event()
         start.record(cur)
+        used = []
         for n, (a, b) in enumerate(chunks):
             j = n % len(self.streams)
             s = self.streams[j]
-            s.wait_event(start)
+            if j not in used:
+                s.wait_event(start)
+                used.append(j)
             with torch.cuda.stream(s):
                 body(j, a, b, s)
-        for s in self.streams:
+        for j in used:
             ev = torch.cuda.Event()
-            ev.record(s)
+            ev.record(self.streams[j])
             cur.wait_event(ev)
+
+    def _launch(self, key, T, body):
+        """Eager on the first call for `key`, captured into a CUDA graph on
+        the second, replayed afterwards."""
+        if not self.graph:
+            self._run(T, body)
+            return
+        g = self._graphs.get(key)
+        if g is None and key in self._seen:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._run(T, body)
+            self._graphs[key] = g
+        if g is None:
+            self._seen.add(key)
+            self._run(T, body)
+        else:
+            g.replay()
+
+    def _tail_bufs(self, n, make):
+        """Buffers of a shorter last chunk, made once per size (outside any capture)."""
+        if n not in self._tail:
+            self._tail[n] = make(n)
+        return self._tail[n]
 
     def block_forward(self, x_host, w_r, bias, w_conv, w_gate, w_out, out_host, renorm=False):
         """x_host [T, Dm] and out_host [T, Dm]: pinned host tensors."""
         T = x_host.shape[0]
+        De = w_conv.shape[1]
+        for a, b in self._chunks(T):
+            if b - a != self.chunk:
+                self._tail_bufs(b - a, lambda n: BlockBuffers(n, self.Dm, De, self.E, self.k,
+                                                              self.x[0].dtype, self.x[0].device))
 
         def body(j, a, b, s):
             xd = self.x[j][: b - a]
             xd.copy_(x_host[a:b], non_blocking=True)
-            bufs = self.bufs[j]
-            if b - a != self.chunk:
-                bufs = BlockBuffers(b - a, self.Dm, w_conv.shape[1], self.E, self.k, xd.dtype,
-                                    xd.device)
+            bufs = self.bufs[j] if b - a == self.chunk else self._tail[b - a]
             blk = block_forward(xd, w_r, bias, w_conv, w_gate, w_out, self.k, renorm, bufs,
                                 stream=s)
             out_host[a:b].copy_(blk.out, non_blocking=True)
 
-        self._run(T, body)
+        key = ("block", T, x_host.data_ptr(), out_host.data_ptr(), w_r.data_ptr(),
+               0 if bias is None else bias.data_ptr(), w_conv.data_ptr(), w_gate.data_ptr(),
+               w_out.data_ptr(), bool(renorm))
+        self._launch(key, T, body)
         return out_host
 
     def inproj_forward(self, x_host, w_r, w, out_host, renorm=False, bias=None):
         """x_host [T, Dm], out_host [T, N_out]: pinned host tensors."""
         T = x_host.shape[0]
+        for a, b in self._chunks(T):
+            if b - a != self.chunk:
+                self._tail_bufs(b - a, lambda n: RoutingBuffers(n, self.Dm, self.E, self.k,
+                                                                self.x[0].dtype, self.x[0].device))
 
         def body(j, a, b, s):
             xd = self.x[j][: b - a]
             xd.copy_(x_host[a:b], non_blocking=True)
-            bufs = self.bufs[j]
-            if b - a != self.chunk:
-                bufs = RoutingBuffers(b - a, self.Dm, self.E, self.k, xd.dtype, xd.device)
+            bufs = self.bufs[j] if b - a == self.chunk else self._tail[b - a]
             od = self.out[j][: b - a]
             sl = None if self.slots[j] is None else self.slots[j][: (b - a) * self.k]
             inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s)
             out_host[a:b].copy_(od, non_blocking=True)
 
-        self._run(T, body)
+        key = ("inproj", T, x_host.data_ptr(), out_host.data_ptr(), w_r.data_ptr(), w.data_ptr(),
+               0 if bias is None else bias.data_ptr(), bool(renorm))
+        self._launch(key, T, body)
         return out_host

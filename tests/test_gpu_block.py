@@ -114,11 +114,14 @@ def test_host_pipeline_matches_single_call(T, Dm, De, E, k, renorm):
     x_h = d["x"].cpu().pin_memory()
     out_h = torch.empty((T, Dm), dtype=torch.bfloat16, pin_memory=True)
     pipe = rom.HostPipeline(T, Dm, None, E, k, torch.bfloat16, "cuda", chunks=5, De=De)
-    pipe.block_forward(x_h, d["w_r"], None, d["w_conv"], d["w_gate"], d["w_out"], out_h,
-                       renorm=renorm)
-    torch.cuda.synchronize()
-    assert_close(out_h.float().numpy(), to_np(ref), "bf16", "O (pipelined vs single call)",
-                 magnitude_scaled_abs=True)
+    # first call eager, second captured into a CUDA graph, third replayed
+    for call in range(3):
+        out_h.zero_()
+        pipe.block_forward(x_h, d["w_r"], None, d["w_conv"], d["w_gate"], d["w_out"], out_h,
+                           renorm=renorm)
+        torch.cuda.synchronize()
+        assert_close(out_h.float().numpy(), to_np(ref), "bf16",
+                     f"O (pipelined vs single call, call {call})", magnitude_scaled_abs=True)
     orc_ref = oracle_block(inp, k, renorm)
     assert_close(out_h.float().numpy().astype(np.float64), orc_ref["O"], "bf16", "O (pipelined)",
                  magnitude_scaled_abs=True)

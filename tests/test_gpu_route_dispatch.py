@@ -23,6 +23,14 @@ ROUTE_CASES = [
     (513, 128, 33, 3, True, "f32", 0.2),
     (200, 256, 1, 1, False, "bf16", 0.02),
     (1, 64, 5, 2, False, "f32", 0.3),
+    # above the small-batch limit (1024 tokens): the chunk-per-CTA routers
+    (2100, 512, 8, 1, False, "bf16", 0.02),
+    (1500, 512, 16, 2, True, "bf16", 0.02),
+    (1300, 256, 4, 1, False, "bf16", 0.1),
+    (1200, 256, 8, 2, False, "f32", 0.05),
+    # small batches with 16 experts, float32 data, a 64-token decode shape
+    (64, 4096, 4, 1, False, "bf16", 0.02),
+    (333, 512, 16, 2, True, "f32", 0.05),
 ]
 
 
@@ -69,11 +77,13 @@ def test_route_zero_router_tie_rule(k, renorm):
                                rtol=1e-6)
 
 
-def test_route_near_ties_are_decided_exactly():
+@pytest.mark.parametrize("T", [512, 2048])
+def test_route_near_ties_are_decided_exactly(T):
     """Two router columns that differ by a tiny perturbation give float32
     logit gaps below the float32 rounding bound; the kernel must fall back to
-    float64 and agree with the oracle on every token."""
-    T, Dm, E = 512, 1024, 4
+    float64 and agree with the oracle on every token (T = 512: the per-token
+    router; T = 2048: the streaming router)."""
+    Dm, E = 1024, 4
     inp = make_block_inputs(T, Dm, 1, E, seed=17)
     w = inp["w_r"].copy()
     rng = np.random.default_rng(5)
@@ -81,7 +91,7 @@ def test_route_near_ties_are_decided_exactly():
     w[:, 2] = w[:, 0] * np.float32(0.5)
     w[:, 3] = -w[:, 0]
     rt = orc.route(inp["x"], w, 1)
-    assert np.mean(rt["margin"] < 1e-4) > 0.5  # most tokens are near-ties in float32 terms
+    assert np.mean(rt["margin"] < 1e-4) > 0.3  # many tokens are near-ties in float32 terms
     b = run_route(to_dev(inp["x"], "bf16"), to_dev(w, "f32"), None, E, 1, False)
     amb = assert_routing_matches(b.topk_idx.cpu().numpy(),
                                  b.topk_w.cpu().numpy().astype(np.float64), rt)
