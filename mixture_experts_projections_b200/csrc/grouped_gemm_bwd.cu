@@ -90,10 +90,12 @@ struct Mode {
 // Epilogue of one accumulator tile for one warp: thread i reads TMEM lane
 // t_row.lane + i, which holds output row `row` (wgrad: row m of dW_e; dgrad:
 // row `row` of expert e's rows e_begin .. e_end - 1), columns
-// n_blk * 256 .. + 255.
+// n_blk * 256 .. + 255. Each 32-column chunk is stored row by row through the
+// warp's staging tile `stg` (row-coalesced stores).
 template <int MODE>
 __device__ __forceinline__ void bwd_epilogue_rows(const BwdParams& p, uint32_t t_row, int e,
-                                                  int e_begin, int e_end, int row, int n_blk) {
+                                                  int e_begin, int e_end, int row, int n_blk,
+                                                  float* stg) {
   const int n0 = n_blk * BN;
   if (MODE == kBwdWgrad) {
     const bool has_k = e_end > e_begin;
@@ -108,14 +110,10 @@ __device__ __forceinline__ void bwd_epilogue_rows(const BwdParams& p, uint32_t t
       uint32_t a[32];
       tmem_ld32(t_row + c * 32, a);
       tmem_ld_wait();
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(dst_row + n0 + c * 32);
+      float f[32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = has_k ? make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                       __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int j = 0; j < 32; ++j) f[j] = has_k ? __uint_as_float(a[j]) : 0.f;
+      store_rows_f32(stg, f, valid ? dst_row + n0 + c * 32 : nullptr);
     }
   } else {
     const int row_local = row;
@@ -129,26 +127,23 @@ __device__ __forceinline__ void bwd_epilogue_rows(const BwdParams& p, uint32_t t
       uint32_t a[32];
       tmem_ld32(t_row + c * 32, a);
       tmem_ld_wait();
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(p.out0 + slot * p.N + n0 + c * 32);
+      if (MODE == kBwdDgradOut && valid) {
+        const uint4* hp = reinterpret_cast<const uint4*>(p.h_sorted + prow * p.N + n0 + c * 32);
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                               __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
-        if (MODE == kBwdDgradOut) {
-          const uint4* hp = reinterpret_cast<const uint4*>(p.h_sorted + prow * p.N + n0 + c * 32);
+        for (int v = 0; v < 4; ++v) {
+          const uint4 hv = __ldg(hp + v);
+          const uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 hv = __ldg(hp + v);
-            const uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dot = fmaf(__uint_as_float(w[i] << 16), __uint_as_float(a[8 * v + 2 * i]), dot);
-              dot = fmaf(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(a[8 * v + 2 * i + 1]), dot);
-            }
+          for (int i = 0; i < 4; ++i) {
+            dot = fmaf(__uint_as_float(w[i] << 16), __uint_as_float(a[8 * v + 2 * i]), dot);
+            dot = fmaf(__uint_as_float(w[i] & 0xFFFF0000u), __uint_as_float(a[8 * v + 2 * i + 1]), dot);
           }
         }
       }
+      float f[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(a[j]);
+      store_rows_f32(stg, f, valid ? p.out0 + slot * p.N + n0 + c * 32 : nullptr);
     }
     if (MODE == kBwdDgradOut && valid) p.dr_part[slot * p.n_tiles_n + n_blk] = dot;
   }
@@ -196,7 +191,10 @@ struct PairCtl {
   int mt[kMaxExperts];
 };
 
-constexpr size_t kPairSmemBytes = P_STAGES * P_STAGE_BYTES + sizeof(PairCtl) + 1024;
+constexpr size_t kPairCtlBytes = (sizeof(PairCtl) + 15) / 16 * 16;
+// ring, control block, the 4 epilogue warps' staging tiles, alignment slack
+constexpr size_t kPairSmemBytes =
+    P_STAGES * P_STAGE_BYTES + kPairCtlBytes + 4 * kStageFloats * sizeof(float) + 1024;
 
 template <int MODE>
 __global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
@@ -472,6 +470,8 @@ __global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
     // -------------------------------------------------- epilogue (warps 2..5, both CTAs)
     const int q = warp & 3;
     const uint32_t tempty0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
+    float* stg = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES + kPairCtlBytes) +
+                 (warp - 2) * kStageFloats;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < total; tile += npairs) {
@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(Mode<MODE>::kThreads, 1)
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const int row = m_blk * PM + half + q * 32 + lane;
-      bwd_epilogue_rows<MODE>(p, t_row, e, ctl.off[e], ctl.off[e + 1], row, n_blk);
+      bwd_epilogue_rows<MODE>(p, t_row, e, ctl.off[e], ctl.off[e + 1], row, n_blk, stg);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

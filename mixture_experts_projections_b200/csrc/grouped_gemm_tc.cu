@@ -78,10 +78,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 // Epilogue of one accumulator tile for one warp: thread i reads TMEM lane
 // t_row.lane + i, i.e. sorted row `prow` (stored only when `valid`), output
-// columns n0 .. n0 + (128 for the gate modes, 256 otherwise) - 1.
+// columns n0 .. n0 + (128 for the gate modes, 256 otherwise) - 1. The
+// float32 outputs (per-slot partials) go row by row through the warp's
+// staging tile `stg` (row-coalesced stores); the bf16 rows, half as wide,
+// are stored directly in 16-byte pieces, which measured faster for them.
 template <int MODE>
 __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, bool valid,
-                                              int64_t prow, int n0) {
+                                              int64_t prow, int n0, float* stg) {
   if (MODE == kEpiGateH) {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
@@ -116,15 +119,13 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
       tmem_ld32(t_row + c * 32, u);
       tmem_ld32(t_row + 128 + c * 32, z);
       tmem_ld_wait();
-      if (valid) {
-        uint4* du = reinterpret_cast<uint4*>(out + slot * p.N + n0 + c * 32);
-        uint4* dz = reinterpret_cast<uint4*>(out + (p.R + slot) * p.N + n0 + c * 32);
+      float f[32];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          du[v] = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
-          dz[v] = make_uint4(z[4 * v], z[4 * v + 1], z[4 * v + 2], z[4 * v + 3]);
-        }
-      }
+      for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(u[j]);
+      store_rows_f32(stg, f, valid ? out + slot * p.N + n0 + c * 32 : nullptr);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(z[j]);
+      store_rows_f32(stg, f, valid ? out + (p.R + slot) * p.N + n0 + c * 32 : nullptr);
     }
   } else {
     const int64_t slot = valid ? p.sorted_slot[prow] : 0;
@@ -135,8 +136,8 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
       uint32_t a[32];
       tmem_ld32(t_row + c * 32, a);
       tmem_ld_wait();
-      if (valid) {
-        if (MODE == kEpiScaleToken) {
+      if (MODE == kEpiScaleToken) {
+        if (valid) {
           __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
           uint4* dst = reinterpret_cast<uint4*>(out + (slot / p.k) * p.N + n0 + c * 32);
 #pragma unroll
@@ -148,14 +149,13 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
             w.w = pack_bf16(r * __uint_as_float(a[8 * v + 6]), r * __uint_as_float(a[8 * v + 7]));
             dst[v] = w;
           }
-        } else {
-          float* out = static_cast<float*>(p.out);
-          float4* dst = reinterpret_cast<float4*>(out + slot * p.N + n0 + c * 32);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(r * __uint_as_float(a[4 * v]), r * __uint_as_float(a[4 * v + 1]),
-                                 r * __uint_as_float(a[4 * v + 2]), r * __uint_as_float(a[4 * v + 3]));
         }
+      } else {
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = r * __uint_as_float(a[j]);
+        float* out = static_cast<float*>(p.out);
+        store_rows_f32(stg, f, valid ? out + slot * p.N + n0 + c * 32 : nullptr);
       }
     }
   }
@@ -198,7 +198,10 @@ struct PairCtl {
   int mt[kMaxExperts];
 };
 
-constexpr size_t kPairSmemBytes = P_STAGES * P_STAGE_BYTES + sizeof(PairCtl) + 1024;
+constexpr size_t kPairCtlBytes = (sizeof(PairCtl) + 15) / 16 * 16;
+// ring, control block, the 4 epilogue warps' staging tiles, alignment slack
+constexpr size_t kPairSmemBytes =
+    P_STAGES * P_STAGE_BYTES + kPairCtlBytes + 4 * kStageFloats * sizeof(float) + 1024;
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -357,6 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------- epilogue (warps 2..5)
     const int q = warp & 3;
     const uint32_t tempty0 = mapa_shared(smem_u32(&ctl.tempty[0]), 0);
+    float* stg = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE_BYTES + kPairCtlBytes) +
+                 (warp - 2) * kStageFloats;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < total; tile += npairs) {
@@ -369,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t prow = static_cast<int64_t>(ctl.off[e]) + row_local;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * UMMA_N);
-      epilogue_rows<MODE>(p, t_row, valid, prow, n_blk * kTileN);
+      epilogue_rows<MODE>(p, t_row, valid, prow, n_blk * kTileN, stg);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -397,11 +402,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // MMA's M side (128 per tile) and the expert's tokens its N side (64 per
 // tile), so a tile streams 128 x K of weights once and the tile count is
 // E x N/128 x ceil(n_e / 64) -- enough tiles to cover the SMs even when every
-// expert has only a handful of tokens. Same output as the Out / in-projection
+// expert has only a handful of tokens. The kernel is bound by HBM, not by
+// the SM count, so the grid is sized to give every CTA the same number of
+// tiles (320 tiles: 107 CTAs of 3 tiles, not 148 CTAs and a partial wave). Same output as the Out / in-projection
 // epilogue: out[token][n] = r * acc (bf16, k == 1) or per slot in float32.
+constexpr int SW_BM = 128;                     // weight rows per tile (MMA M)
 constexpr int SW_BN = 64;                      // tokens per tile (MMA N)
 constexpr int SW_STAGES = 8;
-constexpr int SW_A_BYTES = BM * BK * 2;        // 16 KB of weights
+constexpr int SW_A_BYTES = SW_BM * BK * 2;     // 16 KB of weights
 constexpr int SW_B_BYTES = SW_BN * BK * 2;     // 8 KB of tokens
 constexpr int SW_STAGE_BYTES = SW_A_BYTES + SW_B_BYTES;
 constexpr uint32_t SW_TMEM_COLS = 2 * SW_BN;
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   SwapCtl& ctl = *reinterpret_cast<SwapCtl*>(smem + SW_STAGES * SW_STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
-  const int n_wt = p.N / BM;  // weight-row tiles per expert
+  const int n_wt = p.N / SW_BM;  // weight-row tiles per expert
 
   for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = p.offsets[i];
   __syncthreads();
@@ -491,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int e, w_blk, t_blk;
         coords(tile, e, w_blk, t_blk);
-        const int n0 = w_blk * BM;
+        const int n0 = w_blk * SW_BM;
         const int r0 = ctl.off[e] + t_blk * SW_BN;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
@@ -516,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, SW_BN);
+      const uint32_t idesc = idesc_bf16_f32(SW_BM, SW_BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -564,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * SW_BN);
-      const int n = w_blk * BM + q * 32 + lane;  // this thread's output column
+      const int n = w_blk * SW_BM + q * 32 + lane;  // this thread's output column
       const int n_e = ctl.off[e + 1] - ctl.off[e];
 #pragma unroll 1
       for (int c = 0; c < SW_BN / 32; ++c) {
@@ -679,10 +687,10 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
   const bool gate = (mode == kEpiGateH || mode == kEpiGateSlots);
   const int tile_n = gate ? 128 : 256;
   // Few tokens (decode): the swap-AB kernel streams every weight tile once.
-  if (!gate && R <= kSwapMaxRows && N % BM == 0 && K % 8 == 0 && E <= kMaxExperts) {
+  if (!gate && R <= kSwapMaxRows && N % SW_BM == 0 && K % 8 == 0 && E <= kMaxExperts) {
     if (R == 0) return cudaSuccess;
     CUtensorMap tw, tx;
-    if (!make_map(&tw, w0, K, N, E, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tw, w0, K, N, E, SW_BM)) return cudaErrorInvalidValue;
     if (!make_map(&tx, a_sorted, K, R, 0, SW_BN)) return cudaErrorInvalidValue;
     Params p{};
     p.offsets = offsets;
@@ -695,8 +703,14 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
     p.E = E;
     p.k = k;
     p.status = status;
-    const int64_t max_tiles = ((R + SW_BN - 1) / SW_BN + E) * static_cast<int64_t>(N / BM);
-    const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), max_tiles));
+    // Upper bound of the tile count (the exact count depends on the routing,
+    // read on the device); every CTA gets ceil(tiles / SMs) tiles.
+    const int64_t max_tiles = ((R + SW_BN - 1) / SW_BN + E) * static_cast<int64_t>(N / SW_BM);
+    const int64_t tiles_ub = std::min<int64_t>(
+        max_tiles, static_cast<int64_t>(E) * (N / SW_BM) * ((R + SW_BN - 1) / SW_BN));
+    const int64_t sms = device_sm_count();
+    const int64_t per_cta = (tiles_ub + sms - 1) / sms;
+    const int grid = static_cast<int>(std::min<int64_t>(sms, (tiles_ub + per_cta - 1) / per_cta));
     auto kern = (mode == kEpiScaleToken) ? tc_swap_gemm_kernel<kEpiScaleToken>
                                          : tc_swap_gemm_kernel<kEpiScaleSlots>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

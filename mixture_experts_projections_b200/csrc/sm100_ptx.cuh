@@ -237,6 +237,39 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 }
 
 
+// ------------------------------------------------------------------ epilogue stores
+// An epilogue warp holds a 32 x 32 block one row per thread (thread i: row i,
+// 32 consecutive columns, as tcgen05.ld 32x32b leaves it). Storing it so
+// directly makes every store instruction touch 32 rows. These helpers stage
+// the block in a padded shared-memory tile (kStagePitch floats per row:
+// 16-byte aligned rows, conflict-free both ways) and store it row by row, so
+// that one instruction writes 128 consecutive bytes of one float32 row.
+// `row` is the calling thread's row address (nullptr: the row is not
+// stored); every lane of the warp calls.
+constexpr int kStagePitch = 36;
+constexpr int kStageFloats = 32 * kStagePitch;  // per warp
+
+__device__ __forceinline__ void stage_block(float* stg, const float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  float4* s4 = reinterpret_cast<float4*>(stg + lane * kStagePitch);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_rows_f32(float* stg, const float (&v)[32], float* row) {
+  const int lane = threadIdx.x & 31;
+  stage_block(stg, v);
+#pragma unroll 8
+  for (int r = 0; r < 32; ++r) {
+    float* dst = reinterpret_cast<float*>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(row), r));
+    const float x = stg[r * kStagePitch + lane];
+    if (dst) dst[lane] = x;
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ SM pairs
 // A cluster of two CTAs on neighbouring SMs runs one tcgen05.mma of
 // M = 256 (cta_group::2): CTA v of the pair holds rows 128v .. 128v+127 of A,
