@@ -101,6 +101,21 @@ def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
     assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
 
 
+def test_inproj_skewed_routing_small_batch():
+    """96 tokens over 4 experts (the swap-AB GEMM path); with this seed one
+    expert receives 36 of them and another 17."""
+    T, Dm, N, E = 96, 256, 512, 4
+    inp = make_inproj_inputs(T, Dm, N, E, seed=615, router_std=0.05)
+    ref = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=1, renorm=False)
+    assert np.bincount(ref["topk_idx"].reshape(-1), minlength=E).max() > 32
+    out, rb = rom.inproj_forward(to_dev(inp["x"], "bf16"), to_dev(inp["w_r"], "f32"),
+                                 weights_to_dev(inp["w"], "bf16"), k=1, renorm=False)
+    torch.cuda.synchronize()
+    assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
+                           ref)
+    assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
+
+
 @pytest.mark.parametrize("T,Dm,De,E,k,renorm", [(5000, 256, 256, 8, 1, False),
                                                 (3000, 256, 384, 8, 2, True),
                                                 (900, 256, 256, 4, 1, False)])
