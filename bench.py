@@ -304,8 +304,12 @@ def run_ours(args, rank, world, local_rank):
     if rom.rom_get_status() != 0:
         raise RuntimeError("device status word reports an error after warm-up")
 
-    # Each phase captured once as a CUDA graph (the launch sequence of the
-    # library is static: its kernels read the expert counts on the device).
+    # The step captured once as one CUDA graph (the launch sequence of the
+    # library is static: its kernels read the expert counts on the device),
+    # and each phase once more on its own for the per-phase breakdown.
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step()
     graphs = []
     for ph in phases:
         g = torch.cuda.CUDAGraph()
@@ -328,21 +332,34 @@ def run_ours(args, rank, world, local_rank):
         return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(phases))]
                          for i in range(n)])
 
+    def timed_steps(n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            torch.cuda._sleep(200_000)  # GPU-side head start so that the host stays ahead
+            evs[i][0].record(stream)
+            g_step.replay()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(n)])
+
     for _ in range(2):  # graph warm-up
         timed_loop(lambda j: graphs[j].replay(), 1)
+        timed_steps(1)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
+    step_ms = timed_steps(args.steps)
     ph_ms = timed_loop(lambda j: graphs[j].replay(), args.steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
     eager_ms = timed_loop(lambda j: phases[j](), args.steps)
-    t_total_ms = float(ph_ms.sum())
+    t_total_ms = float(step_ms.sum())
     part_names = ["route_dispatch", "proj0", "proj1", "backward"][:len(phases)]
     part_ms = {n: float(ph_ms[:, j].mean()) for j, n in enumerate(part_names)}
     # The dominant kernel alone (one eager launch between two events, the
@@ -385,7 +402,7 @@ def run_ours(args, rank, world, local_rank):
         if i >= args.warmup:
             e2e_ms.append(s0.elapsed_time(s1))
     e2e_total = float(np.sum(e2e_ms))
-    del graphs
+    del graphs, g_step
 
     stats = torch.tensor([t_total_ms, e2e_total], dtype=torch.float64, device=x.device)
     if world > 1:
