@@ -25,6 +25,10 @@ BLOCK_CASES = [
     (517, 64, 128, 8, 1, False, "f32", 0.05, None),
     (300, 96, 72, 5, 2, True, "f32", 0.2, None),
     (150, 512, 512, 8, 1, False, "bf16", 0.02, {3: -40.0, 5: -40.0}),  # two empty experts
+    # over 1024 routed rows (the SM-pair Out GEMM) with d_model % 256 == 128:
+    # a last tile of 128 output columns
+    (1300, 384, 256, 8, 1, False, "bf16", 0.02, None),
+    (800, 640, 256, 8, 2, True, "bf16", 0.05, None),
 ]
 
 
