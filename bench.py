@@ -515,8 +515,10 @@ def main():
                 "kernels_ms": res["part_ms"], "kernels_ms_eager": res["part_ms_eager"],
                 "eager_ms_per_step": res["eager_ms"],
                 "step": "forward + backward" if wl.backward else "forward",
-                "timing": "step: each phase replayed as a CUDA graph, CUDA events on the launching "
-                          "stream between phases; roofline kernel: eager launch between two events",
+                "timing": "step: the whole step replayed as one CUDA graph between two CUDA "
+                          "events on the launching stream (max over ranks); kernels_ms: each "
+                          "phase replayed as its own graph; roofline kernel: eager launch "
+                          "between two events",
                 "e2e": {"value": wl.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": res["x_bytes"], "d2h_bytes_per_step": res["out_bytes"]},
                 "gpu_launches": res["launches"], "clocks": res["clocks"],
