@@ -180,14 +180,21 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
 // TMEM: both end at a cluster barrier that every path reaches after bounded
 // waits.
 constexpr int PM = 256;                      // rows per pair tile
-constexpr int P_STAGES = 6;
+// Ring depth: 7 stages for the bf16-output modes, 6 (plus the epilogue
+// warps' staging tiles) for the float32-output modes.
+constexpr int P_MAX_STAGES = 7;
+template <int MODE>
+struct PairGeo {
+  static constexpr bool kStaged = (MODE == kEpiGateSlots || MODE == kEpiScaleSlots);
+  static constexpr int kStages = kStaged ? 6 : 7;
+};
 constexpr int P_A_BYTES = BM * BK * 2;       // 16 KB: this CTA's 128 rows
 constexpr int P_B_BYTES = 128 * BK * 2;      // 16 KB: this CTA's half of B
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 
 struct PairCtl {
-  uint64_t full[P_STAGES];
-  uint64_t empty[P_STAGES];
+  uint64_t full[P_MAX_STAGES];
+  uint64_t empty[P_MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -200,8 +207,11 @@ struct PairCtl {
 
 constexpr size_t kPairCtlBytes = (sizeof(PairCtl) + 15) / 16 * 16;
 // ring, control block, the 4 epilogue warps' staging tiles, alignment slack
-constexpr size_t kPairSmemBytes =
-    P_STAGES * P_STAGE_BYTES + kPairCtlBytes + 4 * kStageFloats * sizeof(float) + 1024;
+template <int MODE>
+constexpr size_t pair_smem_bytes() {
+  return PairGeo<MODE>::kStages * P_STAGE_BYTES + kPairCtlBytes +
+         (PairGeo<MODE>::kStaged ? 4 * kStageFloats * sizeof(float) : 0) + 1024;
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -210,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB1, const Params p) {
   constexpr bool kGate = (MODE == kEpiGateH || MODE == kEpiGateSlots);
   constexpr int kTileN = kGate ? 128 : 256;  // output columns per tile
+  constexpr int P_STAGES = PairGeo<MODE>::kStages;
   extern __shared__ uint8_t smem_raw[];
   // Same 1024-byte aligned offset in both CTAs (same kernel, same static
   // layout), as the pair MMA reads the peer's operands at the leader's offsets.
@@ -645,6 +656,7 @@ template <int MODE>
 cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                              const Params& p, int64_t max_tiles, cudaStream_t stream) {
   auto kern = tc_pair_gemm_kernel<MODE>;
+  constexpr size_t kPairSmemBytes = pair_smem_bytes<MODE>();
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kPairSmemBytes));
   if (err != cudaSuccess) return err;
