@@ -204,6 +204,24 @@ def to_dev(torch, a, bf16):
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
 
 
+def max_over_ranks(values, device, world):
+    """Elementwise maximum of per-rank timings (ms totals) over all ranks of the
+    default process group: a multi-rank step lasts as long as its slowest
+    rank. Every rank calls it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(tokens_per_rank, world, step_ms):
+    """Whole-job throughput of replicas: every rank processes its own batch of
+    `tokens_per_rank` tokens in a step that lasts `step_ms` (max over ranks)."""
+    return tokens_per_rank * world / (step_ms / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -404,10 +422,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_total = float(np.sum(e2e_ms))
     del graphs, g_step
 
-    stats = torch.tensor([t_total_ms, e2e_total], dtype=torch.float64, device=x.device)
-    if world > 1:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    t_total_ms, e2e_total = float(stats[0]), float(stats[1])
+    t_total_ms, e2e_total = max_over_ranks([t_total_ms, e2e_total], x.device, world)
     res = dict(wl=wl, step_ms=t_total_ms / args.steps, part_ms=part_ms,
                part_ms_eager=part_ms_eager,
                eager_ms=float(eager_ms.sum()) / args.steps,
@@ -487,7 +502,7 @@ def main():
     if rank == 0:
         peaks, src = load_peaks()
         step_s = res["step_ms"] / 1e3
-        value = wl.T * world / step_s
+        value = job_tokens_per_s(wl.T, world, res["step_ms"])
         tot_flops = sum(flops.values())
         if wl.kind == "inproj":
             n_hit = int(np.count_nonzero(res["counts"]))
@@ -519,7 +534,7 @@ def main():
                           "events on the launching stream (max over ranks); kernels_ms: each "
                           "phase replayed as its own graph; roofline kernel: eager launch "
                           "between two events",
-                "e2e": {"value": wl.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
+                "e2e": {"value": job_tokens_per_s(wl.T, world, res["e2e_ms"]), "unit": "tokens/s",
                         "h2d_bytes_per_step": res["x_bytes"], "d2h_bytes_per_step": res["out_bytes"]},
                 "gpu_launches": res["launches"], "clocks": res["clocks"],
                 "expert_load": (res["counts"] / max(1, res["counts"].sum())).round(4).tolist()}

@@ -1,0 +1,83 @@
+"""Host logic of `bench.py --gpus N` (replicas, one process per GPU), run on CPU
+with world_size-2 gloo process groups: the step time is the maximum over the
+ranks, the job throughput counts every rank's tokens, and the reference arm
+runs on rank 0 only. The forward needs no collective on the data path, so
+the timing reduction is the only exchange between ranks."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, per_rank, expect):
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(per_rank[rank], "cpu", world)
+        assert got == expect, (rank, got, expect)
+        # every rank agrees on the job value computed from the reduced time
+        v = bench.job_tokens_per_s(1000, world, got[0])
+        assert abs(v - 1000 * world / (expect[0] / 1e3)) < 1e-6 * v
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_step_time_is_the_maximum_over_two_gloo_ranks():
+    world = 2
+    per_rank = [[10.0, 7.5], [12.5, 3.0]]  # [step ms total, e2e ms total] per rank
+    expect = [12.5, 7.5]
+    mp.start_processes(_rank_main, args=(world, _free_port(), per_rank, expect), nprocs=world,
+                       start_method="spawn", join=True)
+
+
+def test_job_throughput_counts_every_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.job_tokens_per_s(16384, 1, 0.5) == pytest.approx(16384 / 0.5e-3)
+    assert bench.job_tokens_per_s(16384, 8, 0.5) == pytest.approx(8 * 16384 / 0.5e-3)
+
+
+def _run_reference(rank, world):
+    env = dict(os.environ, RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+               MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    return subprocess.run(
+        [sys.executable, "bench.py", "--impl", "reference", "--gpus", str(world), "--steps", "1",
+         "--warmup", "3", "--workload", "tiny_fp32"],
+        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+
+
+def test_reference_arm_on_a_non_zero_rank_exits_quietly():
+    r = _run_reference(1, 2)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
+
+
+def test_reference_arm_on_rank_zero_prints_one_line():
+    r = _run_reference(0, 2)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
