@@ -440,6 +440,21 @@ struct SwapCtl {
 
 constexpr size_t kSwapSmemBytes = SW_STAGES * SW_STAGE_BYTES + sizeof(SwapCtl) + 1024;
 
+// Output row and router weight of one token of the tile, for the lane that
+// holds it (one token per lane, so the slot and weight loads of a chunk of
+// 32 tokens are issued together rather than one dependent pair per store).
+template <int MODE>
+__device__ __forceinline__ void swap_token(const Params& p, int64_t prow, bool valid, int& orow,
+                                           float& r) {
+  orow = 0;
+  r = 0.f;
+  if (valid) {
+    const int slot = p.sorted_slot[prow];
+    r = p.topk_w[slot];
+    orow = MODE == kEpiScaleToken ? slot / p.k : slot;
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_swap_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
@@ -579,29 +594,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       int e, w_blk, t_blk;
       coords(tile, e, w_blk, t_blk);
+      const int n_e = ctl.off[e + 1] - ctl.off[e];
+      const int nv = min(SW_BN, n_e - t_blk * SW_BN);  // valid token columns, >= 1
+      // token info first: its loads overlap the wait for the accumulator
+      const int64_t prow0 = static_cast<int64_t>(ctl.off[e]) + t_blk * SW_BN;
+      int orow[2];
+      float rw[2];
+      swap_token<MODE>(p, prow0 + lane, lane < nv, orow[0], rw[0]);
+      swap_token<MODE>(p, prow0 + 32 + lane, 32 + lane < nv, orow[1], rw[1]);
       if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * SW_BN);
       const int n = w_blk * SW_BM + q * 32 + lane;  // this thread's output column
-      const int n_e = ctl.off[e + 1] - ctl.off[e];
-#pragma unroll 1
-      for (int c = 0; c < SW_BN / 32; ++c) {
-        const int j0 = t_blk * SW_BN + c * 32;  // first token of this column chunk
-        if (j0 >= n_e) break;
-        uint32_t a[32];
-        tmem_ld32(t_row + c * 32, a);
-        tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j0 + j >= n_e) continue;
-          const int64_t prow = ctl.off[e] + j0 + j;
-          const int64_t slot = p.sorted_slot[prow];
-          const float v = p.topk_w[slot] * __uint_as_float(a[j]);
-          if (MODE == kEpiScaleToken)
-            static_cast<__nv_bfloat16*>(p.out)[(slot / p.k) * p.N + n] = __float2bfloat16_rn(v);
-          else
-            static_cast<float*>(p.out)[slot * p.N + n] = v;
+      for (int c = 0; c < SW_BN / 32; ++c) {
+        if (32 * c < nv) {  // warp-uniform
+          uint32_t a[32];
+          tmem_ld32(t_row + c * 32, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (32 * c + j < nv) {  // warp-uniform
+              const int o = __shfl_sync(0xffffffffu, orow[c], j);
+              const float v = __shfl_sync(0xffffffffu, rw[c], j) * __uint_as_float(a[j]);
+              const int64_t i = static_cast<int64_t>(o) * p.N + n;
+              if (MODE == kEpiScaleToken)
+                static_cast<__nv_bfloat16*>(p.out)[i] = __float2bfloat16_rn(v);
+              else
+                static_cast<float*>(p.out)[i] = v;
+            }
+          }
         }
       }
       tc_fence_before();

@@ -29,6 +29,9 @@ BLOCK_CASES = [
     # a last tile of 128 output columns
     (1300, 384, 256, 8, 1, False, "bf16", 0.02, None),
     (800, 640, 256, 8, 2, True, "bf16", 0.05, None),
+    # few routed rows (the swap-AB Out GEMM) over d_inner = 1024 and 1536
+    (500, 512, 1024, 8, 1, False, "bf16", 0.02, None),
+    (400, 256, 1536, 4, 2, True, "bf16", 0.05, None),
 ]
 
 
@@ -90,6 +93,10 @@ INPROJ_CASES = [
     (64, 512, 1280, 4, 1, False),
     (200, 256, 768, 4, 2, True),
     (37, 1024, 512, 8, 1, False),
+    # several 64-token tiles per expert, float32 slots
+    (300, 1024, 768, 4, 2, True),
+    # ragged last K block (K = 1000), partial token tiles of both 32-column halves
+    (700, 1000, 512, 4, 1, False),
 ]
 
 
@@ -103,6 +110,19 @@ def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
                            ref)
     assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
+
+
+def test_inproj_is_deterministic():
+    """The in-projection accumulates in a fixed order and writes every output
+    once: two calls give identical bits."""
+    inp = make_inproj_inputs(64, 4096, 1024, 4, seed=7, router_std=0.05)
+    args = (to_dev(inp["x"], "bf16"), to_dev(inp["w_r"], "f32"), weights_to_dev(inp["w"], "bf16"))
+    a, _ = rom.inproj_forward(*args, k=1, renorm=False)
+    a = a.clone()
+    b, _ = rom.inproj_forward(*args, k=1, renorm=False)
+    torch.cuda.synchronize()
+    assert rom.rom_get_status() == 0
+    assert torch.equal(a, b)
 
 
 def test_inproj_skewed_routing_small_batch():
