@@ -55,17 +55,44 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
-def csrc_digest():
-    """sha256 over the CUDA sources and the C header (identifies the kernels)."""
+def strip_c_comments(src):
+    """C / C++ / CUDA source without its comments, trailing blanks and blank
+    lines; string and character literals are kept as written."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
+def csrc_digest(root=ROOT):
+    """sha256 over the CUDA sources and the C header with their comments
+    removed (identifies the kernels: a comment edit leaves it unchanged)."""
     import glob
     import hashlib
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "mixture_experts_projections_b200", "csrc", "*.cu*")))
-    files.append(os.path.join(ROOT, "include", "rom.h"))
+    files = sorted(glob.glob(os.path.join(root, "mixture_experts_projections_b200", "csrc", "*.cu*")))
+    files.append(os.path.join(root, "include", "rom.h"))
     for f in files:
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(strip_c_comments(fh.read()).encode())
     return h.hexdigest()
 
 

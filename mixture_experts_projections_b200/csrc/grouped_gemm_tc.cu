@@ -22,7 +22,7 @@
 //   last tile of 128 columns when N % 256 == 128: the weight rows past N are
 //   zero-filled by TMA and those columns are not stored).
 // CTA: persistent (one pair of CTAs per pair of SMs), 6 warps:
-//   warp 0  TMA producer (one thread), 6-stage ring (32 KB/stage per CTA)
+//   warp 0  TMA producer (one thread), 6- or 7-stage ring (32 KB/stage/CTA)
 //   warp 1  TMEM allocator; in CTA 0 also the MMA issuer (one thread)
 //   warps 2-5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile run
@@ -168,8 +168,8 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
 // CTA 0 the 128 W_in columns, CTA 1 the same 128 W_g columns; Out: CTA v
 // the output columns 128v .. 128v+127), so each SM streams 32 KB per K step
 // instead of 48 KB, and the 128 x 256 accumulator of its own rows lands in
-// its own TMEM, where its own epilogue warps read it as in the one-CTA
-// kernel. Protocol:
+// its own TMEM, where its own epilogue warps read it, one row per
+// thread. Protocol:
 //   full[s]   lives in CTA 0: CTA 0's producer arms it with both CTAs'
 //             bytes; both producers' TMA loads complete on it.
 //   empty[s]  one per CTA: the MMA commit arrives on both (multicast).
