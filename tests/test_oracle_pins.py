@@ -51,6 +51,23 @@ def test_worked_example_closed_form():
     np.testing.assert_allclose(fw["O"], exp, rtol=1e-14, atol=1e-14)
 
 
+def test_silu_closed_forms_and_extremes():
+    """SiLU(z) = z sigma(z): SiLU(ln 3) = (3/4) ln 3, SiLU(z) - SiLU(-z) = z,
+    SiLU'(0) = 1/2 and SiLU'(z) + SiLU'(-z) = 1; no overflow for |z| ~ 1e3
+    (SiLU -> z above, -> 0 below)."""
+    l3 = math.log(3.0)
+    assert orc.silu(np.array([l3]))[0] == pytest.approx(0.75 * l3, rel=1e-15)
+    z = np.linspace(-40.0, 40.0, 161)
+    np.testing.assert_allclose(orc.silu(z) - orc.silu(-z), z, rtol=1e-14, atol=1e-14)
+    assert orc.silu_grad(np.array([0.0]))[0] == pytest.approx(0.5, rel=1e-15)
+    np.testing.assert_allclose(orc.silu_grad(z) + orc.silu_grad(-z), 1.0, rtol=1e-14)
+    with np.errstate(over="raise", invalid="raise", divide="raise"):
+        big = np.array([-1000.0, -750.0, 750.0, 1000.0])
+        out = orc.silu(big)
+    assert np.all(np.isfinite(out))
+    np.testing.assert_allclose(out, [0.0, 0.0, 750.0, 1000.0], atol=1e-300)
+
+
 def test_softmax_sums_to_one_and_matches_scipy():
     inp = make_block_inputs(64, 32, 16, 8, seed=3)
     rt = orc.route(inp["x"], inp["w_r"], 2)
