@@ -502,8 +502,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = WORKLOADS[args.workload]
     flops = block_flops(wl)
-    metric = ("tokens/s for RoM projection block fwd+bwd" if wl.backward
-              else "tokens/s for RoM projection block fwd")
+    metric = (f"tokens/s and TFLOPS (% bf16 peak) for RoM projection block "
+              f"{'fwd+bwd' if wl.backward else 'fwd'}, {world} B200")
     config = {"workload": wl.name, "tokens": wl.T, "d_model": wl.Dm,
               ("d_out" if wl.kind == "inproj" else "d_inner"): wl.De, "experts": wl.E,
               "top_k": wl.k, "renorm": wl.renorm, "parallelism": f"replicas x{world}",

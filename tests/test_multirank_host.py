@@ -81,3 +81,10 @@ def test_reference_arm_on_rank_zero_prints_one_line():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["unit"] == "tokens/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_metric_names_the_block_and_the_gpu_count():
+    r = _run_reference(0, 1)
+    assert r.returncode == 0, r.stderr
+    line = json.loads([ln for ln in r.stdout.splitlines() if ln.strip()][0])
+    assert line["metric"] == "tokens/s and TFLOPS (% bf16 peak) for RoM projection block fwd, 1 B200"
