@@ -1,0 +1,59 @@
+"""Host arithmetic of bench.py, on CPU: the roofline numerators (algorithmic
+FLOPs and bytes per launch) and the summary of the SM-clock samples that
+decides whether a timed run was throttled (fed with nvidia-smi CSV lines)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from mixture_experts_projections_b200.inputs import WORKLOADS  # noqa: E402
+
+
+def test_block_flops_of_the_workloads():
+    f = bench.block_flops(WORKLOADS["prefill_16k"])
+    assert f["conv_gate"] == pytest.approx(549.76e9, rel=1e-4)  # 4 * 16384 * 2048 * 4096
+    assert f["out"] == pytest.approx(274.88e9, rel=1e-4)
+    assert "backward" not in f
+    t2 = bench.block_flops(WORKLOADS["top2_fwd_bwd"])
+    # R = 65536 routed rows: 5.154 TFLOP forward, twice that backward
+    assert t2["conv_gate"] + t2["out"] == pytest.approx(5.154e12, rel=1e-3)
+    assert t2["backward"] == pytest.approx(2 * 5.154e12, rel=1e-3)
+    assert bench.block_flops(WORKLOADS["decode_swimba_inproj"]) == {
+        "inproj": 2.0 * 64 * 4096 * 10240}
+
+
+def test_inproj_bytes_of_the_decode_workload():
+    wl = WORKLOADS["decode_swimba_inproj"]
+    # 335.5 MB of weights (4 experts hit) + 0.5 MB x + 1.3 MB out
+    assert bench.inproj_bytes(wl, 4) == 4 * 4096 * 10240 * 2 + 64 * 4096 * 2 + 64 * 10240 * 2
+    assert bench.inproj_bytes(wl, 4) == pytest.approx(337.4e6, rel=1e-3)
+    # only the experts that received tokens stream their weights
+    assert bench.inproj_bytes(wl, 3) == bench.inproj_bytes(wl, 4) - 4096 * 10240 * 2
+
+
+def _line(sm, smax, hw="Not Active", hwt="Not Active", swt="Not Active", cap="Not Active"):
+    return f"0, {sm}, {smax}, 812.50, 0x0000000000000000, {hw}, {hwt}, {swt}, {cap}"
+
+
+def test_clock_summary_unthrottled():
+    s = bench.summarize_clocks([_line(1965, 1965), _line(1950, 1965), _line(1965, 1965)])
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3}
+
+
+def test_clock_summary_reports_every_active_reason():
+    s = bench.summarize_clocks([_line(1830, 1965, cap="Active"), _line(1700, 1965, cap="Active"),
+                                _line(1500, 1965, hwt="Active"), _line(1965, 1965)])
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert s["sm_mhz"] == pytest.approx(1765.0)
+    assert s["samples"] == 4
+
+
+def test_clock_summary_skips_lines_that_do_not_parse():
+    s = bench.summarize_clocks(["", "garbage", _line("[N/A]", 1965), _line(1965, 1965),
+                                "0, 1965, 1965"])
+    assert s["samples"] == 1 and s["sm_mhz"] == 1965.0
+    empty = bench.summarize_clocks([])
+    assert empty["sm_mhz"] is None and empty["sm_max_mhz"] is None and empty["samples"] == 0
