@@ -164,3 +164,32 @@ def test_host_pipeline_matches_single_call(T, Dm, De, E, k, renorm):
     orc_ref = oracle_block(inp, k, renorm)
     assert_close(out_h.float().numpy().astype(np.float64), orc_ref["O"], "bf16", "O (pipelined)",
                  magnitude_scaled_abs=True)
+
+
+
+@pytest.mark.parametrize("T,Dm,N,E,k,renorm", [(5000, 256, 512, 4, 1, False),
+                                               (3000, 512, 768, 8, 2, True)])
+def test_host_pipeline_inproj_matches_single_call(T, Dm, N, E, k, renorm):
+    """The in-projection on pinned host buffers (chunks over three streams;
+    eager, captured and replayed calls) matches one call on the whole batch
+    and the oracle within the forward's bar (a short last chunk may take the
+    swap-AB GEMM where the whole batch takes the SM-pair one)."""
+    inp = make_inproj_inputs(T, Dm, N, E, seed=T + 1, router_std=0.05)
+    x = to_dev(inp["x"], "bf16")
+    w_r = to_dev(inp["w_r"], "f32")
+    w = weights_to_dev(inp["w"], "bf16")
+    ref, _ = rom.inproj_forward(x, w_r, w, k=k, renorm=renorm)
+    ref = ref.clone()
+    x_h = x.cpu().pin_memory()
+    out_h = torch.empty((T, N), dtype=torch.bfloat16, pin_memory=True)
+    pipe = rom.HostPipeline(T, Dm, N, E, k, torch.bfloat16, "cuda", chunks=5)
+    for call in range(3):
+        out_h.zero_()
+        pipe.inproj_forward(x_h, w_r, w, out_h, renorm=renorm)
+        torch.cuda.synchronize()
+        assert rom.rom_get_status() == 0
+        assert_close(out_h.float().numpy(), to_np(ref), "bf16",
+                     f"S (pipelined vs single call, call {call})", magnitude_scaled_abs=True)
+    orc_ref = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=k, renorm=renorm)
+    assert_close(out_h.float().numpy().astype(np.float64), orc_ref["S"], "bf16", "S (pipelined)",
+                 magnitude_scaled_abs=True)
