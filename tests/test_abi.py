@@ -118,3 +118,83 @@ def test_binding_fails_loudly_without_library(tmp_path):
             rom.load_library(str(tmp_path / "missing.so"))
         finally:
             rom._lib = old
+
+
+# Every case below fails validation, so nothing reaches the device (the
+# pointers are never dereferenced).
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), 1), (dict(k=9), 1), (dict(N=0), 1), (dict(T=-1), 1), (dict(N=12), 2),
+    (dict(dout=None), 1), (dict(rdo_sorted=ctypes.c_void_p((1 << 20) + 4)), 2),
+])
+def test_bwd_gather_rejects_bad_arguments(lib, kw, code):
+    a = dict(dout=FAKE, T=10, k=2, N=64, sorted_slot=FAKE, topk_w=FAKE, rdo_sorted=FAKE,
+             stream=None)
+    a.update(kw)
+    assert lib.rom_bwd_gather(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(R=255), 1), (dict(E=0), 1), (dict(E=65), 1), (dict(k=9), 1), (dict(Dm=100), 2),
+    (dict(De=128), 2), (dict(offsets=None), 1), (dict(g_slots=ctypes.c_void_p((1 << 20) + 4)), 2),
+])
+def test_bwd_dgrad_out_rejects_bad_arguments(lib, kw, code):
+    a = dict(rdo_sorted=FAKE, R=256, Dm=256, w_out=FAKE, De=256, E=8, k=2, offsets=FAKE,
+             sorted_slot=FAKE, h_sorted=FAKE, g_slots=FAKE, dr_part=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_bwd_dgrad_out(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), 1), (dict(De=0), 1), (dict(De=6), 2), (dict(uz=None), 1),
+    (dict(dhz_sorted=ctypes.c_void_p((1 << 20) + 2)), 2),
+])
+def test_bwd_gate_rejects_bad_arguments(lib, kw, code):
+    a = dict(uz=FAKE, g_slots=FAKE, T=10, k=2, De=64, slot_pos=FAKE, dhz_sorted=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_bwd_gate(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(R=-1), 1), (dict(k=3, E=2), 1), (dict(De=100), 2), (dict(Dm=128), 2),
+    (dict(w_g=None), 1), (dict(dx_slots=ctypes.c_void_p((1 << 20) + 4)), 2),
+])
+def test_bwd_dgrad_in_rejects_bad_arguments(lib, kw, code):
+    a = dict(dhz_sorted=FAKE, R=256, De=256, w_in=FAKE, w_g=FAKE, Dm=256, E=8, k=2,
+             offsets=FAKE, sorted_slot=FAKE, dx_slots=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_bwd_dgrad_in(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_parts=0), 1), (dict(renorm=2), 1), (dict(renorm=0), 2), (dict(Dm=6), 2),
+    (dict(k=9), 1), (dict(w_r=None), 1), (dict(dx=ctypes.c_void_p((1 << 20) + 2)), 2),
+])
+def test_route_bwd_rejects_bad_arguments(lib, kw, code):
+    a = dict(T=10, k=2, E=8, Dm=64, renorm=1, topk_idx=FAKE, topk_w=FAKE, dr_part=FAKE,
+             n_parts=1, dx_slots=FAKE, w_r=FAKE, dlogits=FAKE, dx=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_route_bwd(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=0), 1), (dict(m_split=-1), 1), (dict(m_split=384), 1), (dict(M=200), 2),
+    (dict(N=128), 2), (dict(m_split=64), 2), (dict(out1=None), 1), (dict(out0=None), 1),
+])
+def test_bwd_wgrad_rejects_bad_arguments(lib, kw, code):
+    a = dict(a_sorted=FAKE, M=256, b_sorted=FAKE, N=256, R=512, E=8, offsets=FAKE, m_split=128,
+             out0=FAKE, out1=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_bwd_wgrad(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), 1), (dict(E=0), 1), (dict(k=9), 1), (dict(renorm=2), 1), (dict(Dm=12), 2),
+    (dict(offsets=None), 1), (dict(x_sorted=None), 1), (dict(x=ctypes.c_void_p((1 << 20) + 2)), 2),
+    (dict(T=128 * 65537, E=1), 3),  # more chunk histograms than the fixed scratch holds
+])
+def test_route_dispatch_noalloc_rejects_bad_arguments(lib, kw, code):
+    a = dict(x=FAKE, dtype=1, T=300, Dm=64, w_r=FAKE, bias=None, E=8, k=1, renorm=0,
+             topk_idx=FAKE, topk_w=FAKE, counts=None, offsets=FAKE, sorted_slot=FAKE,
+             slot_pos=FAKE, x_sorted=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_route_dispatch_noalloc(*a.values()) == code
