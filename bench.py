@@ -552,10 +552,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    try:
-        res = run_ours(args, rank, world, local_rank)
-    finally:
-        pass
+    res = run_ours(args, rank, world, local_rank)
     if rank == 0:
         config["l2"] = res["l2"]
         peaks, src = load_peaks()
