@@ -48,7 +48,9 @@ typedef enum {
   ROM_ERR_UNSUPPORTED = 2, /* valid but not implemented (shape or alignment limit) */
   ROM_ERR_WORKSPACE = 3,   /* workspace missing or smaller than rom_workspace_size() */
   ROM_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-  ROM_ERR_TIMEOUT = 5      /* device side: a bounded wait ran out (see rom_get_status) */
+  ROM_ERR_TIMEOUT = 5,     /* device side: a bounded wait ran out (see rom_get_status) */
+  ROM_ERR_ROUTING = 6      /* device side: rom_dispatch found expert indices outside [0, E) or
+                              histograms that do not match them (see rom_get_status) */
 } rom_status;
 
 typedef enum { ROM_F32 = 0, ROM_BF16 = 1 } rom_dtype;
@@ -116,6 +118,14 @@ int rom_route(const void* x, int dtype, int64_t T, int Dm, const float* w_r, con
  *  sorted_slot [T*k]     out, int32: sorted position -> slot
  *  slot_pos    [T*k]     out, int32: slot -> sorted position
  *  x_sorted    [T*k][Dm] out, dtype: x_sorted[p] = x[sorted_slot[p] / k]
+ *
+ * The kernel checks topk_idx and the workspace before using them as indices:
+ * every index must lie in [0, E), and the histograms must be the ones
+ * rom_route() wrote for these indices. If not (for example after the router
+ * gave up on a bounded wait), it records ROM_ERR_ROUTING in the device status
+ * word (rom_get_status) and writes outputs that stay in range for the kernels
+ * that read them (offsets monotone in [0, T*k], sorted_slot and slot_pos in
+ * [0, T*k)); their values then carry no meaning.
  */
 int rom_dispatch(const void* x, int dtype, int64_t T, int Dm, int E, int k,
                  const int32_t* topk_idx, const void* ws, size_t ws_bytes, int32_t* offsets,
@@ -279,7 +289,10 @@ int rom_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int6
  * Sharing: every call on a device uses the same array. Calls that can
  * overlap on the GPU (unordered streams) race on it and must not be issued;
  * calls on one stream are safe. The array keeps the last call's contents,
- * which is harmless: the router rewrites every entry the dispatch reads.
+ * which is harmless: the router rewrites every entry the dispatch reads, and
+ * if the router gives up on a bounded wait the dispatch's own checks catch
+ * stale entries (ROM_ERR_ROUTING). Device-side errors go to the same status
+ * word as for rom_route() and rom_dispatch() (rom_get_status).
  *
  * Set-up: the first call on a device looks up the array's device address
  * (with that device current) and caches it; make that first call before

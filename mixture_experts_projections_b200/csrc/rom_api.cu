@@ -26,19 +26,6 @@ int current_device() {
   return d;
 }
 
-// Device address of this device's status word (nullptr on failure).
-int* status_ptr() {
-  const int d = current_device();
-  if (d < 0) return nullptr;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_status_ptr[d]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    g_status_ptr[d] = static_cast<int*>(p);
-  }
-  return g_status_ptr[d];
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int to_status(cudaError_t e) {
@@ -61,6 +48,18 @@ __global__ void debug_wait_kernel(uint64_t limit_ns, int* status) {
 }
 
 }  // namespace
+
+int* status_ptr() {
+  const int d = current_device();
+  if (d < 0) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status_ptr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[d] = static_cast<int*>(p);
+  }
+  return g_status_ptr[d];
+}
 
 int device_sm_count() {
   const int d = current_device();
@@ -95,6 +94,8 @@ const char* rom_status_string(int status) {
       return "ROM_ERR_CUDA";
     case ROM_ERR_TIMEOUT:
       return "ROM_ERR_TIMEOUT";
+    case ROM_ERR_ROUTING:
+      return "ROM_ERR_ROUTING";
     default:
       return "ROM_ERR_UNKNOWN";
   }
@@ -149,9 +150,11 @@ int rom_dispatch(const void* x, int dtype, int64_t T, int Dm, int E, int k,
     if (!aligned16(x) || !aligned16(x_sorted)) return ROM_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < rom_workspace_size(T, E)) return ROM_ERR_WORKSPACE;
   }
+  int* st = rom::status_ptr();
+  if (!st) return ROM_ERR_CUDA;
   return rom::to_status(rom::launch_dispatch(x, bf16, T, Dm, E, k, topk_idx,
                                              static_cast<const int32_t*>(ws), offsets,
-                                             sorted_slot, slot_pos, x_sorted,
+                                             sorted_slot, slot_pos, x_sorted, st,
                                              static_cast<cudaStream_t>(stream)));
 }
 

@@ -15,7 +15,14 @@ constexpr int kMaxTopK = 8;
 
 inline int64_t num_chunks(int64_t T) { return (T + kChunkTokens - 1) / kChunkTokens; }
 
+// Device status codes written by kernels (the same values as rom_status).
+constexpr int kStatusRouting = 6;  // == ROM_ERR_ROUTING
+
 int device_sm_count();  // cached per device
+
+// Device address of this device's status word (nullptr on failure), looked
+// up once per device with that device current.
+int* status_ptr();
 
 cudaError_t launch_router(const void* x, bool bf16, int64_t T, int Dm, const float* w_r,
                           const float* bias, int E, int k, int renorm, int32_t* topk_idx,
@@ -37,10 +44,13 @@ cudaError_t launch_router_stream(const void* x, int64_t T, int Dm, const float* 
                                  float* topk_w, int32_t* counts, int32_t* chunk_hist, int* status,
                                  cudaStream_t stream);
 
+// Records kStatusRouting in *status (when not null) if topk_idx or
+// chunk_hist are out of range or inconsistent; the outputs then stay in
+// range (offsets monotone in [0, T*k], sorted_slot and slot_pos in [0, T*k)).
 cudaError_t launch_dispatch(const void* x, bool bf16, int64_t T, int Dm, int E, int k,
                             const int32_t* topk_idx, const int32_t* chunk_hist,
                             int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,
-                            void* x_sorted, cudaStream_t stream);
+                            void* x_sorted, int* status, cudaStream_t stream);
 
 // Epilogue variants of the grouped GEMMs.
 enum EpiMode : int {

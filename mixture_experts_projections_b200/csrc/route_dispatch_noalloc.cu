@@ -16,7 +16,10 @@
 // array, so calls that may overlap on the GPU (different streams without
 // ordering) race on it; calls on one stream are ordered and safe. The router
 // overwrites every entry that the dispatch then reads, so nothing has to be
-// cleared between calls even though the array keeps the previous contents.
+// cleared between calls even though the array keeps the previous contents;
+// should the router give up on a bounded wait, the dispatch checks the
+// entries against the expert indices and reports ROM_ERR_ROUTING instead of
+// using stale ones.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -75,15 +78,20 @@ extern "C" int rom_route_dispatch_noalloc(const void* x, int dtype, int64_t T, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* scratch = rom::noalloc_scratch();
   if (!scratch) return ROM_ERR_CUDA;
+  // The device status word: a bounded wait of the router that runs out, or
+  // routing the dispatch finds inconsistent, is recorded there for
+  // rom_get_status(), as for rom_route() and rom_dispatch().
+  int* st = rom::status_ptr();
+  if (!st) return ROM_ERR_CUDA;
   if (counts && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess)
     return ROM_ERR_CUDA;
   if (T > 0) {
     const cudaError_t e = rom::launch_router(x, bf16, T, Dm, w_r, bias, E, k, renorm, topk_idx,
-                                             topk_w, counts, scratch, nullptr, s);
+                                             topk_w, counts, scratch, st, s);
     if (e != cudaSuccess) return e == cudaErrorInvalidValue ? ROM_ERR_UNSUPPORTED : ROM_ERR_CUDA;
   }
   const cudaError_t e = rom::launch_dispatch(x, bf16, T, Dm, E, k, topk_idx, scratch, offsets,
-                                             sorted_slot, slot_pos, x_sorted, s);
+                                             sorted_slot, slot_pos, x_sorted, st, s);
   if (e != cudaSuccess) return e == cudaErrorInvalidValue ? ROM_ERR_UNSUPPORTED : ROM_ERR_CUDA;
   return ROM_OK;
 }

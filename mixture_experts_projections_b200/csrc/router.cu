@@ -17,9 +17,9 @@
 // per-expert |w_e| this bounds sum_i |x_i w_ie| <= |x| |w_e| (Cauchy-Schwarz),
 // hence the float32 rounding error of each logit by gamma_n |x| |w_e| (+ the
 // bias add), n being the longest accumulation chain and
-// gamma_n = n u / (1 - n u). If a gap that decides S_t or its slot order is
-// not larger than the two bounds, the warp recomputes that token's logits in
-// float64 and decides on those. The selection is then the one exact
+// gamma_n = n u / (1 - n u). If the lower bound of some selected logit does
+// not clear the upper bound of every expert ranked after it, the warp
+// recomputes that token's logits in float64 and decides on those. The selection is then the one exact
 // arithmetic would make, except for gaps below the float64 rounding level.
 // Equal logits go to the lower expert index.
 #include <cuda_bf16.h>
@@ -99,6 +99,13 @@ template <int W>
 __device__ __forceinline__ float seg_sum(float v) {
 #pragma unroll
   for (int o = W / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int W>
+__device__ __forceinline__ float seg_max(float v) {
+#pragma unroll
+  for (int o = W / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 
@@ -366,13 +373,25 @@ __global__ void __launch_bounds__(kRouterThreads)
         float selv[kMaxTopK + 1];
         int slot[VPT];
         seg_select<W, VPT, float>(lv, le, E, k, sel, selv, slot);
+        // Certain when, for every slot j < k, the lower bound of the j-th
+        // selected logit clears the upper bound of every expert ranked after
+        // it: the unselected experts (their largest upper bound, over the
+        // segment) and the selected slots j+1 .. k-1 (a running maximum,
+        // walking the slots from the last). The bounds differ per expert
+        // through |w_e|, so the next-ranked expert alone does not decide.
+        float ub_rest = -INFINITY;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v)
+          if (le[v] < E && slot[v] < 0)
+            ub_rest = fmaxf(ub_rest, lv[v] + gamma * xn * s_wnorm[le[v]] + 1.2e-7f * fabsf(lv[v]));
+        ub_rest = seg_max<W>(ub_rest);
         bool certain = true;
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-          if (j < k && sel[j + 1] >= 0) {
+        for (int j = kMaxTopK - 1; j >= 0; --j) {
+          if (j < k) {
             const float ea = gamma * xn * s_wnorm[sel[j]] + 1.2e-7f * fabsf(selv[j]);
-            const float eb = gamma * xn * s_wnorm[sel[j + 1]] + 1.2e-7f * fabsf(selv[j + 1]);
-            if (!(selv[j] - selv[j + 1] > ea + eb)) certain = false;
+            if (!(selv[j] - ea > ub_rest)) certain = false;
+            ub_rest = fmaxf(ub_rest, selv[j] + ea);
           }
         }
         // Tokens whose float32 decision is not certain: float64 logits.

@@ -12,8 +12,9 @@
 // warps give the logits; every logit has passed through at most
 // m + 5 + 8 + 1 roundings (m = the features of one thread), which with |x| and
 // |w_e| bounds its error by gamma_n |x| |w_e| (Cauchy-Schwarz). A token whose
-// deciding gaps are not larger than the bounds is re-decided on float64
-// logits computed by the same CTA. Equal logits go to the lower expert index.
+// selected logits' lower bounds do not all clear the upper bound of every
+// expert ranked after them is re-decided on float64 logits computed by the
+// same CTA. Equal logits go to the lower expert index.
 // The chunk histograms the dispatch reads are accumulated with integer
 // atomics (the launcher zeroes them), so the result is deterministic.
 #include <cuda_bf16.h>
@@ -131,12 +132,21 @@ __global__ void __launch_bounds__(kThreads)
         if (bi >= 0) used |= 1ull << bi;
       }
     }
+    // The decision is certain when, for every slot j < k, the lower bound of
+    // the j-th selected logit lies above the upper bound of EVERY expert
+    // ranked after it (not only the next one: the bounds differ per expert
+    // through |w_e|, so a lower-ranked expert with a wide bound can reach
+    // higher than the one just below).
     bool certain = true;
-    for (int j = 0; j < k; ++j)
-      if (sel[j + 1] >= 0) {
-        const int a = sel[j], b = sel[j + 1];
-        if (!(l[a] - l[b] > err[a] + err[b])) certain = false;
-      }
+    uint64_t above = 0;
+    for (int j = 0; j < k; ++j) {
+      const int a = sel[j];
+      above |= 1ull << a;
+      const float lb = l[a] - err[a];
+#pragma unroll
+      for (int e = 0; e < EB; ++e)
+        if (!((above >> e) & 1ull) && !(lb > l[e] + err[e])) certain = false;
+    }
     s_refine = certain ? 0 : 1;
   }
   __syncthreads();

@@ -16,9 +16,10 @@
 // of the same tokens, which adds them in order h = 1 .. Q-1. Each logit
 // therefore goes through at most 64 / Q + ceil(d_model / 64) + (Q - 1) + 1
 // roundings in a fixed order; with |x| and |w_e| this bounds its error by
-// gamma_n |x| |w_e| (Cauchy-Schwarz). A token whose deciding gaps are not
-// larger than the bounds is re-decided on float64 logits (warp-cooperative,
-// weights from shared memory). Equal logits go to the lower expert index.
+// gamma_n |x| |w_e| (Cauchy-Schwarz). A token whose selected logits' lower
+// bounds do not all clear the upper bound of every expert ranked after them
+// is re-decided on float64 logits (warp-cooperative, weights from shared
+// memory). Equal logits go to the lower expert index.
 // Every wait is bounded; no block-wide barrier follows the set-up.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -293,12 +294,20 @@ __global__ void __launch_bounds__(Geo<Q>::kThreads, 1)
         for (int e = 0; e < EB; ++e) r = (e == i) ? a[e] : r;
         return r;
       };
+      // Certain when, for every slot j < k, the lower bound of the j-th
+      // selected logit clears the upper bound of every expert ranked after
+      // it (the bounds differ per expert through |w_e|).
       bool certain = true;
+      uint64_t above = 0;
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j)
-        if (j < k && sel[j + 1] >= 0) {
-          const int a = sel[j], b = sel[j + 1];
-          if (!(pick(l, a) - pick(l, b) > pick(err, a) + pick(err, b))) certain = false;
+        if (j < k) {
+          const int a = sel[j];
+          above |= 1ull << a;
+          const float lb = pick(l, a) - pick(err, a);
+#pragma unroll
+          for (int e = 0; e < EB; ++e)
+            if (e < E && !((above >> e) & 1ull) && !(lb > l[e] + err[e])) certain = false;
         }
       unsigned todo = __ballot_sync(0xffffffffu, valid && !certain);
       while (todo) {

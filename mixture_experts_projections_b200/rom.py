@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librom.so")
 
 ROM_OK, ROM_ERR_INVALID_ARG, ROM_ERR_UNSUPPORTED, ROM_ERR_WORKSPACE, ROM_ERR_CUDA, \
-    ROM_ERR_TIMEOUT = range(6)
+    ROM_ERR_TIMEOUT, ROM_ERR_ROUTING = range(7)
 ROM_F32, ROM_BF16 = 0, 1
 ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ = 0, 1, 2
 ROM_COMBINE_SUM, ROM_COMBINE_GATE = 0, 1

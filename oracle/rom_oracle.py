@@ -19,7 +19,7 @@ Plain, slow, float64 numpy. Every function follows a passage of the pages:
   Extended abstract, second paragraph -- expert in-projections emit the X, B
   and C streams, and the routing-weighted streams are summed.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * The short convolution and selective scan between the projections are not
   changed by the method; the oracle stands the identity in for them (Y = H).

@@ -3,11 +3,13 @@ layout and compare CUDA results with the CPU oracle.
 
 Tolerances (the floating-point bar of the parity tests):
   * routing indices, counts, offsets and the permutation: bit-exact;
-  * routing weights r: relative 2e-5. r = exp(l_e - m) / sum, so its
-    relative error is about twice the absolute error of the logits, and a
-    float32 logit (d_model products accumulated in float32) carries up to
-    ~1e-5 of rounding at d_model of a few thousand -- the selection itself
-    stays exact (near ties are re-decided in float64);
+  * routing weights r: a per-token relative bound derived from the float32
+    arithmetic of the routers (``routing_weight_rtol``): twice the largest
+    rounding error a float32 logit can carry (gamma_n * sum_i |x_i w_ie|,
+    n = the longest accumulation chain of any router), plus the softmax's own
+    rounding ((E + 8) u and 2 u times the logit spread, u = 2^-24). It holds
+    for every token whatever the router; the largest measured error and its
+    ratio to the bound are printed at the end of the run;
   * bf16 outputs: max abs error <= 2e-2 and relative Frobenius error <= 5e-3
     against the float64 oracle. The full-size workloads are held to exactly
     that. The synthetic test shapes and the bf16 intermediate h can reach
@@ -28,7 +30,10 @@ from mixture_experts_projections_b200.inputs import bf16_bits
 BF16_MAX_ABS = 2e-2
 BF16_REL_FRO = 5e-3
 F32_REL = 1e-5
-TOPK_W_RTOL = 2e-5
+U32 = 2.0 ** -24  # unit roundoff of float32
+
+# Largest routing-weight errors seen in this run (printed by conftest.py).
+ROUTING_WEIGHT_STATS = {"checks": 0, "tokens": 0, "max_rel": 0.0, "max_ratio": 0.0}
 
 
 def to_dev(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
@@ -87,10 +92,43 @@ def assert_close(got, ref, dtype: str, what: str, magnitude_scaled_abs: bool = F
     return max_abs, rel
 
 
-def assert_routing_matches(gpu_idx: np.ndarray, gpu_w: np.ndarray, rt: dict, band=1e-9):
+def routing_weight_rtol(x, w_r, bias=None) -> np.ndarray:
+    """Per-token bound on |r_gpu - r| / r for the float32 routing weights.
+
+    A float32 logit accumulated over d_model products in a chain of at most n
+    roundings is off by at most gamma_n * sum_i |x_i w_ie| (+ u |b_e| for the
+    bias add); a token decided on float64 logits carries at most u |l_e| from
+    the final cast. Every router's chain is shorter than
+    n = d_model / 32 + 32 (per-token router: features per thread + 5 + 8 + 2;
+    streaming router: 64 / Q + d_model / 64 + Q + 1; register-tiled router:
+    the lane's slice + 7), and gamma_n gets the 1 % slack the kernels use.
+    ln r = l_j - logsumexp(l), so logit errors move ln r by at most twice the
+    largest one. The softmax itself adds at most (E + 8) u (expf within 2 ulp
+    per term, the sum of E positive terms, the division) plus u |l - max l|
+    for each of the two exponent arguments.
+    """
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w_r, np.float64)
+    E = w.shape[1]
+    n = x.shape[1] / 32.0 + 32.0
+    gamma = 1.01 * n * U32 / (1.0 - n * U32)
+    logits = x @ w
+    delta = gamma * (np.abs(x) @ np.abs(w))
+    if bias is not None:
+        b = np.asarray(bias, np.float64)
+        logits = logits + b[None, :]
+        delta = delta + U32 * np.abs(b)[None, :]
+    delta = delta + 2.0 * U32 * np.abs(logits)
+    spread = logits.max(axis=1) - logits.min(axis=1)
+    return 2.0 * delta.max(axis=1) + (E + 8) * U32 + 2.0 * U32 * spread
+
+
+def assert_routing_matches(gpu_idx: np.ndarray, gpu_w: np.ndarray, rt: dict, *, x, w_r,
+                           bias=None, band=1e-9):
     """Exact index equality; tokens whose oracle decision margin is below
     `band` (numerically ambiguous in float64) may differ only to another
-    valid choice. Returns the number of such ambiguous tokens."""
+    valid choice. Routing weights within ``routing_weight_rtol`` of the
+    oracle's, token by token. Returns the number of ambiguous tokens."""
     ref_idx = rt["topk_idx"]
     ambiguous = rt["margin"] <= band
     mism = np.any(gpu_idx != ref_idx, axis=1)
@@ -102,5 +140,16 @@ def assert_routing_matches(gpu_idx: np.ndarray, gpu_w: np.ndarray, rt: dict, ban
         chosen = lg[gpu_idx[t]]
         assert np.all(np.diff(chosen) <= band), "ambiguous token: slots not in descending order"
     ok = ~mism
-    np.testing.assert_allclose(gpu_w[ok], rt["topk_w"][ok], rtol=TOPK_W_RTOL, atol=1e-7)
+    ref_w = np.asarray(rt["topk_w"], np.float64)
+    rel = np.abs(np.asarray(gpu_w, np.float64) - ref_w) / np.maximum(ref_w, 1e-300)
+    bound = routing_weight_rtol(x, w_r, bias)[:, None]
+    bad_w = ok[:, None] & (rel > bound)
+    assert not np.any(bad_w), (f"routing weights of {int(bad_w.any(axis=1).sum())} tokens exceed "
+                               f"the bound: worst rel {rel[bad_w].max():.3e}")
+    if np.any(ok):
+        st = ROUTING_WEIGHT_STATS
+        st["checks"] += 1
+        st["tokens"] += int(ok.sum())
+        st["max_rel"] = max(st["max_rel"], float(rel[ok].max()))
+        st["max_ratio"] = max(st["max_ratio"], float((rel / bound)[ok].max()))
     return int(ambiguous.sum())

@@ -42,6 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings_and_version(lib):
     assert lib.rom_status_string(0) == b"ROM_OK"
     assert lib.rom_status_string(5) == b"ROM_ERR_TIMEOUT"
+    assert lib.rom_status_string(6) == b"ROM_ERR_ROUTING"
     assert lib.rom_status_string(99) == b"ROM_ERR_UNKNOWN"
     assert lib.rom_version() >= 1
 

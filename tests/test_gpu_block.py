@@ -56,7 +56,7 @@ def test_block_forward_matches_oracle(T, Dm, De, E, k, renorm, dtype, std, bias)
     assert rom.rom_get_status() == 0
     rb = out.routing
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
-                           ref)
+                           ref, x=inp["x"], w_r=inp["w_r"], bias=inp["bias"])
     assert_close(to_np(out.out), ref["O"], dtype, "O", magnitude_scaled_abs=True)
     if k == 1:
         # the intermediate h in sorted order matches Y (.) G of the oracle
@@ -73,7 +73,8 @@ def test_tiny_fp32_workload():
     out = rom.block_forward(d["x"], d["w_r"], d["bias"], d["w_conv"], d["w_gate"], d["w_out"],
                             k=wl.k)
     assert_routing_matches(out.routing.topk_idx.cpu().numpy(),
-                           out.routing.topk_w.cpu().numpy().astype(np.float64), ref)
+                           out.routing.topk_w.cpu().numpy().astype(np.float64), ref, x=inp["x"],
+                           w_r=inp["w_r"])
     assert_close(to_np(out.out), ref["O"], "f32", "O")
 
 
@@ -108,7 +109,7 @@ def test_inproj_matches_oracle(T, Dm, N, E, k, renorm):
                                  weights_to_dev(inp["w"], "bf16"), k=k, renorm=renorm)
     torch.cuda.synchronize()
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
-                           ref)
+                           ref, x=inp["x"], w_r=inp["w_r"])
     assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
 
 
@@ -136,7 +137,7 @@ def test_inproj_skewed_routing_small_batch():
                                  weights_to_dev(inp["w"], "bf16"), k=1, renorm=False)
     torch.cuda.synchronize()
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
-                           ref)
+                           ref, x=inp["x"], w_r=inp["w_r"])
     assert_close(to_np(out), ref["S"], "bf16", "S", magnitude_scaled_abs=True)
 
 

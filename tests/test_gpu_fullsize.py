@@ -35,7 +35,8 @@ def test_block_workload_full_size(name):
     rb = out.routing
     rt = orc.route(inp["x"], inp["w_r"], wl.k, bias=inp["bias"], renorm=wl.renorm)
     idx = rb.topk_idx.cpu().numpy()
-    amb = assert_routing_matches(idx, rb.topk_w.cpu().numpy().astype(np.float64), rt)
+    amb = assert_routing_matches(idx, rb.topk_w.cpu().numpy().astype(np.float64), rt,
+                                 x=inp["x"], w_r=inp["w_r"], bias=inp["bias"])
     assert amb == 0
     dsp = orc.dispatch(idx, wl.E)
     R = wl.T * wl.k
@@ -59,5 +60,5 @@ def test_decode_swimba_inproj_full():
                                  weights_to_dev(inp["w"], "bf16"), k=wl.k)
     torch.cuda.synchronize()
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
-                           ref)
+                           ref, x=inp["x"], w_r=inp["w_r"])
     assert_close(to_np(out), ref["S"], "bf16", "S")

@@ -6,9 +6,11 @@ pool) cannot pass the workspace that rom_route() and rom_dispatch() exchange.
 rom_route_dispatch_noalloc keeps that scratch in a fixed device array inside
 the library instead. These tests call it through the C ABI, twice in a row
 (the array keeps the previous call's contents), and check that it returns
-exactly what the two workspace-based calls return: bit-identical routing
-indices, counts, offsets, permutation and gathered rows, and routing weights
-within the routing-weight tolerance of the other parity tests.
+exactly what the two workspace-based calls return: the same kernels run on
+the same inputs, so routing indices and weights, counts, offsets,
+permutation and gathered rows are bit-identical. They also check that a call
+leaves the device's free memory unchanged, and that a sequence of calls of
+different sizes and expert counts never sees the previous call's scratch.
 
 The file is named so that pytest collects it last.
 """
@@ -20,7 +22,7 @@ import torch
 
 from mixture_experts_projections_b200 import rom
 from mixture_experts_projections_b200.inputs import make_block_inputs
-from parity_util import TOPK_W_RTOL, to_dev
+from parity_util import to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -50,11 +52,19 @@ def _noalloc_call(lib, x, w_r, bias, E, k, renorm):
     return out
 
 
+def _assert_same(got, ref, R):
+    for n in ("topk_idx", "topk_w", "counts", "offsets"):
+        assert torch.equal(got[n], getattr(ref, n)), n
+    for n in ("sorted_slot", "slot_pos", "x_sorted"):
+        assert torch.equal(got[n], getattr(ref, n)[:R]), n
+
+
 CASES = [
     # T, Dm, E, k, renorm, dtype
-    (1000, 256, 8, 1, False, "bf16"),
+    (1000, 256, 8, 1, False, "bf16"),     # per-token router
     (777, 512, 16, 2, True, "bf16"),
-    (300, 64, 5, 2, False, "f32"),
+    (300, 64, 5, 2, False, "f32"),        # register-tiled router
+    (4096, 2048, 8, 1, False, "bf16"),    # streaming router (32 chunks of histograms)
 ]
 
 
@@ -69,14 +79,53 @@ def test_noalloc_matches_workspace_entry_points_on_two_calls(T, Dm, E, k, renorm
     for _ in range(2):
         got = _noalloc_call(lib, x, w_r, None, E, k, renorm)
         torch.cuda.synchronize()
-        assert torch.equal(got["topk_idx"], ref.topk_idx)
-        np.testing.assert_allclose(got["topk_w"].cpu().numpy(), ref.topk_w.cpu().numpy(),
-                                   rtol=TOPK_W_RTOL, atol=0)
-        assert torch.equal(got["counts"], ref.counts)
-        assert torch.equal(got["offsets"], ref.offsets)
-        assert torch.equal(got["sorted_slot"], ref.sorted_slot[:R])
-        assert torch.equal(got["slot_pos"], ref.slot_pos[:R])
-        assert torch.equal(got["x_sorted"], ref.x_sorted[:R])
+        _assert_same(got, ref, R)
+    assert rom.rom_get_status() == rom.ROM_OK
+
+
+def test_noalloc_sequence_of_sizes_never_reads_stale_scratch():
+    """A large call with 16 experts, then smaller ones with 5 and 8 experts,
+    then the large one again: each equals the workspace-based calls, although
+    the shared array still holds the previous call's histograms."""
+    lib = rom.load_library()
+    seq = [(3000, 512, 16, 2, True, "bf16"), (500, 256, 5, 1, False, "bf16"),
+           (2100, 512, 8, 1, False, "bf16"), (130, 128, 8, 2, False, "f32"),
+           (3000, 512, 16, 2, True, "bf16")]
+    for i, (T, Dm, E, k, renorm, dtype) in enumerate(seq):
+        inp = make_block_inputs(T, Dm, 1, E, seed=100 + i, dtype=dtype, router_std=0.1)
+        x = to_dev(inp["x"], dtype)
+        w_r = to_dev(inp["w_r"], "f32")
+        ref = rom.route_and_dispatch(x, w_r, None, E, k, renorm)
+        got = _noalloc_call(lib, x, w_r, None, E, k, renorm)
+        torch.cuda.synchronize()
+        _assert_same(got, ref, T * k)
+        assert rom.rom_get_status() == rom.ROM_OK
+
+
+def test_noalloc_call_allocates_no_device_memory():
+    """After a first call (which loads the kernels and looks up the array's
+    address), a call leaves the device's free memory exactly as it was."""
+    lib = rom.load_library()
+    T, Dm, E, k = 4096, 2048, 8, 1
+    inp = make_block_inputs(T, Dm, 1, E, seed=5, router_std=0.1)
+    x = to_dev(inp["x"], "bf16")
+    w_r = to_dev(inp["w_r"], "f32")
+    first = _noalloc_call(lib, x, w_r, None, E, k, False)
+    torch.cuda.synchronize()
+    out = {n: torch.empty_like(t) for n, t in first.items()}
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    code = lib.rom_route_dispatch_noalloc(
+        _p(x), rom.ROM_BF16, T, Dm, _p(w_r), None, E, k, 0, _p(out["topk_idx"]),
+        _p(out["topk_w"]), _p(out["counts"]), _p(out["offsets"]), _p(out["sorted_slot"]),
+        _p(out["slot_pos"]), _p(out["x_sorted"]),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert code == rom.ROM_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    for n in first:
+        assert torch.equal(out[n], first[n]), n
     assert rom.rom_get_status() == rom.ROM_OK
 
 
