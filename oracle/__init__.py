@@ -4,7 +4,7 @@ Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
 reference arm may import this package. The product path never does.
 """
 from .rom_oracle import (block_backward, block_forward, dispatch, inproj_forward, route,
-                         sigmoid, silu, silu_grad, softmax)
+                         sigmoid, silu, silu_grad, softmax, variant_block_forward)
 
 __all__ = ["block_backward", "block_forward", "dispatch", "inproj_forward", "route", "sigmoid",
-           "silu", "silu_grad", "softmax"]
+           "silu", "silu_grad", "softmax", "variant_block_forward"]

@@ -273,3 +273,69 @@ def block_backward(x, w_r, w_in, w_g, w_out, dout, k, bias=None, renorm=False):
     dbias = dlogits.sum(axis=0)
     return dict(dX=dX, dW_in=dW_in, dW_g=dW_g, dW_out=dW_out, dlogits=dlogits, dr=dr,
                 dW_r=dW_r, dbias=dbias, forward=fw)
+
+
+def variant_block_forward(x, w_in, w_g, w_out, k, routers, weighted, bias=None, renorm=False,
+                          tokens=None):
+    """Mamba projection block whose three projections are each dense or routed.
+
+    Covers the configurations the RoM page compares (Knowl 3 and Knowl 4):
+      * RoM (Conv, Gate, Out): one router shared by the three projections;
+        only Out is weighted by r (Knowl 1). Equals ``block_forward``.
+      * RoM (Gate, Out): Conv is a dense projection; Gate and Out share one
+        router (Knowl 3, "Samba + RoM (Gate, Out)").
+      * Independent MoE on Conv, Gate and Out: each projection is a
+        conventional MoE layer with its own router, its experts' outputs
+        weighted by that router's probabilities (Knowl 4).
+
+    ``routers`` maps "conv", "gate" and "out" to a router weight [D_m, E] or
+    to None for a dense projection (the weight stack then holds one matrix
+    and it is applied to every token with weight 1). Routers are evaluated
+    separately for each projection; passing the same matrix twice shares the
+    decision, since it is the same computation. ``weighted`` maps the three
+    names to True when that projection's expert outputs are scaled by r.
+    ``bias`` is an optional additive logit bias used by every router.
+
+    H_t = sum_{i in S^conv_t} w^conv_{t,i} x_t W_in,i
+    G_t = SiLU(sum_{i in S^gate_t} w^gate_{t,i} x_t W_g,i)
+    O_t = sum_{i in S^out_t} w^out_{t,i} (Y_t (.) G_t) W_out,i,   Y = H,
+    with w = r for a weighted projection, 1 otherwise.
+    Returns a dict with O, H, Gpre, G, YG and the three routings.
+    """
+    x = _f64(x)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+    T = x.shape[0]
+
+    def routing(name):
+        w_r = routers.get(name)
+        if w_r is None:
+            return None
+        return route(x, w_r, k, bias=bias, renorm=renorm)
+
+    def project(name, a, w):
+        """Sum over the projection's selected experts of (weight) * a W_i."""
+        rt = rts[name]
+        N = np.shape(w)[2]
+        out = np.zeros((T, N))
+        if rt is None:
+            return out + a @ _f64(w[0])
+        S, r = rt["topk_idx"], rt["topk_w"]
+        for i in range(np.shape(w)[0]):
+            for j in range(k):
+                sel = np.nonzero(S[:, j] == i)[0]
+                if sel.size == 0:
+                    continue
+                part = a[sel] @ _f64(w[i])
+                if weighted[name]:
+                    part = r[sel, j][:, None] * part
+                out[sel] += part
+        return out
+
+    rts = {n: routing(n) for n in ("conv", "gate", "out")}
+    H = project("conv", x, w_in)
+    Gpre = project("gate", x, w_g)
+    G = silu(Gpre)
+    YG = H * G
+    O = project("out", YG, w_out)
+    return dict(O=O, H=H, Gpre=Gpre, G=G, YG=YG, routing=rts)

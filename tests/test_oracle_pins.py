@@ -355,3 +355,133 @@ def test_oracle_regression_fixture():
         np.testing.assert_allclose(bw["forward"]["O"], c["O"], rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(bw["dX"], c["dX"], rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(bw["dlogits"], c["dlogits"], rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------- projection variants (Knowl 3, Knowl 4)
+
+
+def _brute_routing(x, w_r, k, renorm):
+    """Selection mask and weights [T, E] by a rank count: expert e is chosen
+    when fewer than k experts beat it (larger logit, or equal logit and a
+    lower index); weights from scipy's softmax."""
+    lg = x @ w_r
+    T, E = lg.shape
+    p = sp_softmax(lg, axis=1)
+    mask = np.zeros((T, E))
+    for t in range(T):
+        for e in range(E):
+            beats = sum(1 for f in range(E) if lg[t, f] > lg[t, e] or (lg[t, f] == lg[t, e] and f < e))
+            mask[t, e] = 1.0 if beats < k else 0.0
+    w = p * mask
+    if renorm:
+        w = w / w.sum(axis=1, keepdims=True)
+    return mask, w
+
+
+def _brute_variant(x, w_in, w_g, w_out, k, routers, weighted, renorm):
+    """Every expert of every projection evaluated densely, then masked."""
+    x = x.astype(np.float64)
+
+    def proj(name, a, w):
+        if routers[name] is None:
+            return a @ w[0].astype(np.float64)
+        mask, wt = _brute_routing(x, routers[name].astype(np.float64), k, renorm)
+        c = wt if weighted[name] else mask
+        return sum(c[:, [e]] * (a @ w[e].astype(np.float64)) for e in range(w.shape[0]))
+
+    H = proj("conv", x, w_in)
+    G = _silu_ref(proj("gate", x, w_g))
+    return proj("out", H * G, w_out)
+
+
+def _three_routers(Dm, E, seed, std=0.5):
+    rng = np.random.default_rng(seed)
+    return [(std * rng.standard_normal((Dm, E))).astype(np.float32) for _ in range(3)]
+
+
+@pytest.mark.parametrize("k,renorm", [(1, False), (2, False), (2, True)])
+def test_variant_with_one_shared_router_is_rom(k, renorm):
+    inp = make_block_inputs(40, 12, 10, 5, seed=31, router_std=0.4)
+    w_r = inp["w_r"]
+    rom = orc.block_forward(inp["x"], w_r, inp["w_conv"], inp["w_gate"], inp["w_out"], k=k,
+                            renorm=renorm)
+    var = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"], k,
+                                    {"conv": w_r, "gate": w_r, "out": w_r},
+                                    {"conv": False, "gate": False, "out": True}, renorm=renorm)
+    np.testing.assert_allclose(var["O"], rom["O"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("k,renorm,E", [(1, False, 4), (2, False, 5), (2, True, 3), (3, False, 6)])
+def test_independent_moe_matches_brute_force(k, renorm, E):
+    inp = make_block_inputs(30, 10, 9, E, seed=40 + E)
+    rc, rg, ro = _three_routers(10, E, seed=E)
+    routers = {"conv": rc, "gate": rg, "out": ro}
+    weighted = {"conv": True, "gate": True, "out": True}
+    var = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"], k,
+                                    routers, weighted, renorm=renorm)
+    ref = _brute_variant(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"], k, routers,
+                         weighted, renorm)
+    np.testing.assert_allclose(var["O"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_independent_moe_top1_closed_form():
+    """Top-1: each projection is its own router's winner, scaled by its
+    probability: O = p^o ((p^c x W_in,c) (.) SiLU(p^g x W_g,g)) W_out,o."""
+    E = 4
+    inp = make_block_inputs(25, 8, 6, E, seed=7)
+    rc, rg, ro = _three_routers(8, E, seed=3)
+    var = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                                    {"conv": rc, "gate": rg, "out": ro},
+                                    {"conv": True, "gate": True, "out": True})
+    x = inp["x"].astype(np.float64)
+    for t in range(x.shape[0]):
+        pc, pg, po = (sp_softmax(x[t] @ r.astype(np.float64)) for r in (rc, rg, ro))
+        c, g, o = int(np.argmax(pc)), int(np.argmax(pg)), int(np.argmax(po))
+        h = pc[c] * (x[t] @ inp["w_conv"][c])
+        gg = _silu_ref(pg[g] * (x[t] @ inp["w_gate"][g]))
+        np.testing.assert_allclose(var["O"][t], po[o] * ((h * gg) @ inp["w_out"][o]), rtol=1e-12,
+                                   atol=1e-13)
+
+
+def test_all_dense_variant_is_the_dense_projection():
+    inp = make_block_inputs(20, 8, 6, 1, seed=2)
+    var = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                                    {"conv": None, "gate": None, "out": None},
+                                    {"conv": True, "gate": True, "out": True})
+    x = inp["x"].astype(np.float64)
+    dense = ((x @ inp["w_conv"][0]) * _silu_ref(x @ inp["w_gate"][0])) @ inp["w_out"][0]
+    np.testing.assert_allclose(var["O"], dense, rtol=1e-13, atol=1e-13)
+
+
+def test_rom_gate_out_variant_top1_closed_form():
+    """RoM (Gate, Out): Conv dense, Gate and Out share one router; top-1:
+    O = p_e ((x W_in) (.) SiLU(x W_g,e)) W_out,e."""
+    E = 4
+    inp = make_block_inputs(25, 8, 6, E, seed=8, router_std=0.4)
+    w_in_dense = inp["w_conv"][:1]
+    var = orc.variant_block_forward(inp["x"], w_in_dense, inp["w_gate"], inp["w_out"], 1,
+                                    {"conv": None, "gate": inp["w_r"], "out": inp["w_r"]},
+                                    {"conv": False, "gate": False, "out": True})
+    x = inp["x"].astype(np.float64)
+    for t in range(x.shape[0]):
+        p = sp_softmax(x[t] @ inp["w_r"].astype(np.float64))
+        e = int(np.argmax(p))
+        h = (x[t] @ w_in_dense[0]) * _silu_ref(x[t] @ inp["w_gate"][e])
+        np.testing.assert_allclose(var["O"][t], p[e] * (h @ inp["w_out"][e]), rtol=1e-12,
+                                   atol=1e-13)
+
+
+def test_independent_routers_relabel_one_projection_alone():
+    """Permuting the expert labels of the Gate router together with the Gate
+    experts, and nothing else, leaves O unchanged: each projection follows its
+    own router."""
+    E = 5
+    inp = make_block_inputs(30, 10, 8, E, seed=12)
+    rc, rg, ro = _three_routers(10, E, seed=9)
+    weighted = {"conv": True, "gate": True, "out": True}
+    a = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"], 2,
+                                  {"conv": rc, "gate": rg, "out": ro}, weighted)
+    perm = np.array([3, 0, 4, 1, 2])
+    b = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"][perm], inp["w_out"], 2,
+                                  {"conv": rc, "gate": rg[:, perm], "out": ro}, weighted)
+    np.testing.assert_allclose(a["O"], b["O"], rtol=1e-12, atol=1e-12)
