@@ -11,15 +11,20 @@ HBM when the timed region starts. Between timed steps the L2 is flushed (a
 256 MiB write, outside the step's events), except where the step's inputs
 (tokens and weights) exceed twice the L2: then every step streams them from
 HBM anyway, and a flush would only add the write-back of its own dirty lines
-to the next step. `config["l2"]` says which. Each step is timed with CUDA
+to the next step. The line's "l2" key says which. Each step is timed with CUDA
 events on the launching stream; the dominant kernel is bracketed by its own
 events for the roofline. Under torchrun every rank runs an independent
 replica on its own GPU (the block needs no collective in the forward); the
 reported time is the max over ranks and `value` counts all ranks' tokens.
 
-`--impl reference` times the CPU oracle (the float64 numpy definition) on a
-bounded sample of the same workload on the host cores; under torchrun only
-rank 0 runs it.
+A single-GPU run also times the other configurations of the block (decode
+in-projection, top-2 forward + backward, load-imbalanced, tiny float32, and
+the independently routed and RoM (Gate, Out) projection variants at the
+prefill shape) and reports them under "workloads"; `--no-extra` skips them.
+
+`--impl reference` times the CPU oracle (the float64 numpy definition) on the
+host cores, on the whole workload per step when that fits about two minutes
+(else a random token sample); under torchrun only rank 0 runs it.
 
 Prints one JSON line (rank 0).
 """
@@ -114,6 +119,11 @@ def block_flops(wl):
     R = wl.T * wl.k
     if wl.kind == "inproj":
         return {"inproj": 2.0 * R * wl.Dm * wl.De}
+    if wl.kind == "variant":
+        # Conv and Gate as two projections (dense ones over the T tokens), then Out
+        rows_conv = wl.T if wl.variant == "gate_out" else R
+        return {"conv": 2.0 * rows_conv * wl.Dm * wl.De, "gate": 2.0 * R * wl.Dm * wl.De,
+                "out": 2.0 * R * wl.De * wl.Dm}
     f = {"conv_gate": 4.0 * R * wl.Dm * wl.De, "out": 2.0 * R * wl.De * wl.Dm}
     if wl.backward:  # dgrad (Out, In+Gate) and wgrad (Out, In+Gate): twice the forward
         f["backward"] = 2.0 * (f["conv_gate"] + f["out"])
@@ -124,6 +134,18 @@ def inproj_bytes(wl, n_experts_hit):
     """Algorithmic HBM bytes of the routed in-projection: the weights of the
     experts that received tokens, x in, the output out (bf16)."""
     return n_experts_hit * wl.Dm * wl.De * 2 + wl.T * wl.Dm * 2 + wl.T * wl.De * 2
+
+
+def variant_spec(wl, inp):
+    """Routers (None: dense) and weighting of the projections of a variant
+    workload: which router drives which projection."""
+    if wl.variant == "independent":
+        return ({"conv": inp["w_r"], "gate": inp["w_r_gate"], "out": inp["w_r_out"]},
+                {"conv": True, "gate": True, "out": True})
+    if wl.variant == "gate_out":
+        return ({"conv": None, "gate": inp["w_r"], "out": inp["w_r"]},
+                {"conv": False, "gate": False, "out": True})
+    raise ValueError(wl.variant)
 
 
 # ------------------------------------------------------------------ clocks
@@ -214,6 +236,11 @@ def oracle_sample_run(wl, inp, tokens):
     t0 = time.perf_counter()
     if wl.kind == "inproj":
         orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=wl.k, tokens=tokens)
+    elif wl.kind == "variant":
+        routers, weighted = variant_spec(wl, inp)
+        w_conv = inp["w_conv"][:1] if routers["conv"] is None else inp["w_conv"]
+        orc.variant_block_forward(inp["x"], w_conv, inp["w_gate"], inp["w_out"], wl.k, routers,
+                                  weighted, renorm=wl.renorm, tokens=tokens)
     else:
         orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
                           k=wl.k, bias=inp["bias"], renorm=wl.renorm, tokens=tokens)
@@ -262,56 +289,31 @@ def job_tokens_per_s(tokens_per_rank, world, step_ms):
     return tokens_per_rank * world / (step_ms / 1e3)
 
 
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
+def build_workload(torch, rom, wl, inp):
+    """Device inputs of one workload and its step as phases.
 
-    from mixture_experts_projections_b200 import rom
-
-    torch.cuda.set_device(local_rank)
-    rom.load_library()
-    wl = WORKLOADS[args.workload]
+    Returns a dict: phases [(name, fn)], dominant (fn, "flop"|"byte" work
+    function of the routing counts), out (result tensor), counts (expert
+    counts of the main routing), x, in_bytes (a step's inputs), launches
+    (our kernels per step), e2e (the public host-buffer call or None).
+    """
     bf16 = wl.dtype == "bf16"
-    inp = make_workload_inputs(wl, seed=0)
-    stream = torch.cuda.current_stream()
     x = to_dev(torch, inp["x"], bf16)
     w_r = to_dev(torch, inp["w_r"], False)
     bias = None if inp.get("bias") is None else to_dev(torch, inp["bias"], False)
-    if wl.kind == "inproj":
-        w = to_dev(torch, inp["w"], bf16).transpose(1, 2).contiguous()
-        bufs = rom.RoutingBuffers(wl.T, wl.Dm, wl.E, wl.k, x.dtype, x.device)
-        out = torch.empty((wl.T, wl.De), dtype=x.dtype, device=x.device)
-        slots = (torch.empty((wl.T * wl.k, wl.De), dtype=torch.float32, device=x.device)
-                 if wl.k > 1 else None)
-    else:
-        ws = {n: to_dev(torch, inp[n], bf16).transpose(1, 2).contiguous()
-              for n in ("w_conv", "w_gate", "w_out")}
-        bufs = rom.BlockBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
-    del inp["x"]
-    # inputs of one step: the tokens and every weight the step reads
-    in_bytes = x.numel() * x.element_size() + w_r.numel() * w_r.element_size()
-    if wl.kind == "inproj":
-        in_bytes += w.numel() * w.element_size()
-    else:
-        in_bytes += sum(t.numel() * t.element_size() for t in ws.values())
-    if wl.backward:
-        in_bytes += x.numel() * x.element_size()  # dO, same shape as X
-    flush_l2 = in_bytes < 2 * L2_BYTES
-    flush = (torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=x.device)
-             if flush_l2 else None)
-    l2_note = ("flushed before every timed step (256 MiB write)" if flush_l2 else
-               f"not flushed: the step's inputs ({in_bytes / 1e6:.0f} MB) exceed twice the L2 "
-               f"({L2_BYTES / 1e6:.0f} MB) and are streamed from HBM every step")
-
-    def do_flush():
-        if flush is not None:
-            flush.zero_()
     R = wl.T * wl.k
     dt = rom.ROM_BF16 if bf16 else rom.ROM_F32
-
-    # The step as three phases: route + dispatch, the dominant projection
-    # (Conv+Gate, or the in-projection), and the rest.
+    flops = block_flops(wl)
+    in_bytes = x.numel() * x.element_size() + w_r.numel() * w_r.element_size()
+    res = {"x": x}
     if wl.kind == "inproj":
+        w = to_dev(torch, inp["w"], bf16).transpose(1, 2).contiguous()
+        in_bytes += w.numel() * w.element_size()
+        bufs = rom.RoutingBuffers(wl.T, wl.Dm, wl.E, wl.k, x.dtype, x.device)
+        out = torch.empty((wl.T, wl.De), dtype=x.dtype, device=x.device)
+        slots = (torch.empty((R, wl.De), dtype=torch.float32, device=x.device)
+                 if wl.k > 1 else None)
+
         def ph_route():
             rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, bufs)
 
@@ -323,9 +325,55 @@ def run_ours(args, rank, world, local_rank):
         def ph_p1():
             if wl.k > 1:
                 rom.rom_combine(rom.ROM_COMBINE_SUM, dt, slots, wl.T, wl.k, wl.De, None, out)
-        out_t = out
-        counts_t = bufs.counts
+        res.update(phases=[("route_dispatch", ph_route), ("proj0", ph_p0), ("proj1", ph_p1)],
+                   dominant=(ph_p0, "byte",
+                             lambda counts: inproj_bytes(wl, int(np.count_nonzero(counts)))),
+                   out=out, counts=bufs.counts, launches=3 + (1 if wl.k > 1 else 0))
+        pipe = rom.HostPipeline(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
+        res["e2e"] = (pipe, lambda hx, ho: pipe.inproj_forward(hx, w_r, w, ho, renorm=wl.renorm,
+                                                                bias=bias))
+    elif wl.kind == "variant":
+        routers, weighted = variant_spec(wl, inp)
+        d_r = {}
+        for n, r in routers.items():  # the same array -> one device tensor (shared routing)
+            if r is not None and id(r) not in d_r:
+                d_r[id(r)] = w_r if r is inp["w_r"] else to_dev(torch, r, False)
+        d_routers = {n: (None if r is None else d_r[id(r)]) for n, r in routers.items()}
+        ws = {n: to_dev(torch, inp[n][:1] if (routers[p] is None) else inp[n], bf16)
+              .transpose(1, 2).contiguous()
+              for n, p in (("w_conv", "conv"), ("w_gate", "gate"), ("w_out", "out"))}
+        in_bytes += sum(t.numel() * t.element_size() for t in ws.values())
+        in_bytes += sum(t.numel() * t.element_size() for t in d_r.values() if t is not w_r)
+        bufs = rom.VariantBuffers(wl.T, wl.Dm, wl.De, wl.k, x.dtype, x.device)
+        args = (x, d_routers, weighted, ws["w_conv"], ws["w_gate"], ws["w_out"], wl.k)
+
+        def phase(names):
+            return lambda: rom.variant_block_forward(*args, renorm=wl.renorm, bias=bias,
+                                                     bufs=bufs, phases=names)
+        phase(("route", "project", "output"))()  # makes the routing buffers
+        rb_c = bufs.routings[id(d_routers["conv"])] if d_routers["conv"] is not None else None
+
+        def dominant():  # the Conv projection alone
+            if rb_c is None:
+                rom.rom_expert_proj(rom.ROM_PROJ_SLOTS, x, ws["w_conv"], None, 1, 1, None, None,
+                                    None, bufs.uz[:wl.T])
+            else:
+                rom.rom_expert_proj(rom.ROM_PROJ_SLOTS, rb_c.x_sorted[:R], ws["w_conv"], None,
+                                    wl.E, wl.k, rb_c.offsets, rb_c.sorted_slot,
+                                    rb_c.topk_w if weighted["conv"] else None, bufs.uz[:R])
+        n_routings = len(d_r)
+        main_rb = bufs.routings[id(w_r)]
+        res.update(phases=[("route_dispatch", phase(("route",))),
+                           ("proj0", phase(("project",))), ("proj1", phase(("output",)))],
+                   dominant=(dominant, "flop", lambda counts: flops["conv"]),
+                   out=bufs.out, counts=main_rb.counts,
+                   launches=2 * n_routings + 2 + 2 + (1 if wl.k > 1 else 0))
+        res["e2e"] = None
     else:
+        ws = {n: to_dev(torch, inp[n], bf16).transpose(1, 2).contiguous()
+              for n in ("w_conv", "w_gate", "w_out")}
+        in_bytes += sum(t.numel() * t.element_size() for t in ws.values())
+        bufs = rom.BlockBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
         rb = bufs.routing
 
         def ph_route():
@@ -348,40 +396,68 @@ def run_ours(args, rank, world, local_rank):
                                     bufs.o_slots)
                 rom.rom_combine(rom.ROM_COMBINE_SUM, dt, bufs.o_slots, wl.T, wl.k, wl.Dm, None,
                                 bufs.out)
-        out_t = bufs.out
-        counts_t = rb.counts
-    phases = [ph_route, ph_p0, ph_p1]
-    if wl.backward:
-        dout = to_dev(torch, inp["dout"], bf16)
-        bwd_bufs = rom.BackwardBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.device)
+        phases = [("route_dispatch", ph_route), ("proj0", ph_p0), ("proj1", ph_p1)]
+        if wl.backward:
+            dout = to_dev(torch, inp["dout"], bf16)
+            in_bytes += dout.numel() * dout.element_size()
+            bwd_bufs = rom.BackwardBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.device)
 
-        def ph_bwd():
-            rom.block_backward(bufs, dout, w_r, ws["w_conv"], ws["w_gate"], ws["w_out"],
-                               renorm=wl.renorm, bufs=bwd_bufs)
-        phases.append(ph_bwd)
+            def ph_bwd():
+                rom.block_backward(bufs, dout, w_r, ws["w_conv"], ws["w_gate"], ws["w_out"],
+                                   renorm=wl.renorm, bufs=bwd_bufs)
+            phases.append(("backward", ph_bwd))
+        res.update(phases=phases, dominant=(ph_p0, "flop", lambda counts: flops["conv_gate"]),
+                   out=bufs.out, counts=rb.counts,
+                   launches=4 + (2 if wl.k > 1 else 0) + (7 if wl.backward else 0))
+        if wl.backward:
+            res["e2e"] = None  # host copies around one step (below)
+        else:
+            pipe = rom.HostPipeline(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device, De=wl.De)
+            res["e2e"] = (pipe, lambda hx, ho: pipe.block_forward(
+                hx, w_r, bias, ws["w_conv"], ws["w_gate"], ws["w_out"], ho, renorm=wl.renorm))
+    res["in_bytes"] = in_bytes
+    return res
+
+
+def measure(args, wl, world, local_rank, with_e2e):
+    """Times one workload on this rank's GPU; returns the per-rank figures."""
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_projections_b200 import rom
+
+    inp = make_workload_inputs(wl, seed=0)
+    stream = torch.cuda.current_stream()
+    b = build_workload(torch, rom, wl, inp)
+    del inp
+    x, out_t = b["x"], b["out"]
+    phases = [f for _, f in b["phases"]]
+    names = [n for n, _ in b["phases"]]
+    flush_l2 = b["in_bytes"] < 2 * L2_BYTES
+    flush = (torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=x.device)
+             if flush_l2 else None)
+    l2_note = ("flushed before every timed step (256 MiB write)" if flush_l2 else
+               f"not flushed: the step's inputs ({b['in_bytes'] / 1e6:.0f} MB) exceed twice the "
+               f"L2 ({L2_BYTES / 1e6:.0f} MB) and are streamed from HBM every step")
+
+    def do_flush():
+        if flush is not None:
+            flush.zero_()
 
     def step():
         for ph in phases:
             ph()
-        return out_t
-
-    # our kernels per step: router + dispatch (+ the memset of counts, not ours),
-    # the projection(s) and, for top-k > 1, the combines
-    if wl.kind == "inproj":
-        launches_per_step = 3 + (1 if wl.k > 1 else 0)
-    else:
-        launches_per_step = 4 + (2 if wl.k > 1 else 0) + (7 if wl.backward else 0)
 
     for _ in range(args.warmup):
         do_flush()
         step()
     torch.cuda.synchronize()
     if rom.rom_get_status() != 0:
-        raise RuntimeError("device status word reports an error after warm-up")
+        raise RuntimeError(f"{wl.name}: device status word reports an error after warm-up")
 
-    # The step captured once as one CUDA graph (the launch sequence of the
-    # library is static: its kernels read the expert counts on the device),
-    # and each phase once more on its own for the per-phase breakdown.
+    # The step captured once as one CUDA graph (the library's launch sequence
+    # is static: its kernels read the expert counts on the device), and each
+    # phase once more on its own for the per-phase breakdown.
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step):
         step()
@@ -393,100 +469,168 @@ def run_ours(args, rank, world, local_rank):
         graphs.append(g)
     torch.cuda.synchronize()
 
-    def timed_loop(run_phase, n):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)]
+    def timed_loop(run_phase, n, count):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(count + 1)]
                for _ in range(n)]
         for i in range(n):
             do_flush()
             torch.cuda._sleep(200_000)  # GPU-side head start so that the host stays ahead
             evs[i][0].record(stream)
-            for j in range(len(phases)):
+            for j in range(count):
                 run_phase(j)
                 evs[i][j + 1].record(stream)
         torch.cuda.synchronize()
-        return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(phases))]
+        return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(count)]
                          for i in range(n)])
 
-    def timed_steps(n):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
-        for i in range(n):
-            do_flush()
-            torch.cuda._sleep(200_000)  # GPU-side head start so that the host stays ahead
-            evs[i][0].record(stream)
-            g_step.replay()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        return np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(n)])
-
     for _ in range(2):  # graph warm-up
-        timed_loop(lambda j: graphs[j].replay(), 1)
-        timed_steps(1)
+        timed_loop(lambda j: graphs[j].replay(), 1, len(phases))
+        timed_loop(lambda j: g_step.replay(), 1, 1)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    step_ms = timed_steps(args.steps)
-    ph_ms = timed_loop(lambda j: graphs[j].replay(), args.steps)
+    step_ms = timed_loop(lambda j: g_step.replay(), args.steps, 1)[:, 0]
+    ph_ms = timed_loop(lambda j: graphs[j].replay(), args.steps, len(phases))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    eager_ms = timed_loop(lambda j: phases[j](), args.steps)
+    eager_ms = timed_loop(lambda j: phases[j](), args.steps, len(phases))
+    # The dominant kernel alone: one eager launch between two events, the
+    # host ahead of the GPU (no graph-launch latency in its duration).
+    dom_fn, dom_kind, dom_work = b["dominant"]
+    dom_ms = timed_loop(lambda j: dom_fn(), args.steps, 1)[:, 0]
+    counts = b["counts"].cpu().numpy()
     t_total_ms = float(step_ms.sum())
-    part_names = ["route_dispatch", "proj0", "proj1", "backward"][:len(phases)]
-    part_ms = {n: float(ph_ms[:, j].mean()) for j, n in enumerate(part_names)}
-    # The dominant kernel alone (one eager launch between two events, the
-    # host ahead of the GPU): no graph-launch latency in its duration.
-    part_ms_eager = {n: float(eager_ms[:, j].mean()) for j, n in enumerate(part_names)}
 
     # ---------------------------------------------- e2e through host buffers
     # The public host-buffer call: inputs in pinned host memory, result copied
     # back, copies inside the timed region. Forward-only workloads go through
     # rom.HostPipeline (chunks over 3 streams: copies overlap the kernels);
-    # the forward + backward step copies x in and O out around one step.
-    h_x = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-    h_x.copy_(x)
-    h_out = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
-    pipe = None
-    if not wl.backward:
-        pipe = rom.HostPipeline(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device,
-                                De=None if wl.kind == "inproj" else wl.De)
+    # the others copy x in and O out around one step.
+    e2e_total = 0.0
+    if with_e2e:
+        h_x = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        h_x.copy_(x)
+        h_out = torch.empty(out_t.shape, dtype=out_t.dtype, pin_memory=True)
 
-    def e2e_call():
-        if pipe is None:
-            x.copy_(h_x, non_blocking=True)
-            o = step()
-            h_out.copy_(o, non_blocking=True)
-        elif wl.kind == "inproj":
-            pipe.inproj_forward(h_x, w_r, w, h_out, renorm=wl.renorm, bias=bias)
-        else:
-            pipe.block_forward(h_x, w_r, bias, ws["w_conv"], ws["w_gate"], ws["w_out"], h_out,
-                               renorm=wl.renorm)
+        def e2e_call():
+            if b["e2e"] is None:
+                x.copy_(h_x, non_blocking=True)
+                step()
+                h_out.copy_(out_t, non_blocking=True)
+            else:
+                b["e2e"][1](h_x, h_out)
 
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        do_flush()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        e2e_call()
-        s1.record(stream)
-        s1.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(s0.elapsed_time(s1))
-    e2e_total = float(np.sum(e2e_ms))
+        e2e_ms = []
+        for i in range(args.warmup + args.steps):
+            do_flush()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            e2e_call()
+            s1.record(stream)
+            s1.synchronize()
+            if i >= args.warmup:
+                e2e_ms.append(s0.elapsed_time(s1))
+        e2e_total = float(np.sum(e2e_ms))
     del graphs, g_step
 
     t_total_ms, e2e_total = max_over_ranks([t_total_ms, e2e_total], x.device, world)
-    res = dict(wl=wl, step_ms=t_total_ms / args.steps, part_ms=part_ms,
-               part_ms_eager=part_ms_eager,
-               eager_ms=float(eager_ms.sum()) / args.steps,
-               e2e_ms=e2e_total / args.steps, clocks=clk, launches=launches_per_step * args.steps,
-               counts=counts_t.cpu().numpy(), x_bytes=x.numel() * x.element_size(), l2=l2_note,
-               out_bytes=out_t.numel() * out_t.element_size())
-    return res
+    return dict(wl=wl, step_ms=t_total_ms / args.steps,
+                part_ms={n: float(ph_ms[:, j].mean()) for j, n in enumerate(names)},
+                part_ms_eager={n: float(eager_ms[:, j].mean()) for j, n in enumerate(names)},
+                eager_ms=float(eager_ms.sum()) / args.steps, dominant_ms=float(dom_ms.mean()),
+                dominant_kind=dom_kind, dominant_work=float(dom_work(counts)),
+                e2e_ms=e2e_total / args.steps, clocks=clk, launches=b["launches"] * args.steps,
+                counts=counts, x_bytes=x.numel() * x.element_size(), l2=l2_note,
+                out_bytes=out_t.numel() * out_t.element_size())
+
+
+def roofline(res, peaks, src):
+    """Roofline of the dominant kernel: algorithmic work per launch over its
+    eager-launch duration, against the measured peak."""
+    wl = res["wl"]
+    t_k = res["dominant_ms"] / 1e3
+    if res["dominant_kind"] == "byte":
+        ach = res["dominant_work"] / t_k / 1e9
+        return {"bound": "hbm", "kernel": "rom_expert_proj(INPROJ)", "achieved": ach,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                "traffic": profiled_traffic(wl.name), "peak_source": f"{src} hbm_gbs"}
+    ach = res["dominant_work"] / t_k / 1e12
+    pk = peaks["bf16_tflops"]
+    kern = "rom_expert_proj(SLOTS, Conv)" if wl.kind == "variant" else "rom_expert_proj(CONV_GATE)"
+    return {"bound": "tensor", "kernel": kern, "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+            "frac": ach / pk, "traffic": profiled_traffic(wl.name),
+            "peak_source": f"{src} bf16_tflops (burst)"}
+
+
+def workload_config(wl, world):
+    return {"workload": wl.name, "tokens": wl.T, "d_model": wl.Dm,
+            ("d_out" if wl.kind == "inproj" else "d_inner"): wl.De, "experts": wl.E,
+            "top_k": wl.k, "renorm": wl.renorm, "parallelism": f"replicas x{world}",
+            **({"projections": wl.variant} if wl.kind == "variant" else {})}
+
+
+def summary_entry(res, peaks, src, world):
+    """Per-workload figures of the extra workloads of one bench run."""
+    wl = res["wl"]
+    tot = sum(block_flops(wl).values())
+    step_s = res["step_ms"] / 1e3
+    return {"config": workload_config(wl, world), "l2": res["l2"],
+            "step": "forward + backward" if wl.backward else "forward",
+            "ms_per_step": res["step_ms"], "tokens_per_s": job_tokens_per_s(wl.T, world,
+                                                                            res["step_ms"]),
+            "block_tflops": tot / step_s / 1e12, "roofline": roofline(res, peaks, src),
+            "kernels_ms": res["part_ms"], "kernels_ms_eager": res["part_ms_eager"],
+            "clocks": res["clocks"], "gpu_launches": res["launches"],
+            "expert_load": (res["counts"] / max(1, res["counts"].sum())).round(4).tolist()}
+
+
+def reference_arm(args, wl, metric, config, world):
+    """The CPU oracle, as it stands, on the host cores (rank 0 only): each
+    step evaluates a token sample of the workload, the whole workload when
+    its estimated time fits the run's budget (about two minutes)."""
+    inp = make_workload_inputs(wl, seed=0)
+    rng = np.random.default_rng(1)
+    n_steps = args.warmup + args.steps
+    budget_s = 120.0
+    probe = np.sort(rng.choice(wl.T, size=min(wl.T, 4096), replace=False))
+    per_tok = oracle_sample_run(wl, inp, probe) / len(probe)
+    # the whole workload when it fits (a large batch costs less per token
+    # than the probe), else the sample that fills the budget
+    if per_tok * wl.T * n_steps <= 1.5 * budget_s:
+        n = wl.T
+    else:
+        n = int(min(wl.T, max(16, budget_s / n_steps / max(per_tok, 1e-9))))
+    times = []
+    for i in range(n_steps):
+        toks = np.sort(rng.choice(wl.T, size=n, replace=False)) if n < wl.T else None
+        dt = oracle_sample_run(wl, inp, toks)
+        if i >= args.warmup:
+            times.append(dt)
+    t = float(np.sum(times))
+    val = n * args.steps / t
+    sample = (f"all {wl.T} tokens of {wl.name} per step" if n >= wl.T else
+              f"{n} random tokens of the {wl.T} of {wl.name} per step")
+    return {"impl": "reference", "metric": metric, "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "l2": "n/a (host CPU run)",
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample + " (float64 numpy oracle)"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# Workloads timed next to the headline in a single-GPU run: the other
+# configurations of the block, each reported under "workloads".
+EXTRA_WORKLOADS = ["decode_swimba_inproj", "top2_fwd_bwd", "imbalanced_8x4096", "tiny_fp32",
+                   "independent_moe_16k", "rom_gate_out_16k"]
 
 
 def main():
@@ -497,6 +641,8 @@ def main():
     ap.add_argument("--workload", default="prefill_16k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time the headline workload only (no other configurations)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (smaller profiling cases)")
     args = ap.parse_args()
@@ -510,40 +656,14 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = WORKLOADS[args.workload]
-    flops = block_flops(wl)
     metric = (f"tokens/s and TFLOPS (% bf16 peak) for RoM projection block "
               f"{'fwd+bwd' if wl.backward else 'fwd'}, {world} B200")
-    config = {"workload": wl.name, "tokens": wl.T, "d_model": wl.Dm,
-              ("d_out" if wl.kind == "inproj" else "d_inner"): wl.De, "experts": wl.E,
-              "top_k": wl.k, "renorm": wl.renorm, "parallelism": f"replicas x{world}",
-              "l2": "flushed before every timed step (256 MiB write)"}
+    config = workload_config(wl, world)
 
     if args.impl == "reference":
         if rank != 0:
             return
-        inp = make_workload_inputs(wl, seed=0)
-        rng = np.random.default_rng(1)
-        n = 64 if wl.kind == "block" else wl.T
-        times = []
-        for i in range(args.warmup + args.steps):
-            toks = np.sort(rng.choice(wl.T, size=min(n, wl.T), replace=False))
-            dt = oracle_sample_run(wl, inp, toks)
-            if i >= args.warmup:
-                times.append(dt)
-        t = float(np.sum(times))
-        val = len(toks) * args.steps / t
-        config["l2"] = "n/a (host CPU run)"
-        line = {"impl": "reference", "metric": metric, "value": val, "unit": "tokens/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": config,
-                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
-                                 "kind": "oracle",
-                                 "sample": f"{min(n, wl.T)} random tokens of {wl.T} per step"},
-                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        print(json.dumps(reference_arm(args, wl, metric, config, world)), flush=True)
         return
 
     import torch
@@ -552,34 +672,25 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    res = run_ours(args, rank, world, local_rank)
+    torch.cuda.set_device(local_rank)
+    from mixture_experts_projections_b200 import rom
+    rom.load_library()
+    res = measure(args, wl, world, local_rank, with_e2e=True)
+    extra = {}
+    if world == 1 and not args.no_extra and args.tokens is None:
+        for name in EXTRA_WORKLOADS:
+            if name != wl.name:
+                extra[name] = measure(args, WORKLOADS[name], world, local_rank, with_e2e=False)
     if rank == 0:
-        config["l2"] = res["l2"]
         peaks, src = load_peaks()
         step_s = res["step_ms"] / 1e3
-        value = job_tokens_per_s(wl.T, world, res["step_ms"])
-        tot_flops = sum(flops.values())
-        if wl.kind == "inproj":
-            n_hit = int(np.count_nonzero(res["counts"]))
-            t_k = res["part_ms_eager"]["proj0"] / 1e3
-            ach = inproj_bytes(wl, n_hit) / t_k / 1e9
-            roof = {"bound": "hbm", "kernel": "rom_expert_proj(INPROJ)", "achieved": ach,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
-                    "traffic": profiled_traffic(wl.name), "peak_source": f"{src} hbm_gbs"}
-        else:
-            t_k = res["part_ms_eager"]["proj0"] / 1e3
-            ach = flops["conv_gate"] / t_k / 1e12
-            pk = peaks["bf16_tflops"]
-            roof = {"bound": "tensor", "kernel": "rom_expert_proj(CONV_GATE)", "achieved": ach,
-                    "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-                    "traffic": profiled_traffic(wl.name),
-                    "peak_source": f"{src} bf16_tflops (burst)"}
-        line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
-                "csrc_sha256": csrc_digest(),
+        tot_flops = sum(block_flops(wl).values())
+        line = {"metric": metric, "value": job_tokens_per_s(wl.T, world, res["step_ms"]),
+                "unit": "tokens/s", "n_gpus": world, "csrc_sha256": csrc_digest(),
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["step_ms"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
-                "config": config, "roofline": roof,
+                "config": config, "l2": res["l2"], "roofline": roofline(res, peaks, src),
                 "block_tflops": tot_flops / step_s / 1e12,
                 "block_frac_of_bf16_peak": tot_flops / step_s / 1e12 / peaks["bf16_tflops"],
                 "kernels_ms": res["part_ms"], "kernels_ms_eager": res["part_ms_eager"],
@@ -589,10 +700,13 @@ def main():
                           "events on the launching stream (max over ranks); kernels_ms: each "
                           "phase replayed as its own graph; roofline kernel: eager launch "
                           "between two events",
-                "e2e": {"value": job_tokens_per_s(wl.T, world, res["e2e_ms"]), "unit": "tokens/s",
-                        "h2d_bytes_per_step": res["x_bytes"], "d2h_bytes_per_step": res["out_bytes"]},
+                "e2e": {"value": job_tokens_per_s(wl.T, world, res["e2e_ms"]),
+                        "unit": "tokens/s", "h2d_bytes_per_step": res["x_bytes"],
+                        "d2h_bytes_per_step": res["out_bytes"]},
                 "gpu_launches": res["launches"], "clocks": res["clocks"],
                 "expert_load": (res["counts"] / max(1, res["counts"].sum())).round(4).tolist()}
+        if extra:
+            line["workloads"] = {n: summary_entry(r, peaks, src, world) for n, r in extra.items()}
         if not args.no_cpu_baseline and world == 1:
             inp = make_workload_inputs(wl, seed=0)
             line["cpu_baseline"] = cpu_baseline(wl, inp)

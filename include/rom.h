@@ -58,12 +58,14 @@ typedef enum { ROM_F32 = 0, ROM_BF16 = 1 } rom_dtype;
 typedef enum {
   ROM_PROJ_CONV_GATE = 0, /* Conv (input) and Gate projections, shared selection */
   ROM_PROJ_OUT = 1,       /* Out projection, weighted by r */
-  ROM_PROJ_INPROJ = 2     /* Swimba routed in-projection, weighted by r */
+  ROM_PROJ_INPROJ = 2,    /* Swimba routed in-projection, weighted by r */
+  ROM_PROJ_SLOTS = 3      /* one projection to float32 slot rows (Conv or Gate on their own) */
 } rom_proj;
 
 typedef enum {
-  ROM_COMBINE_SUM = 0, /* out[t] = sum_j in[t*k+j]                     */
-  ROM_COMBINE_GATE = 1 /* h_t = (sum_j u_{t,j}) * SiLU(sum_j z_{t,j}) */
+  ROM_COMBINE_SUM = 0,       /* out[t] = sum_j in[t*k+j]                     */
+  ROM_COMBINE_GATE = 1,      /* h_t = (sum_j u_{t,j}) * SiLU(sum_j z_{t,j}) */
+  ROM_COMBINE_GATE_DENSE = 2 /* h_t = u_t * SiLU(sum_j z_{t,j}), u_t dense  */
 } rom_combine_mode;
 
 /* Human-readable name of a rom_status value (static string). */
@@ -150,7 +152,15 @@ int rom_dispatch(const void* x, int dtype, int64_t T, int Dm, int E, int k,
  *     k  > 1: out = float32 [R][N] in slot order (rom_combine(ROM_COMBINE_SUM)).
  *  ROM_PROJ_INPROJ (Swimba page, Extended abstract): w0 = W [E][N][K], the
  *     X|B|C in-projection; same weighting and outputs as ROM_PROJ_OUT.
- *
+ *  ROM_PROJ_SLOTS: w0 = W [E][N][K], w1 = NULL: one projection on its own,
+ *     out = float32 [R][N] in SLOT order for any k, row s = the slot's sorted
+ *     row times W_e^T, scaled by topk_w[s] when topk_w is not NULL and
+ *     unscaled when it is NULL. With a router of its own this is the Conv or
+ *     the Gate projection of independently routed MoE-Mamba, a conventional
+ *     MoE layer per projection (RoM page, Knowl 4); with offsets == NULL,
+ *     sorted_slot == NULL and E == 1 it is a dense projection of the R rows
+ *     in row order (RoM page, Knowl 3: "RoM (Gate, Out)" keeps Conv dense).
+ *     rom_combine(ROM_COMBINE_GATE or ROM_COMBINE_GATE_DENSE) then forms h.
  *  bf16 (tensor cores, tcgen05 + TMA): requires K % 8 == 0, N % 128 == 0 and
  *  16-byte aligned a_sorted, w0, w1 and out. float32 (CUDA-core FMA): any K, N.
  */
@@ -166,7 +176,16 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
  *                    h_t = (sum_j u[t*k+j]) * SiLU(sum_j z[t*k+j]) (RoM page,
  *                    Knowl 1: SiLU after the sum over the selected experts);
  *                    out = h_sorted [T*k][N] dtype with h_t written to row
- *                    slot_pos[t*k+j] for every j.
+ *                    slot_pos[t*k+j] for every j. u and z may come from
+ *                    different routings (ROM_PROJ_SLOTS, each in its own slot
+ *                    order); slot_pos is then the Out projection's. With
+ *                    slot_pos == NULL, h_t is written once, to row t (a dense
+ *                    Out projection reads h in token order).
+ *  ROM_COMBINE_GATE_DENSE: in = float32 [T + T*k][N]: rows 0..T-1 hold the
+ *                    dense Conv projection u_t (token order), rows T.. the
+ *                    Gate partials z in slot order; h_t = u_t * SiLU(sum_j
+ *                    z[t*k+j]) written like ROM_COMBINE_GATE (RoM page,
+ *                    Knowl 3, "RoM (Gate, Out)": Conv is not expertized).
  *  Requires N % 4 == 0.
  */
 int rom_combine(int mode, int dtype, const void* in, int64_t T, int k, int N,

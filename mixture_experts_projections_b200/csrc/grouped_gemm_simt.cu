@@ -33,7 +33,9 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ float sB1[kGate ? TK : 1][TN + 4];
   const int tid = threadIdx.x;
   const int n_tiles_n = (N + TN - 1) / TN;
-  for (int i = tid; i <= E; i += kThreads) s_off[i] = offsets[i];
+  // No offsets: one expert owns all R rows (a dense projection).
+  for (int i = tid; i <= E; i += kThreads)
+    s_off[i] = offsets ? offsets[i] : (i == 0 ? 0 : static_cast<int>(R));
   __syncthreads();
   if (tid == 0) {
     int run = 0;
@@ -97,8 +99,10 @@ __global__ void __launch_bounds__(kThreads)
     const int r = tr * 4 + i;
     if (r >= rows_here) continue;
     const int64_t prow = row_base + r;
-    const int64_t slot = (MODE == kEpiGateH) ? 0 : sorted_slot[prow];
-    const float rw = (MODE == kEpiScaleToken || MODE == kEpiScaleSlots) ? topk_w[slot] : 0.f;
+    const int64_t slot = (MODE == kEpiGateH) ? 0 : (sorted_slot ? sorted_slot[prow] : prow);
+    const float rw = (MODE == kEpiScaleToken || MODE == kEpiScaleSlots)
+                         ? (topk_w ? topk_w[slot] : 1.f)  // no weights passed: r = 1
+                         : 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n_base + tc * 4 + j;

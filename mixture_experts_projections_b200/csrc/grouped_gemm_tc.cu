@@ -71,6 +71,16 @@ __device__ __forceinline__ float silu_gate(float u, float z) {
   return u * __fdividef(z, 1.0f + __expf(-z));
 }
 
+// Slot of sorted row `prow` (row order itself for a dense projection, which
+// passes no sorted_slot) and the expert row bounds (one expert owning all R
+// rows when no offsets are passed).
+__device__ __forceinline__ int64_t slot_of(const Params& p, int64_t prow) {
+  return p.sorted_slot ? static_cast<int64_t>(p.sorted_slot[prow]) : prow;
+}
+__device__ __forceinline__ int offset_of(const Params& p, int i) {
+  return p.offsets ? p.offsets[i] : (i == 0 ? 0 : static_cast<int>(p.R));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -112,7 +122,7 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
     }
   } else if (MODE == kEpiGateSlots) {
     float* out = static_cast<float*>(p.out);
-    const int64_t slot = valid ? p.sorted_slot[prow] : 0;
+    const int64_t slot = valid ? slot_of(p, prow) : 0;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t u[32], z[32];
@@ -128,8 +138,9 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
       store_rows_f32(stg, f, valid ? out + (p.R + slot) * p.N + n0 + c * 32 : nullptr);
     }
   } else {
-    const int64_t slot = valid ? p.sorted_slot[prow] : 0;
-    const float r = valid ? p.topk_w[slot] : 0.f;
+    const int64_t slot = valid ? slot_of(p, prow) : 0;
+    // no routing weights passed: r = 1
+    const float r = valid ? (p.topk_w ? p.topk_w[slot] : 1.f) : 0.f;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       if (n0 + c * 32 >= p.N) break;  // partial last tile (N % 256 == 128)
@@ -233,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
 
-  for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = p.offsets[i];
+  for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = offset_of(p, i);
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = 0;
@@ -449,8 +460,8 @@ __device__ __forceinline__ void swap_token(const Params& p, int64_t prow, bool v
   orow = 0;
   r = 0.f;
   if (valid) {
-    const int slot = p.sorted_slot[prow];
-    r = p.topk_w[slot];
+    const int slot = static_cast<int>(slot_of(p, prow));
+    r = p.topk_w ? p.topk_w[slot] : 1.f;  // no routing weights: r = 1
     orow = MODE == kEpiScaleToken ? slot / p.k : slot;
   }
 }
@@ -468,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int E = p.E;
   const int n_wt = p.N / SW_BM;  // weight-row tiles per expert
 
-  for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = p.offsets[i];
+  for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = offset_of(p, i);
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = 0;

@@ -161,7 +161,8 @@ int rom_dispatch(const void* x, int dtype, int64_t T, int Dm, int E, int k,
 int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K, const void* w0,
                     const void* w1, int N, int E, int k, const int32_t* offsets,
                     const int32_t* sorted_slot, const float* topk_w, void* out, void* stream) {
-  if (proj != ROM_PROJ_CONV_GATE && proj != ROM_PROJ_OUT && proj != ROM_PROJ_INPROJ)
+  if (proj != ROM_PROJ_CONV_GATE && proj != ROM_PROJ_OUT && proj != ROM_PROJ_INPROJ &&
+      proj != ROM_PROJ_SLOTS)
     return ROM_ERR_INVALID_ARG;
   if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
   if (R < 0 || K <= 0 || N <= 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E ||
@@ -169,12 +170,20 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
     return ROM_ERR_INVALID_ARG;
   if (R >= (int64_t(1) << 31)) return ROM_ERR_UNSUPPORTED;
   const bool gate = proj == ROM_PROJ_CONV_GATE;
-  if (!offsets || !w0 || !out || (gate && !w1)) return ROM_ERR_INVALID_ARG;
-  if (!gate && (!sorted_slot || !topk_w)) return ROM_ERR_INVALID_ARG;
+  const bool slots = proj == ROM_PROJ_SLOTS;
+  // A dense projection (ROM_PROJ_SLOTS only): no routing arrays, one matrix.
+  const bool dense = slots && !offsets && !sorted_slot;
+  if (dense && E != 1) return ROM_ERR_INVALID_ARG;
+  if ((!offsets && !dense) || !w0 || !out || (gate && !w1)) return ROM_ERR_INVALID_ARG;
+  if (!gate && !dense && (!sorted_slot || (!slots && !topk_w))) return ROM_ERR_INVALID_ARG;
   if (gate && k > 1 && !sorted_slot) return ROM_ERR_INVALID_ARG;
   if (R > 0 && !a_sorted) return ROM_ERR_INVALID_ARG;
-  const int mode = gate ? (k == 1 ? rom::kEpiGateH : rom::kEpiGateSlots)
-                        : (k == 1 ? rom::kEpiScaleToken : rom::kEpiScaleSlots);
+  if (slots) w1 = nullptr;
+  // ROM_PROJ_SLOTS is the slot-order float32 epilogue; r = 1 when topk_w is
+  // NULL, and row p is slot p when sorted_slot is NULL.
+  const int mode = gate    ? (k == 1 ? rom::kEpiGateH : rom::kEpiGateSlots)
+                   : slots ? rom::kEpiScaleSlots
+                           : (k == 1 ? rom::kEpiScaleToken : rom::kEpiScaleSlots);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == ROM_F32) {
     return rom::to_status(rom::launch_simt_grouped_gemm(
@@ -193,12 +202,13 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
 
 int rom_combine(int mode, int dtype, const void* in, int64_t T, int k, int N,
                 const int32_t* slot_pos, void* out, void* stream) {
-  if (mode != ROM_COMBINE_SUM && mode != ROM_COMBINE_GATE) return ROM_ERR_INVALID_ARG;
+  if (mode != ROM_COMBINE_SUM && mode != ROM_COMBINE_GATE && mode != ROM_COMBINE_GATE_DENSE)
+    return ROM_ERR_INVALID_ARG;
   if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
   if (T < 0 || k < 1 || k > rom::kMaxTopK || N <= 0) return ROM_ERR_INVALID_ARG;
   if (N % 4 != 0) return ROM_ERR_UNSUPPORTED;
   if (T == 0) return ROM_OK;
-  if (!in || !out || (mode == ROM_COMBINE_GATE && !slot_pos)) return ROM_ERR_INVALID_ARG;
+  if (!in || !out) return ROM_ERR_INVALID_ARG;
   if (!aligned16(in) || !aligned16(out)) return ROM_ERR_UNSUPPORTED;
   return rom::to_status(rom::launch_combine(mode, dtype == ROM_BF16,
                                             static_cast<const float*>(in), T, k, N, slot_pos,

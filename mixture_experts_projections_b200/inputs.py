@@ -45,6 +45,10 @@ class Workload:
     backward: bool = False
     # Swimba stream widths (X, B, C) when kind == "inproj"
     streams: tuple = field(default_factory=tuple)
+    # kind == "variant": "independent" (a router per projection, each
+    # projection a conventional MoE layer) or "gate_out" (dense Conv, one
+    # router shared by Gate and Out)
+    variant: str = ""
 
 
 # Router-bias constants of the load-imbalanced workload. They were found by
@@ -66,11 +70,17 @@ WORKLOADS = {
         dtype="bf16", streams=(8192, 8 * 128, 8 * 128)),
     "top2_fwd_bwd": Workload("top2_fwd_bwd", "block", T=32768, Dm=2560, De=5120, E=16, k=2,
                              dtype="bf16", renorm=True, backward=True),
+    # The prefill shapes with the comparison configurations of the pages:
+    # independent routing of Conv, Gate and Out, and RoM (Gate, Out).
+    "independent_moe_16k": Workload("independent_moe_16k", "variant", T=16384, Dm=2048, De=4096,
+                                    E=8, k=1, dtype="bf16", variant="independent"),
+    "rom_gate_out_16k": Workload("rom_gate_out_16k", "variant", T=16384, Dm=2048, De=4096, E=8,
+                                 k=1, dtype="bf16", variant="gate_out"),
 }
 
 # The order the workloads are listed in (the small fp32 case first).
 WORKLOAD_ORDER = ["tiny_fp32", "prefill_16k", "imbalanced_8x4096", "decode_swimba_inproj",
-                  "top2_fwd_bwd"]
+                  "top2_fwd_bwd", "independent_moe_16k", "rom_gate_out_16k"]
 
 
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
@@ -109,11 +119,14 @@ def bias_vector(E: int, bias_items) -> np.ndarray | None:
 
 
 def make_block_inputs(T, Dm, De, E, *, seed=0, dtype="bf16", router_std=0.02, bias=None,
-                      with_dout=False, zero_router=False):
+                      with_dout=False, zero_router=False, extra_routers=False):
     """Inputs of the Conv/Gate/Out block in the paper's notation.
 
     Returns a dict with x [T,Dm], w_r [Dm,E] (float32), bias [E] or None,
     w_conv and w_gate [E,Dm,De], w_out [E,De,Dm] and, if asked, dout [T,Dm].
+    With ``extra_routers`` two more router weights w_r_gate and w_r_out
+    [Dm,E] are drawn last (after everything above), so the other arrays are
+    those of the same seed without them.
     """
     bf = dtype == "bf16"
     rng = np.random.default_rng(seed)
@@ -128,6 +141,9 @@ def make_block_inputs(T, Dm, De, E, *, seed=0, dtype="bf16", router_std=0.02, bi
                w_conv=w_conv, w_gate=w_gate, w_out=w_out)
     if with_dout:
         out["dout"] = _draw(rng, (T, Dm), 1.0, bf)
+    if extra_routers:
+        out["w_r_gate"] = _draw(rng, (Dm, E), router_std, False)
+        out["w_r_out"] = _draw(rng, (Dm, E), router_std, False)
     return out
 
 
@@ -149,4 +165,5 @@ def make_workload_inputs(wl: Workload, seed=0):
                                   router_std=wl.router_std)
     return make_block_inputs(T, wl.Dm, wl.De, wl.E, seed=seed, dtype=wl.dtype,
                              router_std=wl.router_std, bias=bias_vector(wl.E, wl.bias),
-                             with_dout=wl.backward)
+                             with_dout=wl.backward, extra_routers=wl.variant == "independent")
+

@@ -21,8 +21,8 @@ LIB_PATH = os.path.join(_HERE, "librom.so")
 ROM_OK, ROM_ERR_INVALID_ARG, ROM_ERR_UNSUPPORTED, ROM_ERR_WORKSPACE, ROM_ERR_CUDA, \
     ROM_ERR_TIMEOUT, ROM_ERR_ROUTING = range(7)
 ROM_F32, ROM_BF16 = 0, 1
-ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ = 0, 1, 2
-ROM_COMBINE_SUM, ROM_COMBINE_GATE = 0, 1
+ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ, ROM_PROJ_SLOTS = 0, 1, 2, 3
+ROM_COMBINE_SUM, ROM_COMBINE_GATE, ROM_COMBINE_GATE_DENSE = 0, 1, 2
 
 # Every exported symbol of include/rom.h with its ctypes signature.
 _P = ctypes.c_void_p
@@ -129,6 +129,8 @@ def rom_expert_proj(proj, a_sorted, w0, w1, E, k, offsets, sorted_slot, topk_w, 
                     stream=None):
     R, K = a_sorted.shape
     N = w0.shape[1]
+    if not out.is_contiguous():
+        raise RomError("out must be contiguous")
     _check(load_library().rom_expert_proj(
         proj, _dtype_code(a_sorted), _ptr(a_sorted), R, K, _ptr(w0), _ptr(w1), N, E, k,
         _ptr(offsets), _ptr(sorted_slot), _ptr(topk_w), _ptr(out), _stream(stream)),
@@ -262,6 +264,110 @@ def inproj_forward(x, w_r, w, k=1, renorm=False, bias=None, bufs=None, out=None,
                         rb.sorted_slot, rb.topk_w, slots, stream)
         rom_combine(ROM_COMBINE_SUM, _dtype_code(x), slots, T, k, N, None, out, stream)
     return out, rb
+
+
+# ------------------------------------------------------------------ projection variants
+
+PROJECTIONS = ("conv", "gate", "out")
+
+
+class VariantBuffers:
+    """Buffers of one forward of a projection variant (allocated by torch)."""
+
+    def __init__(self, T, Dm, De, k, dtype, device):
+        R = T * k
+        self.routings = {}  # id(router weight) -> RoutingBuffers, made on first use
+        self.uz = torch.empty((2 * R, De), dtype=torch.float32, device=device)
+        self.h = torch.empty((R, De), dtype=dtype, device=device)
+        self.o_slots = torch.empty((R, Dm), dtype=torch.float32, device=device)
+        self.out = torch.empty((T, Dm), dtype=dtype, device=device)
+
+
+def variant_block_forward(x, routers, weighted, w_conv, w_gate, w_out, k, renorm=False,
+                          bias=None, bufs=None, stream=None,
+                          phases=("route", "project", "output")):
+    """Projection block with each of Conv, Gate and Out dense or routed.
+
+    routers: {"conv", "gate", "out"} -> router weight [Dm, E] float32, or None
+    for a dense projection (its weight stack then holds one matrix). The same
+    tensor passed for several projections is one shared routing decision
+    (routed and dispatched once). weighted: the same keys -> True when that
+    projection's expert outputs are scaled by its routing weights (Out must
+    be weighted when routed). Weights in the library layout [E, N, K].
+
+    Independently routed MoE-Mamba (RoM page, Knowl 4) passes three routers
+    and weights all three; RoM (Gate, Out) (Knowl 3) passes None for Conv and
+    one router for Gate and Out. Returns the VariantBuffers (O in ``.out``).
+
+    ``phases`` runs a subset of the three steps, in order, on ``bufs`` from
+    an earlier call: "route" (route and dispatch every distinct router),
+    "project" (the Conv and Gate projections to float32 rows) and "output"
+    (the gate combine and the Out projection).
+    """
+    T, Dm = x.shape
+    De = w_conv.shape[1]
+    R = T * k
+    if routers["out"] is not None and not weighted["out"]:
+        raise RomError("a routed Out projection is weighted by its routing weights")
+    if routers["gate"] is None and routers["conv"] is not None and k > 1:
+        raise RomError("a dense Gate projection with routed Conv needs k == 1")
+    if bufs is None:
+        bufs = VariantBuffers(T, Dm, De, k, x.dtype, x.device)
+    wts = {"conv": w_conv, "gate": w_gate, "out": w_out}
+    rbs = {}
+    for n in PROJECTIONS:
+        w_r = routers[n]
+        if w_r is None:
+            rbs[n] = None
+            continue
+        key = id(w_r)
+        if key not in bufs.routings:
+            bufs.routings[key] = RoutingBuffers(T, Dm, w_r.shape[1], k, x.dtype, x.device)
+        rb = bufs.routings[key]
+        # route each distinct router once
+        if "route" in phases and not any(rbs.get(m) is rb for m in rbs):
+            route_and_dispatch(x, w_r, bias, w_r.shape[1], k, renorm, rb, stream)
+        rbs[n] = rb
+
+    def project_slots(name, dst):
+        rb = rbs[name]
+        if rb is None:  # dense: one matrix over the tokens in order
+            rom_expert_proj(ROM_PROJ_SLOTS, x, wts[name], None, 1, 1, None, None, None, dst,
+                            stream)
+        else:
+            rom_expert_proj(ROM_PROJ_SLOTS, rb.x_sorted[:R], wts[name], None, wts[name].shape[0],
+                            k, rb.offsets, rb.sorted_slot, rb.topk_w if weighted[name] else None,
+                            dst, stream)
+
+    conv_rows = T if rbs["conv"] is None else R
+    gate_rows = T if rbs["gate"] is None else R
+    if "project" in phases:
+        project_slots("conv", bufs.uz[:conv_rows])
+        project_slots("gate", bufs.uz[conv_rows:conv_rows + gate_rows])
+    if "output" not in phases:
+        return bufs
+    rb_o = rbs["out"]
+    dt = _dtype_code(x)
+    h_pos = None if rb_o is None else rb_o.slot_pos
+    h_rows = T if rb_o is None else R
+    if rbs["conv"] is None and k > 1:
+        rom_combine(ROM_COMBINE_GATE_DENSE, dt, bufs.uz[:T + R], T, k, De, h_pos, bufs.h, stream)
+    else:
+        # both Conv and Gate routed (u and z per slot), or k == 1 (a dense one
+        # has one row per token, which is also its slot)
+        rom_combine(ROM_COMBINE_GATE, dt, bufs.uz[:2 * R], T, k, De, h_pos, bufs.h, stream)
+    if rb_o is None:
+        rom_expert_proj(ROM_PROJ_SLOTS, bufs.h[:T], w_out, None, 1, 1, None, None, None,
+                        bufs.o_slots[:T], stream)
+        rom_combine(ROM_COMBINE_SUM, dt, bufs.o_slots[:T], T, 1, Dm, None, bufs.out, stream)
+    elif k == 1:
+        rom_expert_proj(ROM_PROJ_OUT, bufs.h[:h_rows], w_out, None, w_out.shape[0], k,
+                        rb_o.offsets, rb_o.sorted_slot, rb_o.topk_w, bufs.out, stream)
+    else:
+        rom_expert_proj(ROM_PROJ_OUT, bufs.h[:h_rows], w_out, None, w_out.shape[0], k,
+                        rb_o.offsets, rb_o.sorted_slot, rb_o.topk_w, bufs.o_slots, stream)
+        rom_combine(ROM_COMBINE_SUM, dt, bufs.o_slots, T, k, Dm, None, bufs.out, stream)
+    return bufs
 
 
 # ------------------------------------------------------------------ backward

@@ -77,16 +77,23 @@ def errors(got: np.ndarray, ref: np.ndarray):
     return max_abs, rel
 
 
+# Every output comparison of this run: (what, max abs, its bound, rel Frobenius,
+# its bound), printed by conftest.py at the end of the run.
+PARITY_LOG = []
+
+
 def assert_close(got, ref, dtype: str, what: str, magnitude_scaled_abs: bool = False):
     max_abs, rel = errors(got, ref)
     if dtype == "bf16":
         bound = BF16_MAX_ABS
         if magnitude_scaled_abs and np.size(ref):
             bound = max(BF16_MAX_ABS, 2.0 ** -7 * float(np.max(np.abs(ref))))
+        PARITY_LOG.append((what, max_abs, bound, rel, BF16_REL_FRO))
         assert max_abs <= bound and rel <= BF16_REL_FRO, \
             f"{what}: max abs {max_abs:.3e} (<= {bound:.3e}), rel Frobenius {rel:.3e} (<= {BF16_REL_FRO})"
     else:
         scale = max(1.0, float(np.max(np.abs(ref)))) if np.size(ref) else 1.0
+        PARITY_LOG.append((what, max_abs, F32_REL * scale, rel, F32_REL))
         assert rel <= F32_REL and max_abs <= F32_REL * scale, \
             f"{what}: max abs {max_abs:.3e}, rel Frobenius {rel:.3e} (<= {F32_REL})"
     return max_abs, rel

@@ -71,7 +71,11 @@ def test_route_rejects_bad_arguments(lib, kw, code):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(proj=3), 1), (dict(dtype=2), 1), (dict(K=0), 1), (dict(N=0), 1), (dict(k=2, R=7), 1),
+    (dict(proj=4), 1), (dict(dtype=2), 1), (dict(K=0), 1), (dict(N=0), 1), (dict(k=2, R=7), 1),
+    # ROM_PROJ_SLOTS: a dense projection (no routing arrays) needs E == 1; a
+    # routed one needs both offsets and sorted_slot
+    (dict(proj=3, offsets=None, sorted_slot=None), 1), (dict(proj=3, offsets=None), 1),
+    (dict(proj=3, sorted_slot=None), 1),
     (dict(w1=None), 1), (dict(offsets=None), 1), (dict(N=200), 2), (dict(K=12), 2),
     (dict(out=ctypes.c_void_p((1 << 20) + 8)), 2),
     (dict(proj=1, N=320), 2),
@@ -85,8 +89,8 @@ def test_expert_proj_rejects_bad_arguments(lib, kw, code):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(mode=2), 1), (dict(dtype=3), 1), (dict(k=0), 1), (dict(k=9), 1), (dict(N=6), 2),
-    (dict(mode=1, slot_pos=None), 1), (dict(inp=None), 1),
+    (dict(mode=3), 1), (dict(dtype=3), 1), (dict(k=0), 1), (dict(k=9), 1), (dict(N=6), 2),
+    (dict(inp=None), 1), (dict(mode=2, out=None), 1),
 ])
 def test_combine_rejects_bad_arguments(lib, kw, code):
     a = dict(mode=0, dtype=1, inp=FAKE, T=10, k=2, N=64, slot_pos=FAKE, out=FAKE, stream=None)

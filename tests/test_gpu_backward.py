@@ -83,28 +83,38 @@ def test_backward_is_deterministic():
 
 
 def test_top2_workload_full_size_backward():
-    """Full top-2 workload: dX and dlogits on sampled tokens (each token's
-    gradient depends on that token only); dW of one expert exactly, from the
-    oracle run on every token routed to it."""
+    """Full top-2 workload, whole gradients: every token's dX and dlogits,
+    every expert's dW_conv, dW_gate and dW_out, and the whole forward O. The
+    oracle runs on batches of tokens (a token's forward and its dX, dlogits
+    depend on that token only; the weight gradients are sums over tokens, so
+    the batches' sums add up to them)."""
     wl = WORKLOADS["top2_fwd_bwd"]
     inp = make_workload_inputs(wl)
     fwd, bwd = run_fwd_bwd(inp, wl.k, wl.renorm)
-    idx = fwd.routing.topk_idx.cpu().numpy()
-    rng = np.random.default_rng(0)
-    toks = np.sort(rng.choice(wl.T, size=32, replace=False))
-    ref = orc.block_backward(inp["x"][toks], inp["w_r"], inp["w_conv"], inp["w_gate"],
-                             inp["w_out"], inp["dout"][toks], k=wl.k, renorm=wl.renorm)
-    assert_close(to_np(bwd.dx[torch.from_numpy(toks).cuda()]), ref["dX"], "bf16", "dX (sampled)",
+    E, Dm, De = wl.E, wl.Dm, wl.De
+    dX = np.empty((wl.T, Dm))
+    dl = np.empty((wl.T, E))
+    O = np.empty((wl.T, Dm))
+    dW = {n: np.zeros((E, a, b)) for n, a, b in (("dW_in", Dm, De), ("dW_g", Dm, De),
+                                                   ("dW_out", De, Dm))}
+    step = 4096
+    for a in range(0, wl.T, step):
+        b = min(wl.T, a + step)
+        ref = orc.block_backward(inp["x"][a:b], inp["w_r"], inp["w_conv"], inp["w_gate"],
+                                 inp["w_out"], inp["dout"][a:b], k=wl.k, renorm=wl.renorm)
+        assert np.array_equal(fwd.routing.topk_idx[a:b].cpu().numpy(),
+                              ref["forward"]["topk_idx"])
+        dX[a:b], dl[a:b], O[a:b] = ref["dX"], ref["dlogits"], ref["forward"]["O"]
+        for n in dW:
+            dW[n] += ref[n]
+    assert_close(to_np(fwd.out), O, "bf16", "top2 O (whole)")
+    assert_close(to_np(bwd.dx), dX, "bf16", "top2 dX (whole)", magnitude_scaled_abs=True)
+    assert_close(to_np(bwd.dlogits), dl, "bf16", "top2 dlogits (whole)",
                  magnitude_scaled_abs=True)
-    assert_close(to_np(bwd.dlogits[torch.from_numpy(toks).cuda()]), ref["dlogits"], "bf16",
-                 "dlogits (sampled)", magnitude_scaled_abs=True)
-    e = 5
-    mine = np.nonzero(np.any(idx == e, axis=1))[0]
-    ref_e = orc.block_backward(inp["x"][mine], inp["w_r"], inp["w_conv"], inp["w_gate"],
-                               inp["w_out"], inp["dout"][mine], k=wl.k, renorm=wl.renorm)
-    assert_close(to_np(bwd.dw_conv[e]), ref_e["dW_in"][e].T, "bf16", "dW_conv[e]",
-                 magnitude_scaled_abs=True)
-    assert_close(to_np(bwd.dw_gate[e]), ref_e["dW_g"][e].T, "bf16", "dW_gate[e]",
-                 magnitude_scaled_abs=True)
-    assert_close(to_np(bwd.dw_out[e]), ref_e["dW_out"][e].T, "bf16", "dW_out[e]",
-                 magnitude_scaled_abs=True)
+    for e in range(E):
+        assert_close(to_np(bwd.dw_conv[e]), dW["dW_in"][e].T, "bf16", f"top2 dW_conv[{e}]",
+                     magnitude_scaled_abs=True)
+        assert_close(to_np(bwd.dw_gate[e]), dW["dW_g"][e].T, "bf16", f"top2 dW_gate[{e}]",
+                     magnitude_scaled_abs=True)
+        assert_close(to_np(bwd.dw_out[e]), dW["dW_out"][e].T, "bf16", f"top2 dW_out[{e}]",
+                     magnitude_scaled_abs=True)

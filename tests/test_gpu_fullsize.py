@@ -1,7 +1,7 @@
 """Parity at the full workload sizes, in the launch configuration the bench
 times: routing and dispatch are compared with the oracle on every token
-(bit-exact); the block outputs on a seeded sample of tokens that the oracle
-evaluates one by one (plus the whole output of the small decode workload)."""
+(bit-exact), and the whole block output element by element (the top-2
+workload's whole output and gradients are in test_gpu_backward.py)."""
 import numpy as np
 import pytest
 import torch
@@ -14,16 +14,7 @@ from parity_util import (assert_close, assert_routing_matches, block_to_dev, to_
 
 pytestmark = pytest.mark.gpu
 
-N_SAMPLE = 48
-
-
-def _sample(T, seed=0):
-    rng = np.random.default_rng(seed)
-    s = rng.choice(T, size=min(N_SAMPLE, T), replace=False)
-    return np.sort(np.concatenate([s, [0, T - 1]]))
-
-
-@pytest.mark.parametrize("name", ["prefill_16k", "imbalanced_8x4096", "top2_fwd_bwd"])
+@pytest.mark.parametrize("name", ["prefill_16k", "imbalanced_8x4096"])
 def test_block_workload_full_size(name):
     wl = WORKLOADS[name]
     inp = make_workload_inputs(wl)
@@ -45,11 +36,9 @@ def test_block_workload_full_size(name):
     if name == "imbalanced_8x4096":
         load = np.bincount(idx[:, 0], minlength=wl.E) / wl.T
         assert 0.38 < load[0] < 0.42 and load[7] < 0.02
-    toks = _sample(wl.T)
     ref = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
-                            k=wl.k, bias=inp["bias"], renorm=wl.renorm, tokens=toks)
-    got = to_np(out.out[torch.from_numpy(toks).cuda()])
-    assert_close(got, ref["O"], wl.dtype, f"{name} O (sampled)")
+                            k=wl.k, bias=inp["bias"], renorm=wl.renorm)
+    assert_close(to_np(out.out), ref["O"], wl.dtype, f"{name} O (whole)")
 
 
 def test_decode_swimba_inproj_full():
@@ -61,4 +50,4 @@ def test_decode_swimba_inproj_full():
     torch.cuda.synchronize()
     assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
                            ref, x=inp["x"], w_r=inp["w_r"])
-    assert_close(to_np(out), ref["S"], "bf16", "S")
+    assert_close(to_np(out), ref["S"], "bf16", "decode S (whole)")
