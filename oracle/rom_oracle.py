@@ -146,15 +146,20 @@ def dispatch(topk_idx, E):
                 sorted_slot=sorted_slot.astype(np.int32), slot_pos=slot_pos.astype(np.int32))
 
 
-def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=None):
+def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=None,
+                  core=None, seq_len=None):
     """RoM projection block forward (RoM page, Knowl 1).
 
     H_t = sum_i 1[i in S_t] x_t W_in,i ;  G_t = SiLU(sum_i 1[i in S_t] x_t W_g,i)
-    Y_t = H_t (identity stand-in for the unchanged conv + SSM core)
+    Y_t = H_t (identity stand-in for the unchanged conv + SSM core), or
+    Y = ssm_core(H) when ``core`` holds the core's parameters
     O_t = sum_i r_{t,i} (Y_t (.) G_t) W_out,i
 
-    ``tokens`` (optional index array) evaluates only those tokens; every
-    token is independent of the others in this block.
+    ``tokens`` (optional index array) evaluates only those tokens; without
+    the core every token is independent of the others in this block (with
+    the core, ``tokens`` is refused: a token depends on its sequence's past).
+    ``seq_len``: the tokens are consecutive sequences of that length (for
+    the core).
     Returns a dict with O [T,Dm], H, Gpre (the sum before SiLU), G, YG [T,De]
     and the router outputs.
     """
@@ -175,7 +180,12 @@ def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=N
             H[sel] += x[sel] @ _f64(w_in[i])
             Gpre[sel] += x[sel] @ _f64(w_g[i])
     G = silu(Gpre)
-    Y = H
+    if core is None:
+        Y = H
+    else:
+        if tokens is not None:
+            raise ValueError("the core mixes tokens over time: evaluate whole sequences")
+        Y = ssm_core(H, core, seq_len)["Y"]
     YG = Y * G
     O = np.zeros((T, Dm))
     for i in range(E):
@@ -184,7 +194,7 @@ def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=N
             if sel.size == 0:
                 continue
             O[sel] += r[sel, j][:, None] * (YG[sel] @ _f64(w_out[i]))
-    return dict(O=O, H=H, Gpre=Gpre, G=G, YG=YG, **rt)
+    return dict(O=O, H=H, Gpre=Gpre, G=G, Y=Y, YG=YG, **rt)
 
 
 def inproj_forward(x, w_r, w, k=1, bias=None, renorm=False, tokens=None):
@@ -339,3 +349,86 @@ def variant_block_forward(x, w_in, w_g, w_out, k, routers, weighted, bias=None, 
     YG = H * G
     O = project("out", YG, w_out)
     return dict(O=O, H=H, Gpre=Gpre, G=G, YG=YG, routing=rts)
+
+
+def softplus(v):
+    """softplus(v) = ln(1 + e^v), written to avoid overflow."""
+    v = np.asarray(v, dtype=np.float64)
+    return np.maximum(v, 0.0) + np.log1p(np.exp(-np.abs(v)))
+
+
+def causal_conv1d(h, w, b):
+    """Short causal depthwise convolution over time (one sequence).
+
+    h [L, D]; w [D, K] (tap K-1 multiplies the current step, tap K-1-j the
+    step j back); b [D]. out_t = b + sum_j w[:, K-1-j] * h_{t-j}, with
+    h_{t-j} = 0 before the start of the sequence.
+    """
+    h = _f64(h)
+    w = _f64(w)
+    L, D = h.shape
+    K = w.shape[1]
+    out = np.zeros((L, D)) + _f64(b)[None, :]
+    for j in range(K):
+        out[j:] += w[:, K - 1 - j][None, :] * h[:L - j]
+    return out
+
+
+def selective_scan(u, delta, A, B, C, D):
+    """Selective state-space recurrence of one sequence (Mamba, Gu and Dao
+    2023, Section 3: zero-order hold for A, Euler step for the input).
+
+    u, delta [L, D]; A [D, N]; B, C [L, N]; D [D]. With the state
+    h_t [D, N] (h_0 = 0 before the first step):
+      h_t = exp(delta_t A) (.) h_{t-1} + (delta_t u_t) B_t
+      y_t = h_t C_t + D (.) u_t
+    Returns y [L, D].
+    """
+    u, delta, A, B, C, D = (_f64(a) for a in (u, delta, A, B, C, D))
+    L, Dd = u.shape
+    h = np.zeros(A.shape)
+    y = np.empty((L, Dd))
+    for t in range(L):
+        h = np.exp(delta[t][:, None] * A) * h + (delta[t] * u[t])[:, None] * B[t][None, :]
+        y[t] = h @ C[t] + D * u[t]
+    return y
+
+
+def ssm_core(H, core, seq_len=None):
+    """The dense core between the projections (RoM page, Knowl 1: the short
+    convolution and selective state-space computation applied to H_t give
+    Y_t; Knowl 9: the 1D convolution, x projection and dt projection are
+    shared, not expertized), in the original Mamba form:
+
+      X = SiLU(conv1d(H));  [dt | B | C] = X W_x;
+      delta = softplus(dt W_dt + b_dt);  A = -exp(A_log);
+      Y = selective_scan(X, delta, A, B, C, D).
+
+    ``core`` holds conv_w [D_e, K], conv_b [D_e], w_x [D_e, R + 2N],
+    w_dt [R, D_e], b_dt [D_e], a_log [D_e, N] and d [D_e]. The T rows of H
+    are consecutive sequences of ``seq_len`` tokens (one sequence if None);
+    the convolution and the state restart at every sequence.
+    Returns Y [T, D_e] and the intermediates (X, delta, B, C).
+    """
+    H = _f64(H)
+    T, De = H.shape
+    L = T if seq_len is None else int(seq_len)
+    if T % L:
+        raise ValueError("T must be a multiple of seq_len")
+    N = np.shape(core["a_log"])[1]
+    R = np.shape(core["w_dt"])[0]
+    A = -np.exp(_f64(core["a_log"]))
+    Y = np.empty((T, De))
+    X = np.empty((T, De))
+    dl = np.empty((T, De))
+    Bs = np.empty((T, N))
+    Cs = np.empty((T, N))
+    for s0 in range(0, T, L):
+        sl = slice(s0, s0 + L)
+        xs = silu(causal_conv1d(H[sl], core["conv_w"], core["conv_b"]))
+        dbc = xs @ _f64(core["w_x"])
+        delta = softplus(dbc[:, :R] @ _f64(core["w_dt"]) + _f64(core["b_dt"])[None, :])
+        B, C = dbc[:, R:R + N], dbc[:, R + N:R + 2 * N]
+        Y[sl] = selective_scan(xs, delta, A, B, C, core["d"])
+        X[sl], dl[sl], Bs[sl], Cs[sl] = xs, delta, B, C
+    return dict(Y=Y, X=X, delta=dl, B=Bs, C=Cs)

@@ -485,3 +485,189 @@ def test_independent_routers_relabel_one_projection_alone():
     b = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"][perm], inp["w_out"], 2,
                                   {"conv": rc, "gate": rg[:, perm], "out": ro}, weighted)
     np.testing.assert_allclose(a["O"], b["O"], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------- dense core (Knowl 1, Knowl 9)
+
+
+def test_causal_conv1d_matches_numpy_convolve_and_shifts():
+    rng = np.random.default_rng(0)
+    L, D, K = 37, 5, 4
+    h = rng.standard_normal((L, D))
+    w = rng.standard_normal((D, K))
+    b = rng.standard_normal(D)
+    out = orc.causal_conv1d(h, w, b)
+    for d in range(D):
+        ref = np.convolve(h[:, d], w[d, ::-1], mode="full")[:L] + b[d]
+        np.testing.assert_allclose(out[:, d], ref, rtol=1e-13, atol=1e-13)
+    delta = np.zeros((D, K))
+    delta[:, K - 1] = 1.0
+    np.testing.assert_array_equal(orc.causal_conv1d(h, delta, np.zeros(D)), h)
+    shift = np.zeros((D, K))
+    shift[:, K - 2] = 1.0
+    s = orc.causal_conv1d(h, shift, np.zeros(D))
+    np.testing.assert_array_equal(s[1:], h[:-1])
+    np.testing.assert_array_equal(s[0], 0.0)
+
+
+def test_softplus_matches_logaddexp_without_overflow():
+    v = np.linspace(-800.0, 800.0, 3201)
+    with np.errstate(over="raise"):
+        np.testing.assert_allclose(orc.softplus(v), np.logaddexp(0.0, v), rtol=1e-14, atol=1e-300)
+
+
+def _scan_brute(u, delta, A, B, C, D):
+    """y_t = sum_{s <= t} sum_n C_t[n] exp(A[:, n] sum_{r=s+1..t} delta_r) delta_s u_s B_s[n]
+    + D u_t, summed directly (no recurrence)."""
+    L, Dd = u.shape
+    y = np.zeros((L, Dd))
+    for t in range(L):
+        for s in range(t + 1):
+            decay = np.exp(A * delta[s + 1:t + 1].sum(axis=0)[:, None])  # [D, N]
+            y[t] += (decay * (delta[s] * u[s])[:, None] * B[s][None, :]) @ C[t]
+        y[t] += D * u[t]
+    return y
+
+
+def test_selective_scan_matches_the_direct_sum():
+    rng = np.random.default_rng(1)
+    L, Dd, N = 12, 3, 4
+    u = rng.standard_normal((L, Dd))
+    delta = rng.uniform(0.01, 0.5, (L, Dd))
+    A = -rng.uniform(0.2, 3.0, (Dd, N))
+    B = rng.standard_normal((L, N))
+    C = rng.standard_normal((L, N))
+    D = rng.standard_normal(Dd)
+    np.testing.assert_allclose(orc.selective_scan(u, delta, A, B, C, D),
+                               _scan_brute(u, delta, A, B, C, D), rtol=1e-12, atol=1e-12)
+
+
+def test_selective_scan_first_step_and_causality():
+    rng = np.random.default_rng(2)
+    L, Dd, N = 20, 4, 3
+    u = rng.standard_normal((L, Dd))
+    delta = rng.uniform(0.01, 0.5, (L, Dd))
+    A = -rng.uniform(0.2, 3.0, (Dd, N))
+    B = rng.standard_normal((L, N))
+    C = rng.standard_normal((L, N))
+    D = rng.standard_normal(Dd)
+    y = orc.selective_scan(u, delta, A, B, C, D)
+    # first step: h_1 = delta u B, y = delta u (B . C) + D u
+    np.testing.assert_allclose(y[0], delta[0] * u[0] * (B[0] @ C[0]) + D * u[0], rtol=1e-14)
+    u2 = u.copy()
+    u2[9] += 5.0
+    y2 = orc.selective_scan(u2, delta, A, B, C, D)
+    np.testing.assert_array_equal(y2[:9], y[:9])
+    assert np.all(np.abs(y2[9:] - y[9:]).max(axis=1) > 0)
+
+
+def test_selective_scan_time_invariant_is_a_convolution():
+    """Constant delta, B, C (one state): y = u * k + D u with the geometric
+    kernel k_j = C exp(delta A)^j delta B."""
+    rng = np.random.default_rng(3)
+    L = 30
+    u = rng.standard_normal((L, 1))
+    dlt, a, b, c, d = 0.3, -0.7, 1.3, -0.4, 0.25
+    y = orc.selective_scan(u, np.full((L, 1), dlt), np.array([[a]]), np.full((L, 1), b),
+                           np.full((L, 1), c), np.array([d]))
+    kern = c * np.exp(dlt * a) ** np.arange(L) * dlt * b
+    ref = np.convolve(u[:, 0], kern, mode="full")[:L] + d * u[:, 0]
+    np.testing.assert_allclose(y[:, 0], ref, rtol=1e-12, atol=1e-13)
+
+
+def _core_params(De, N=4, R=3, K=4, seed=0):
+    rng = np.random.default_rng(seed)
+    return dict(conv_w=rng.standard_normal((De, K)) / 2, conv_b=0.1 * rng.standard_normal(De),
+                w_x=rng.standard_normal((De, R + 2 * N)) / np.sqrt(De),
+                w_dt=rng.standard_normal((R, De)) / np.sqrt(R),
+                b_dt=rng.uniform(np.log(1e-3), np.log(1e-1), De),
+                a_log=rng.uniform(0.0, 2.0, (De, N)), d=rng.uniform(0.5, 1.5, De))
+
+
+def test_core_restarts_at_every_sequence():
+    rng = np.random.default_rng(4)
+    H = rng.standard_normal((24, 6))
+    core = _core_params(6)
+    both = orc.ssm_core(H, core, seq_len=12)["Y"]
+    np.testing.assert_allclose(both[:12], orc.ssm_core(H[:12], core)["Y"], rtol=1e-14)
+    np.testing.assert_allclose(both[12:], orc.ssm_core(H[12:], core)["Y"], rtol=1e-14)
+
+
+def test_core_without_state_input_is_the_gated_skip():
+    """B = 0 (its columns of W_x zero): the state stays 0 and Y = D (.)
+    SiLU(conv(H)); with a delta kernel and no bias, Y = D (.) SiLU(H)."""
+    rng = np.random.default_rng(5)
+    De, N, R = 6, 4, 3
+    H = rng.standard_normal((15, De))
+    core = _core_params(De, N=N, R=R)
+    core["w_x"][:, R:R + N] = 0.0
+    core["conv_w"][:] = 0.0
+    core["conv_w"][:, -1] = 1.0
+    core["conv_b"][:] = 0.0
+    np.testing.assert_allclose(orc.ssm_core(H, core)["Y"], core["d"] * _silu_ref(H), rtol=1e-14)
+
+
+def test_block_with_core_uses_y_in_place_of_h():
+    """E = 1 block with the core: O = (core(x W_in) (.) SiLU(x W_g)) W_out,
+    the core evaluated on its own; and with a core that reduces to
+    Y = D (.) SiLU(H) the block output follows in closed form."""
+    inp = make_block_inputs(20, 8, 6, 1, seed=6)
+    core = _core_params(6)
+    x = inp["x"].astype(np.float64)
+    o = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                          core=core)["O"]
+    H = x @ inp["w_conv"][0]
+    Y = orc.ssm_core(H, core)["Y"]
+    np.testing.assert_allclose(o, (Y * _silu_ref(x @ inp["w_gate"][0])) @ inp["w_out"][0],
+                               rtol=1e-12, atol=1e-13)
+    core["w_x"][:, 3:7] = 0.0
+    core["conv_w"][:] = 0.0
+    core["conv_w"][:, -1] = 1.0
+    core["conv_b"][:] = 0.0
+    o2 = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                           core=core)["O"]
+    ref = ((core["d"] * _silu_ref(H)) * _silu_ref(x @ inp["w_gate"][0])) @ inp["w_out"][0]
+    np.testing.assert_allclose(o2, ref, rtol=1e-12, atol=1e-13)
+    with pytest.raises(ValueError):
+        orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                          core=core, tokens=[0, 1])
+
+
+def test_core_equals_its_pieces_computed_independently():
+    """The core's composition -- SiLU(conv), [dt | B | C] = X W_x in that
+    order, delta = softplus(dt W_dt + b_dt), A = -exp(A_log), the scan --
+    evaluated with numpy's convolution, logaddexp and the scan's direct sum."""
+    rng = np.random.default_rng(7)
+    De, N, R, L = 5, 3, 2, 14
+    H = rng.standard_normal((L, De))
+    core = _core_params(De, N=N, R=R, seed=8)
+    X = np.stack([np.convolve(H[:, d], core["conv_w"][d, ::-1], mode="full")[:L]
+                  for d in range(De)], axis=1) + core["conv_b"]
+    X = _silu_ref(X)
+    dbc = X @ core["w_x"]
+    delta = np.logaddexp(0.0, dbc[:, :R] @ core["w_dt"] + core["b_dt"])
+    ref = _scan_brute(X, delta, -np.exp(core["a_log"]), dbc[:, R:R + N], dbc[:, R + N:],
+                      core["d"])
+    np.testing.assert_allclose(orc.ssm_core(H, core)["Y"], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_core_is_stable_over_long_sequences():
+    """A = -exp(A_log) < 0 makes every step contractive: with bounded inputs
+    the output stays bounded over a long sequence (the stability the Swimba
+    page states for a contractive transition)."""
+    rng = np.random.default_rng(9)
+    H = rng.standard_normal((600, 4))
+    core = _core_params(4, seed=10)
+    y = orc.ssm_core(H, core)["Y"]
+    assert np.all(np.isfinite(y)) and np.abs(y).max() < 50.0
+
+
+def test_block_with_core_restarts_per_sequence():
+    inp = make_block_inputs(24, 8, 6, 3, seed=11, router_std=0.5)
+    core = _core_params(6, seed=12)
+    both = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                             core=core, seq_len=12)["O"]
+    for a in (0, 12):
+        one = orc.block_forward(inp["x"][a:a + 12], inp["w_r"], inp["w_conv"], inp["w_gate"],
+                                inp["w_out"], 1, core=core)["O"]
+        np.testing.assert_allclose(both[a:a + 12], one, rtol=1e-13, atol=1e-14)
