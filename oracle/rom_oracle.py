@@ -159,7 +159,8 @@ def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=N
     the core every token is independent of the others in this block (with
     the core, ``tokens`` is refused: a token depends on its sequence's past).
     ``seq_len``: the tokens are consecutive sequences of that length (for
-    the core).
+    the core). A core whose w_x and w_dt hold one matrix per expert
+    ([E, ...]) has its x and dt projections routed with S_t as well.
     Returns a dict with O [T,Dm], H, Gpre (the sum before SiLU), G, YG [T,De]
     and the router outputs.
     """
@@ -185,7 +186,8 @@ def block_forward(x, w_r, w_in, w_g, w_out, k, bias=None, renorm=False, tokens=N
     else:
         if tokens is not None:
             raise ValueError("the core mixes tokens over time: evaluate whole sequences")
-        Y = ssm_core(H, core, seq_len)["Y"]
+        routed = np.ndim(core["w_x"]) == 3  # x and dt projections expertized
+        Y = ssm_core(H, core, seq_len, topk_idx=S if routed else None)["Y"]
     YG = Y * G
     O = np.zeros((T, Dm))
     for i in range(E):
@@ -394,7 +396,21 @@ def selective_scan(u, delta, A, B, C, D):
     return y
 
 
-def ssm_core(H, core, seq_len=None):
+def _routed_projection(a, w, topk_idx):
+    """sum_j a_t W[S_tj] for every token t (unweighted, like the Conv and
+    Gate projections of RoM): a [T, K], w [E, K, N], topk_idx [T, k]."""
+    T = a.shape[0]
+    E, _, N = np.shape(w)
+    out = np.zeros((T, N))
+    for i in range(E):
+        for j in range(topk_idx.shape[1]):
+            sel = np.nonzero(topk_idx[:, j] == i)[0]
+            if sel.size:
+                out[sel] += a[sel] @ _f64(w[i])
+    return out
+
+
+def ssm_core(H, core, seq_len=None, topk_idx=None):
     """The dense core between the projections (RoM page, Knowl 1: the short
     convolution and selective state-space computation applied to H_t give
     Y_t; Knowl 9: the 1D convolution, x projection and dt projection are
@@ -408,6 +424,12 @@ def ssm_core(H, core, seq_len=None):
     w_dt [R, D_e], b_dt [D_e], a_log [D_e, N] and d [D_e]. The T rows of H
     are consecutive sequences of ``seq_len`` tokens (one sequence if None);
     the convolution and the state restart at every sequence.
+
+    With ``topk_idx`` [T, k] (the block's routing) the x and dt projections
+    are expertized too, like Conv and Gate (RoM page, Knowl 3 and Knowl 9:
+    "RoM (Conv, Gate, dt, x, Out)"): w_x [E, D_e, R + 2N] and w_dt [E, R, D_e]
+    hold one matrix per expert, and each token's [dt | B | C] and dt
+    projection are the sums over its selected experts (unweighted).
     Returns Y [T, D_e] and the intermediates (X, delta, B, C).
     """
     H = _f64(H)
@@ -416,7 +438,7 @@ def ssm_core(H, core, seq_len=None):
     if T % L:
         raise ValueError("T must be a multiple of seq_len")
     N = np.shape(core["a_log"])[1]
-    R = np.shape(core["w_dt"])[0]
+    R = np.shape(core["w_dt"])[-2]
     A = -np.exp(_f64(core["a_log"]))
     Y = np.empty((T, De))
     X = np.empty((T, De))
@@ -426,8 +448,14 @@ def ssm_core(H, core, seq_len=None):
     for s0 in range(0, T, L):
         sl = slice(s0, s0 + L)
         xs = silu(causal_conv1d(H[sl], core["conv_w"], core["conv_b"]))
-        dbc = xs @ _f64(core["w_x"])
-        delta = softplus(dbc[:, :R] @ _f64(core["w_dt"]) + _f64(core["b_dt"])[None, :])
+        if topk_idx is None:
+            dbc = xs @ _f64(core["w_x"])
+            pre = dbc[:, :R] @ _f64(core["w_dt"])
+        else:
+            S = np.asarray(topk_idx)[sl]
+            dbc = _routed_projection(xs, core["w_x"], S)
+            pre = _routed_projection(dbc[:, :R], core["w_dt"], S)
+        delta = softplus(pre + _f64(core["b_dt"])[None, :])
         B, C = dbc[:, R:R + N], dbc[:, R + N:R + 2 * N]
         Y[sl] = selective_scan(xs, delta, A, B, C, core["d"])
         X[sl], dl[sl], Bs[sl], Cs[sl] = xs, delta, B, C

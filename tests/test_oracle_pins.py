@@ -671,3 +671,73 @@ def test_block_with_core_restarts_per_sequence():
         one = orc.block_forward(inp["x"][a:a + 12], inp["w_r"], inp["w_conv"], inp["w_gate"],
                                 inp["w_out"], 1, core=core)["O"]
         np.testing.assert_allclose(both[a:a + 12], one, rtol=1e-13, atol=1e-14)
+
+
+def _routed_core_params(De, E, N=3, R=2, seed=0):
+    base = _core_params(De, N=N, R=R, seed=seed)
+    rng = np.random.default_rng(seed + 100)
+    base["w_x"] = rng.standard_normal((E, De, R + 2 * N)) / np.sqrt(De)
+    base["w_dt"] = rng.standard_normal((E, R, De)) / np.sqrt(R)
+    return base
+
+
+def test_routed_core_with_identical_experts_is_the_shared_core():
+    rng = np.random.default_rng(13)
+    De, E = 5, 4
+    H = rng.standard_normal((30, De))
+    p = _routed_core_params(De, E)
+    p["w_x"][:] = p["w_x"][0]
+    p["w_dt"][:] = p["w_dt"][0]
+    shared = dict(p, w_x=p["w_x"][0], w_dt=p["w_dt"][0])
+    S = rng.integers(0, E, (30, 1))
+    np.testing.assert_allclose(orc.ssm_core(H, p, topk_idx=S)["Y"], orc.ssm_core(H, shared)["Y"],
+                               rtol=1e-13, atol=1e-14)
+
+
+def test_routed_core_top1_uses_each_tokens_expert():
+    """Top-1: token t's [dt | B | C] is X_t W_x[e_t] and its dt projection
+    uses W_dt[e_t]; built token by token and fed to the scan's direct sum."""
+    rng = np.random.default_rng(14)
+    De, E, N, R, L = 4, 3, 3, 2, 12
+    H = rng.standard_normal((L, De))
+    p = _routed_core_params(De, E, N=N, R=R, seed=15)
+    S = rng.integers(0, E, (L, 1))
+    X = _silu_ref(orc.causal_conv1d(H, p["conv_w"], p["conv_b"]))
+    dbc = np.stack([X[t] @ p["w_x"][S[t, 0]] for t in range(L)])
+    pre = np.stack([dbc[t, :R] @ p["w_dt"][S[t, 0]] for t in range(L)])
+    delta = np.logaddexp(0.0, pre + p["b_dt"])
+    ref = _scan_brute(X, delta, -np.exp(p["a_log"]), dbc[:, R:R + N], dbc[:, R + N:], p["d"])
+    np.testing.assert_allclose(orc.ssm_core(H, p, topk_idx=S)["Y"], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_block_with_routed_core_uses_the_block_routing():
+    """In the block, the expertized x and dt projections follow S_t: with
+    k = E every expert is selected, so they see the sum of all experts'
+    matrices (a shared core with the summed weights)."""
+    E = 3
+    inp = make_block_inputs(16, 8, 6, E, seed=16, router_std=0.5)
+    p = _routed_core_params(6, E, seed=17)
+    summed = dict(p, w_x=p["w_x"].sum(axis=0), w_dt=p["w_dt"].sum(axis=0))
+    a = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], E,
+                          core=p)["O"]
+    b = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], E,
+                          core=summed)["O"]
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+
+
+def test_block_with_routed_core_top1_follows_its_router():
+    """Top-1 block with an expertized core equals its pieces: the routing of
+    the block's router drives Conv, Gate, the x and dt projections and Out."""
+    E = 3
+    inp = make_block_inputs(16, 8, 6, E, seed=18, router_std=0.5)
+    p = _routed_core_params(6, E, seed=19)
+    o = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"], 1,
+                          core=p)["O"]
+    x = inp["x"].astype(np.float64)
+    pr = sp_softmax(x @ inp["w_r"].astype(np.float64), axis=1)
+    e = np.argmax(pr, axis=1)
+    H = np.stack([x[t] @ inp["w_conv"][e[t]] for t in range(16)])
+    G = _silu_ref(np.stack([x[t] @ inp["w_gate"][e[t]] for t in range(16)]))
+    Y = orc.ssm_core(H, p, topk_idx=e[:, None])["Y"]
+    ref = np.stack([pr[t, e[t]] * ((Y[t] * G[t]) @ inp["w_out"][e[t]]) for t in range(16)])
+    np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-12)
