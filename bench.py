@@ -20,7 +20,9 @@ reported time is the max over ranks and `value` counts all ranks' tokens.
 A single-GPU run also times the other configurations of the block (decode
 in-projection, top-2 forward + backward, load-imbalanced, tiny float32, and
 the independently routed and RoM (Gate, Out) projection variants at the
-prefill shape) and reports them under "workloads"; `--no-extra` skips them.
+prefill shape, and the prefill block with the dense core between the
+projections, its x and dt projections shared or expertized) and reports them
+under "workloads"; `--no-extra` skips them.
 
 `--impl reference` times the CPU oracle (the float64 numpy definition) on the
 host cores, on the whole workload per step when that fits about two minutes
@@ -241,6 +243,16 @@ def oracle_sample_run(wl, inp, tokens):
         w_conv = inp["w_conv"][:1] if routers["conv"] is None else inp["w_conv"]
         orc.variant_block_forward(inp["x"], w_conv, inp["w_gate"], inp["w_out"], wl.k, routers,
                                   weighted, renorm=wl.renorm, tokens=tokens)
+    elif wl.core:
+        # The core mixes tokens over time, so a sample of n tokens is the
+        # first n of the batch (whole sequences, or a prefix of the first
+        # one): their outputs are those of the whole workload.
+        L = wl.seq_len or wl.T
+        n = wl.T if tokens is None else len(tokens)
+        n = (n // L) * L if n >= L else n
+        orc.block_forward(inp["x"][:n], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                          k=wl.k, bias=inp["bias"], renorm=wl.renorm, core=inp["core"],
+                          seq_len=min(n, L))
     else:
         orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
                           k=wl.k, bias=inp["bias"], renorm=wl.renorm, tokens=tokens)
@@ -368,6 +380,40 @@ def build_workload(torch, rom, wl, inp):
                    dominant=(dominant, "flop", lambda counts: flops["conv"]),
                    out=bufs.out, counts=main_rb.counts,
                    launches=2 * n_routings + 2 + 2 + (1 if wl.k > 1 else 0))
+        res["e2e"] = None
+    elif wl.core:
+        # the block with the dense core between the projections (top-1)
+        assert wl.k == 1
+        ws = {n: to_dev(torch, inp[n], bf16).transpose(1, 2).contiguous()
+              for n in ("w_conv", "w_gate", "w_out")}
+        in_bytes += sum(t.numel() * t.element_size() for t in ws.values())
+        core = rom.CoreParams(inp["core"], x.device)
+        L = wl.seq_len or wl.T
+        bufs = rom.BlockBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device, core, L)
+        rb = bufs.routing
+        flat = bufs.uz.view(2 * R, wl.De)
+
+        def ph_route():
+            rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, rb)
+
+        def ph_p0():
+            rom.rom_expert_proj(rom.ROM_PROJ_CONV_GATE_SLOTS, rb.x_sorted[:R], ws["w_conv"],
+                                ws["w_gate"], wl.E, wl.k, rb.offsets, rb.sorted_slot, rb.topk_w,
+                                bufs.uz)
+
+        def ph_core():
+            rom.rom_ssm_core(flat[:wl.T], L, core, flat[:wl.T], bufs.core_ws, routing=rb)
+
+        def ph_p1():
+            rom.rom_combine(rom.ROM_COMBINE_GATE_DENSE, dt, flat, wl.T, 1, wl.De, rb.slot_pos,
+                            bufs.h_sorted)
+            rom.rom_expert_proj(rom.ROM_PROJ_OUT, bufs.h_sorted[:R], ws["w_out"], None, wl.E, 1,
+                                rb.offsets, rb.sorted_slot, rb.topk_w, bufs.out)
+        res.update(phases=[("route_dispatch", ph_route), ("proj0", ph_p0), ("core", ph_core),
+                           ("proj1", ph_p1)],
+                   dominant=(ph_p0, "flop", lambda counts: flops["conv_gate"]),
+                   out=bufs.out, counts=rb.counts,
+                   launches=4 + 7 + 1 + (2 if wl.core_routed else 0))
         res["e2e"] = None
     else:
         ws = {n: to_dev(torch, inp[n], bf16).transpose(1, 2).contiguous()
@@ -630,7 +676,8 @@ def reference_arm(args, wl, metric, config, world):
 # Workloads timed next to the headline in a single-GPU run: the other
 # configurations of the block, each reported under "workloads".
 EXTRA_WORKLOADS = ["decode_swimba_inproj", "top2_fwd_bwd", "imbalanced_8x4096", "tiny_fp32",
-                   "independent_moe_16k", "rom_gate_out_16k"]
+                   "independent_moe_16k", "rom_gate_out_16k", "prefill_16k_core",
+                   "prefill_16k_core_dtx"]
 
 
 def main():
@@ -651,7 +698,9 @@ def main():
 
     if args.tokens is not None:
         import dataclasses
-        WORKLOADS[args.workload] = dataclasses.replace(WORKLOADS[args.workload], T=args.tokens)
+        w0 = WORKLOADS[args.workload]
+        WORKLOADS[args.workload] = dataclasses.replace(
+            w0, T=args.tokens, seq_len=min(w0.seq_len, args.tokens) if w0.seq_len else 0)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -59,7 +59,8 @@ typedef enum {
   ROM_PROJ_CONV_GATE = 0, /* Conv (input) and Gate projections, shared selection */
   ROM_PROJ_OUT = 1,       /* Out projection, weighted by r */
   ROM_PROJ_INPROJ = 2,    /* Swimba routed in-projection, weighted by r */
-  ROM_PROJ_SLOTS = 3      /* one projection to float32 slot rows (Conv or Gate on their own) */
+  ROM_PROJ_SLOTS = 3,     /* one projection to float32 slot rows (Conv or Gate on their own) */
+  ROM_PROJ_CONV_GATE_SLOTS = 4 /* Conv and Gate to float32 u, z slot rows for any k */
 } rom_proj;
 
 typedef enum {
@@ -146,6 +147,9 @@ int rom_dispatch(const void* x, int dtype, int64_t T, int Dm, int E, int k,
  *     k  > 1: out = float32 [2][R][N] in SLOT order: out[0][s] = u, out[1][s] = z
  *             of slot s; rom_combine(ROM_COMBINE_GATE) then sums over the
  *             slots before SiLU.
+ *  ROM_PROJ_CONV_GATE_SLOTS: as ROM_PROJ_CONV_GATE with k > 1 (u and z as
+ *     float32 [2][R][N] in slot order) for any k, including k == 1: the
+ *     input of the dense core (rom_ssm_core), which needs H before the gate.
  *  ROM_PROJ_OUT (RoM page, Knowl 1, O_t): w0 = W_out [E][N][K] (K = D_e, N = D_m),
  *     w1 = NULL. Each row is scaled by r = topk_w[slot] in float32.
  *     k == 1: out = O [T][N] dtype in token order;
@@ -280,6 +284,62 @@ int rom_route_bwd(int64_t T, int k, int E, int Dm, int renorm, const int32_t* to
  */
 int rom_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int64_t R, int E,
                   const int32_t* offsets, int m_split, float* out0, float* out1, void* stream);
+
+/* ------------------------------------------------------------------------
+ * The dense core between the projections (RoM page, Knowl 1: the short
+ * convolution and the selective state-space computation applied to H_t
+ * produce Y_t; Knowl 9: the 1D convolution and the x and dt projections are
+ * shared by all experts), in the original Mamba form (zero-order hold for A,
+ * Euler step for the input):
+ *   X = SiLU(conv1d(H) + conv_b);  [dt | B | C] = X W_x;
+ *   delta = softplus(dt W_dt + b_dt);  A = -exp(A_log);
+ *   h_t = exp(delta_t A) (.) h_{t-1} + (delta_t x_t) B_t,  Y_t = h_t C_t + D (.) x_t.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of workspace rom_ssm_core needs (0 for invalid sizes). Host function. */
+size_t rom_ssm_core_workspace_size(int64_t T, int De, int seq_len, int R, int N, int Np);
+
+/*
+ * rom_ssm_core -- Y = core(H) for T = (T / seq_len) consecutive sequences of
+ * seq_len tokens each (the convolution and the state restart at every
+ * sequence).
+ *
+ *  h       [T][De] float32, token order (the Conv projection H)
+ *  conv_w  [De][K] float32: tap K-1 multiplies the current step, tap K-1-j
+ *          the step j back;  conv_b [De] float32;  K <= 8
+ *  w_x     bf16 [Np][De]: row j < R + 2N is column j of W_x ([De][R + 2N] in
+ *          the pages' x W notation: dt, then B, then C); rows R + 2N .. Np-1
+ *          zero; Np % 128 == 0
+ *  w_dt    bf16 [De][R]: W_dt ([R][De]) transposed; R % 8 == 0
+ *  b_dt    [De], a_log [De][N] (N <= 16), d [De]: float32
+ *  y       [T][De] float32 out; may be the same buffer as h
+ *  ws      workspace of rom_ssm_core_workspace_size() bytes, 256-byte aligned
+ * X and dt are rounded to bf16 for the two projections (tensor cores); the
+ * convolution, softplus and the scan run in float32. Requires De % 128 == 0.
+ */
+int rom_ssm_core(const float* h, int64_t T, int De, int seq_len, const float* conv_w,
+                 const float* conv_b, int K, const void* w_x, int R, int N, int Np,
+                 const void* w_dt, const float* b_dt, const float* a_log, const float* d,
+                 float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace rom_ssm_core_routed needs (0 for invalid sizes). */
+size_t rom_ssm_core_routed_workspace_size(int64_t T, int De, int seq_len, int R, int N, int Np,
+                                          int k);
+
+/*
+ * rom_ssm_core_routed -- rom_ssm_core with the x and dt projections
+ * expertized, routed by the block's own selection (RoM page, Knowl 3: "RoM
+ * (Conv, Gate, dt, x, Out)"; Knowl 9: the dt and x ablation). w_x holds E
+ * matrices [E][Np][De] and w_dt [E][De][R]; offsets, sorted_slot (from
+ * rom_dispatch of the block, k slots per token) select each token's experts,
+ * and its [dt | B | C] and dt projection are the sums over its k selected
+ * experts, unweighted (as H and G). Other arguments as rom_ssm_core.
+ */
+int rom_ssm_core_routed(const float* h, int64_t T, int De, int seq_len, const float* conv_w,
+                        const float* conv_b, int K, const void* w_x, int R, int N, int Np,
+                        const void* w_dt, const float* b_dt, const float* a_log, const float* d,
+                        int E, int k, const int32_t* offsets, const int32_t* sorted_slot,
+                        float* y, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * rom_route_dispatch_noalloc -- rom_route() followed by rom_dispatch(), for

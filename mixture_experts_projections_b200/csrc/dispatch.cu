@@ -58,6 +58,10 @@ __global__ void __launch_bounds__(kDispatchThreads)
   const int64_t s0 = c * chunk_slots;
   const int ns = static_cast<int>(std::min<int64_t>(chunk_slots, R - s0));
   const int ngroups = (ns + 31) / 32;
+  // Launched as a programmatic dependent of the router: the kernel after
+  // this one may start now; the router's outputs are read only after
+  // pdl_wait().
+  pdl_launch_dependents();
 
   for (int e = tid; e < E; e += kDispatchThreads) {
     s_tot[e] = 0;
@@ -70,6 +74,7 @@ __global__ void __launch_bounds__(kDispatchThreads)
     s_bad_hist = 0;
     s_bad_chunk = 0;
   }
+  pdl_wait();
   __syncthreads();
   // Histogram entries outside [0, slots of their chunk] are refused; with
   // that bound no per-expert total can exceed R.
@@ -225,11 +230,21 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int64_t T, int Dm, int E, 
   const int64_t want = (2 * static_cast<int64_t>(device_sm_count())) / nchunks;
   const int nslices = static_cast<int>(
       std::max<int64_t>(1, std::min<int64_t>({want, 16, (row_bytes / 16) / 32})));
-  dispatch_kernel<<<dim3(static_cast<unsigned>(nchunks), static_cast<unsigned>(nslices)),
-                    kDispatchThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), T, row_bytes / 16, E, k, topk_idx, chunk_hist, nchunks,
-      offsets, sorted_slot, slot_pos, static_cast<uint4*>(x_sorted), status);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the CTAs may start (and be resident)
+  // while the router finishes; they wait for it before reading its outputs.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nchunks), static_cast<unsigned>(nslices), 1);
+  cfg.blockDim = dim3(kDispatchThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dispatch_kernel, static_cast<const uint4*>(x), T,
+                            row_bytes / 16, E, k, topk_idx, chunk_hist, nchunks, offsets,
+                            sorted_slot, slot_pos, static_cast<uint4*>(x_sorted), status);
 }
 
 }  // namespace rom

@@ -162,26 +162,27 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
                     const void* w1, int N, int E, int k, const int32_t* offsets,
                     const int32_t* sorted_slot, const float* topk_w, void* out, void* stream) {
   if (proj != ROM_PROJ_CONV_GATE && proj != ROM_PROJ_OUT && proj != ROM_PROJ_INPROJ &&
-      proj != ROM_PROJ_SLOTS)
+      proj != ROM_PROJ_SLOTS && proj != ROM_PROJ_CONV_GATE_SLOTS)
     return ROM_ERR_INVALID_ARG;
   if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
   if (R < 0 || K <= 0 || N <= 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E ||
       k > rom::kMaxTopK || R % k != 0)
     return ROM_ERR_INVALID_ARG;
   if (R >= (int64_t(1) << 31)) return ROM_ERR_UNSUPPORTED;
-  const bool gate = proj == ROM_PROJ_CONV_GATE;
+  const bool gate = proj == ROM_PROJ_CONV_GATE || proj == ROM_PROJ_CONV_GATE_SLOTS;
+  const bool gate_slots = proj == ROM_PROJ_CONV_GATE_SLOTS || (gate && k > 1);
   const bool slots = proj == ROM_PROJ_SLOTS;
   // A dense projection (ROM_PROJ_SLOTS only): no routing arrays, one matrix.
   const bool dense = slots && !offsets && !sorted_slot;
   if (dense && E != 1) return ROM_ERR_INVALID_ARG;
   if ((!offsets && !dense) || !w0 || !out || (gate && !w1)) return ROM_ERR_INVALID_ARG;
   if (!gate && !dense && (!sorted_slot || (!slots && !topk_w))) return ROM_ERR_INVALID_ARG;
-  if (gate && k > 1 && !sorted_slot) return ROM_ERR_INVALID_ARG;
+  if (gate_slots && !sorted_slot) return ROM_ERR_INVALID_ARG;
   if (R > 0 && !a_sorted) return ROM_ERR_INVALID_ARG;
   if (slots) w1 = nullptr;
   // ROM_PROJ_SLOTS is the slot-order float32 epilogue; r = 1 when topk_w is
   // NULL, and row p is slot p when sorted_slot is NULL.
-  const int mode = gate    ? (k == 1 ? rom::kEpiGateH : rom::kEpiGateSlots)
+  const int mode = gate    ? (gate_slots ? rom::kEpiGateSlots : rom::kEpiGateH)
                    : slots ? rom::kEpiScaleSlots
                            : (k == 1 ? rom::kEpiScaleToken : rom::kEpiScaleSlots);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -18,6 +18,19 @@ inline int64_t num_chunks(int64_t T) { return (T + kChunkTokens - 1) / kChunkTok
 // Device status codes written by kernels (the same values as rom_status).
 constexpr int kStatusRouting = 6;  // == ROM_ERR_ROUTING
 
+// Programmatic dependent launch. A kernel launched with
+// cudaLaunchAttributeProgrammaticStreamSerialization may start while the
+// kernel before it on the stream still runs, once every CTA of that kernel
+// has called pdl_launch_dependents() (or exited). It must call pdl_wait()
+// -- which returns when the kernels before it have completed and their
+// writes are visible -- before it reads anything they wrote, and every CTA
+// calls it before exiting, so that its own completion still implies theirs.
+// Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 int device_sm_count();  // cached per device
 
 // Device address of this device's status word (nullptr on failure), looked

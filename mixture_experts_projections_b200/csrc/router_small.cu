@@ -67,6 +67,9 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t t = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + t * Dm);
+  // The dispatch that follows may be launched now: its CTAs wait for this
+  // grid to complete before they read anything it writes.
+  pdl_launch_dependents();
   const int npc = Dm / kPiece;
 
   float v[NV];

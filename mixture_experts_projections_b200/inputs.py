@@ -49,6 +49,13 @@ class Workload:
     # projection a conventional MoE layer) or "gate_out" (dense Conv, one
     # router shared by Gate and Out)
     variant: str = ""
+    # the dense core (conv + selective scan) between the projections instead
+    # of the identity, over sequences of seq_len tokens (0: one sequence)
+    core: bool = False
+    seq_len: int = 0
+    # the core's x and dt projections expertized too ("RoM (Conv, Gate, dt,
+    # x, Out)")
+    core_routed: bool = False
 
 
 # Router-bias constants of the load-imbalanced workload. They were found by
@@ -76,7 +83,18 @@ WORKLOADS = {
                                     E=8, k=1, dtype="bf16", variant="independent"),
     "rom_gate_out_16k": Workload("rom_gate_out_16k", "variant", T=16384, Dm=2048, De=4096, E=8,
                                  k=1, dtype="bf16", variant="gate_out"),
+    # The prefill block with the dense core between the projections.
+    "prefill_16k_core": Workload("prefill_16k_core", "block", T=16384, Dm=2048, De=4096, E=8,
+                                 k=1, dtype="bf16", core=True, seq_len=16384),
+    "prefill_16k_core_dtx": Workload("prefill_16k_core_dtx", "block", T=16384, Dm=2048, De=4096,
+                                     E=8, k=1, dtype="bf16", core=True, seq_len=16384,
+                                     core_routed=True),
 }
+
+# Sizes of the core: state size, convolution taps and the rank of the dt
+# projection (d_model / 16, rounded up to a multiple of 8).
+CORE_STATE = 16
+CORE_TAPS = 4
 
 # The order the workloads are listed in (the small fp32 case first).
 WORKLOAD_ORDER = ["tiny_fp32", "prefill_16k", "imbalanced_8x4096", "decode_swimba_inproj",
@@ -157,13 +175,47 @@ def make_inproj_inputs(T, Dm, N_out, E, *, seed=0, dtype="bf16", router_std=0.02
     return dict(x=x, w_r=w_r, bias=None, w=w)
 
 
+def core_dt_rank(Dm: int) -> int:
+    """Rank of the dt projection: ceil(d_model / 16), rounded up to a multiple of 8."""
+    r = -(-Dm // 16)
+    return max(8, -(-r // 8) * 8)
+
+
+def make_core_params(De, Dm, *, seed=0, N=CORE_STATE, K=CORE_TAPS, experts=None):
+    """Parameters of the dense core for d_inner = De (float32 numpy, in the
+    pages' x W notation), from their own generator (seeded by (seed, 1)) so
+    the block's other inputs do not change:
+      conv_w [De, K] ~ N(0, 1/K), conv_b [De] ~ N(0, 0.1^2),
+      w_x [De, R + 2N] ~ N(0, 1/De) and w_dt [R, De] ~ N(0, 1/R), both
+      rounded to bf16 (the library's projection dtype), R = core_dt_rank(Dm),
+      b_dt [De] ~ U[ln 1e-3, ln 1e-1] (softplus then gives delta of about
+      1e-3 .. 1e-1), a_log [De, N] ~ U[0, 3], d [De] ~ U[0.5, 1.5].
+    With ``experts`` = E, w_x and w_dt hold one matrix per expert
+    ([E, De, R + 2N] and [E, R, De]: the x and dt projections expertized)."""
+    rng = np.random.default_rng([seed, 1])
+    R = core_dt_rank(Dm)
+    lead = () if experts is None else (experts,)
+    return dict(
+        conv_w=_draw(rng, (De, K), 1.0 / np.sqrt(K), False),
+        conv_b=_draw(rng, (De,), 0.1, False),
+        w_x=_draw(rng, lead + (De, R + 2 * N), 1.0 / np.sqrt(De), True),
+        w_dt=_draw(rng, lead + (R, De), 1.0 / np.sqrt(R), True),
+        b_dt=rng.uniform(np.log(1e-3), np.log(1e-1), De).astype(np.float32),
+        a_log=rng.uniform(0.0, 3.0, (De, N)).astype(np.float32),
+        d=rng.uniform(0.5, 1.5, De).astype(np.float32))
+
+
 def make_workload_inputs(wl: Workload, seed=0):
     """Inputs of a named workload at its full size."""
     T = wl.T
     if wl.kind == "inproj":
         return make_inproj_inputs(T, wl.Dm, wl.De, wl.E, seed=seed, dtype=wl.dtype,
                                   router_std=wl.router_std)
-    return make_block_inputs(T, wl.Dm, wl.De, wl.E, seed=seed, dtype=wl.dtype,
-                             router_std=wl.router_std, bias=bias_vector(wl.E, wl.bias),
-                             with_dout=wl.backward, extra_routers=wl.variant == "independent")
+    inp = make_block_inputs(T, wl.Dm, wl.De, wl.E, seed=seed, dtype=wl.dtype,
+                            router_std=wl.router_std, bias=bias_vector(wl.E, wl.bias),
+                            with_dout=wl.backward, extra_routers=wl.variant == "independent")
+    if wl.core:
+        inp["core"] = make_core_params(wl.De, wl.Dm, seed=seed,
+                                       experts=wl.E if wl.core_routed else None)
+    return inp
 

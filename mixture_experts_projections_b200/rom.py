@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "librom.so")
 ROM_OK, ROM_ERR_INVALID_ARG, ROM_ERR_UNSUPPORTED, ROM_ERR_WORKSPACE, ROM_ERR_CUDA, \
     ROM_ERR_TIMEOUT, ROM_ERR_ROUTING = range(7)
 ROM_F32, ROM_BF16 = 0, 1
-ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ, ROM_PROJ_SLOTS = 0, 1, 2, 3
+ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ, ROM_PROJ_SLOTS, ROM_PROJ_CONV_GATE_SLOTS = \
+    0, 1, 2, 3, 4
 ROM_COMBINE_SUM, ROM_COMBINE_GATE, ROM_COMBINE_GATE_DENSE = 0, 1, 2
 
 # Every exported symbol of include/rom.h with its ctypes signature.
@@ -46,6 +47,12 @@ SIGNATURES = {
     "rom_bwd_dgrad_in": (_I, [_P, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P]),
     "rom_route_bwd": (_I, [_L, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
     "rom_bwd_wgrad": (_I, [_P, _I, _P, _I, _L, _I, _P, _I, _P, _P, _P]),
+    "rom_ssm_core_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I]),
+    "rom_ssm_core_routed_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I, _I]),
+    "rom_ssm_core_routed": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P,
+                                 _I, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "rom_ssm_core": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                          ctypes.c_size_t, _P]),
 }
 
 _lib = None
@@ -200,34 +207,132 @@ def route_and_dispatch(x, w_r, bias, E, k, renorm, bufs=None, stream=None):
     return bufs
 
 
+# ------------------------------------------------------------------ dense core
+
+
+class CoreParams:
+    """The dense core's parameters on the device in the library's layout
+    (from float32 arrays in the pages' x W notation: conv_w [De, K],
+    conv_b [De], w_x [De, R + 2N], w_dt [R, De], b_dt [De], a_log [De, N],
+    d [De]; w_x and w_dt must hold bf16 values). With w_x [E, De, R + 2N]
+    and w_dt [E, R, De] the x and dt projections are expertized
+    (``self.E`` matrices, routed with the block's selection)."""
+
+    def __init__(self, p, device="cuda"):
+        import numpy as np
+        De, K = p["conv_w"].shape
+        wx_p = np.asarray(p["w_x"], np.float32)
+        wdt_p = np.asarray(p["w_dt"], np.float32)
+        self.routed = wx_p.ndim == 3
+        if not self.routed:
+            wx_p, wdt_p = wx_p[None], wdt_p[None]
+        self.E = wx_p.shape[0]
+        self.R = wdt_p.shape[1]
+        self.De = De
+        self.N = p["a_log"].shape[1]
+        self.K = K
+        self.Np = -(-(self.R + 2 * self.N) // 128) * 128
+
+        def f32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+        self.conv_w, self.conv_b = f32(p["conv_w"]), f32(p["conv_b"])
+        self.b_dt, self.a_log, self.d = f32(p["b_dt"]), f32(p["a_log"]), f32(p["d"])
+        wx = torch.zeros((self.E, self.Np, De), dtype=torch.float32)
+        wx[:, :self.R + 2 * self.N] = torch.from_numpy(np.ascontiguousarray(wx_p)).transpose(1, 2)
+        self.w_x = wx.to(torch.bfloat16).to(device).contiguous()  # exact: bf16 values
+        self.w_dt = torch.from_numpy(np.ascontiguousarray(wdt_p)).transpose(1, 2).contiguous() \
+            .to(torch.bfloat16).to(device)
+
+
+def rom_ssm_core_workspace_size(T, De, seq_len, R, N, Np):
+    return int(load_library().rom_ssm_core_workspace_size(T, De, seq_len, R, N, Np))
+
+
+def rom_ssm_core(h, seq_len, core, y, ws, stream=None, routing=None):
+    """Y = core(H) (h, y: float32 [T, De], may be the same tensor). An
+    expertized core takes the block's RoutingBuffers as ``routing``."""
+    T, De = h.shape
+    common = (_ptr(h), T, De, seq_len, _ptr(core.conv_w), _ptr(core.conv_b), core.K,
+              _ptr(core.w_x), core.R, core.N, core.Np, _ptr(core.w_dt), _ptr(core.b_dt),
+              _ptr(core.a_log), _ptr(core.d))
+    tail = (_ptr(y), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+            _stream(stream))
+    if core.routed:
+        _check(load_library().rom_ssm_core_routed(
+            *common, core.E, routing.k, _ptr(routing.offsets), _ptr(routing.sorted_slot), *tail),
+            "rom_ssm_core_routed")
+    else:
+        _check(load_library().rom_ssm_core(*common, *tail), "rom_ssm_core")
+
+
+def core_workspace(T, De, seq_len, core, device, k=1):
+    if core.routed:
+        n = int(load_library().rom_ssm_core_routed_workspace_size(T, De, seq_len, core.R, core.N,
+                                                                  core.Np, k))
+    else:
+        n = rom_ssm_core_workspace_size(T, De, seq_len, core.R, core.N, core.Np)
+    return torch.empty((max(n, 256),), dtype=torch.uint8, device=device)
+
+
 class BlockBuffers:
     """Intermediate and output buffers of one RoM block forward."""
 
-    def __init__(self, T, Dm, De, E, k, dtype, device):
+    def __init__(self, T, Dm, De, E, k, dtype, device, core=None, seq_len=None):
         R = T * k
         self.routing = RoutingBuffers(T, Dm, E, k, dtype, device)
         self.h_sorted = torch.empty((max(R, 1), De), dtype=dtype, device=device)
         self.uz = (torch.empty((2, R, De), dtype=torch.float32, device=device)
-                   if k > 1 else None)
+                   if (k > 1 or core is not None) else None)
+        self.core_ws = (core_workspace(T, De, seq_len or T, core, device, k)
+                        if core is not None else None)
+        self.hsum = (torch.empty((T, De), dtype=torch.float32, device=device)
+                     if (core is not None and k > 1) else None)
         self.o_slots = (torch.empty((R, Dm), dtype=torch.float32, device=device)
                         if k > 1 else None)
         self.out = torch.empty((T, Dm), dtype=dtype, device=device)
 
 
-def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=None, stream=None):
+def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=None, stream=None,
+                  core=None, seq_len=None):
     """RoM block forward: route, dispatch, Conv+Gate, (gate combine), Out, (sum).
 
     x [T, Dm] (bf16 or float32), w_r [Dm, E] float32, bias [E] float32 or None,
     w_conv, w_gate [E, De, Dm] and w_out [E, Dm, De] in the library layout.
-    Returns the BlockBuffers holding O (``.out``) and the intermediates.
+    ``core`` (CoreParams): the dense core runs between the projections, Y =
+    core(H), over sequences of ``seq_len`` tokens (all T if None); without it
+    Y = H. Returns the BlockBuffers holding O (``.out``) and the intermediates.
     """
     T, Dm = x.shape
     E, De, _ = w_conv.shape
     if bufs is None:
-        bufs = BlockBuffers(T, Dm, De, E, k, x.dtype, x.device)
+        bufs = BlockBuffers(T, Dm, De, E, k, x.dtype, x.device, core, seq_len)
     rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs.routing, stream)
     R = T * k
     xs = rb.x_sorted[:R]
+    if core is not None:
+        # u and z per slot (float32); H in token order (the sum over the
+        # slots for k > 1); Y = core(H) written just before the z rows, so
+        # that [Y; z] feed the gate combine (Y per token, z per slot).
+        rom_expert_proj(ROM_PROJ_CONV_GATE_SLOTS, xs, w_conv, w_gate, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, bufs.uz, stream)
+        flat = bufs.uz.view(2 * R, De)
+        y_rows = flat[R - T:R]
+        if k > 1:
+            rom_combine(ROM_COMBINE_SUM, ROM_F32, bufs.uz[0], T, k, De, None, bufs.hsum, stream)
+            rom_ssm_core(bufs.hsum, seq_len or T, core, y_rows, bufs.core_ws, stream, rb)
+        else:
+            rom_ssm_core(flat[:T], seq_len or T, core, y_rows, bufs.core_ws, stream, rb)
+        rom_combine(ROM_COMBINE_GATE_DENSE, _dtype_code(x), flat[R - T:], T, k, De, rb.slot_pos,
+                    bufs.h_sorted, stream)
+        if k == 1:
+            rom_expert_proj(ROM_PROJ_OUT, bufs.h_sorted[:R], w_out, None, E, k, rb.offsets,
+                            rb.sorted_slot, rb.topk_w, bufs.out, stream)
+        else:
+            rom_expert_proj(ROM_PROJ_OUT, bufs.h_sorted[:R], w_out, None, E, k, rb.offsets,
+                            rb.sorted_slot, rb.topk_w, bufs.o_slots, stream)
+            rom_combine(ROM_COMBINE_SUM, _dtype_code(x), bufs.o_slots, T, k, Dm, None, bufs.out,
+                        stream)
+        return bufs
     if k == 1:
         rom_expert_proj(ROM_PROJ_CONV_GATE, xs, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
                         rb.topk_w, bufs.h_sorted, stream)

@@ -71,7 +71,7 @@ def test_route_rejects_bad_arguments(lib, kw, code):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(proj=4), 1), (dict(dtype=2), 1), (dict(K=0), 1), (dict(N=0), 1), (dict(k=2, R=7), 1),
+    (dict(proj=5), 1), (dict(dtype=2), 1), (dict(K=0), 1), (dict(N=0), 1), (dict(k=2, R=7), 1),
     # ROM_PROJ_SLOTS: a dense projection (no routing arrays) needs E == 1; a
     # routed one needs both offsets and sorted_slot
     (dict(proj=3, offsets=None, sorted_slot=None), 1), (dict(proj=3, offsets=None), 1),
