@@ -261,17 +261,39 @@ int rom_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const void* w_in
                      const int32_t* sorted_slot, float* dx_slots, void* stream);
 
 /*
- * Router backward and dX: dr_{t,j} = (sum of dr_part[s][0 .. n_parts)) / r_s;
- * dlogits [T][E] float32 (may be NULL; zero off S_t);
- * dx [T][Dm] bf16 = sum_j dx_slots[t*k+j] + sum_j dlogit_{t,j} w_r[:, S_j].
- * The weights must be renormalised (renorm = 1): r = p without
- * renormalisation would need every expert's probability (ROM_ERR_UNSUPPORTED).
+ * Router backward and dX: dr_{t,j} = (sum of dr_part[s][0 .. n_parts)) / r_s,
+ * s = sum_j r_{t,j} dr_{t,j};
+ *   renorm = 1 (r = softmax over the selected logits):
+ *     dlogit = r_j (dr_j - s) on S_t, 0 elsewhere; probs unused (may be NULL);
+ *   renorm = 0 (r = p, the formula of Knowl 1): dlogit_m = p_m (dr_j - s) for
+ *     m = S_j and -p_m s off S_t, which needs probs [T][E] float32, the
+ *     softmax over all E experts (rom_route_probs).
+ * dlogits [T][E] float32 (may be NULL);
+ * dx [T][Dm] bf16 = sum_j dx_slots[t*k+j] + sum_m dlogit_{t,m} w_r[:, m].
  * Requires Dm % 4 == 0.
  */
 int rom_route_bwd(int64_t T, int k, int E, int Dm, int renorm, const int32_t* topk_idx,
-                  const float* topk_w, const float* dr_part, int n_parts,
+                  const float* topk_w, const float* probs, const float* dr_part, int n_parts,
                   const float* dx_slots, const float* w_r, float* dlogits, void* dx,
                   void* stream);
+
+/*
+ * probs [T][E] float32 = softmax(x W_r + bias) over all E experts (float32
+ * logits accumulated in a fixed order): what rom_route_bwd needs for r = p.
+ * x, w_r, bias as for rom_route.
+ */
+int rom_route_probs(const void* x, int dtype, int64_t T, int Dm, const float* w_r,
+                    const float* bias, int E, float* probs, void* stream);
+
+/*
+ * Router weight gradients (the router is trained through the Out
+ * projection's routing weights): dw_r [Dm][E] = sum_t x_t^T dlogit_t and
+ * dbias [E] = sum_t dlogit_t (may be NULL), float32, summed over the tokens
+ * in order. x [T][Dm] as given to rom_route (dtype); dlogits [T][E] float32
+ * from rom_route_bwd. With T == 0 both are written as zeros.
+ */
+int rom_route_wgrad(const void* x, int dtype, int64_t T, int Dm, int E, const float* dlogits,
+                    float* dw_r, float* dbias, void* stream);
 
 /*
  * Weight gradients of every expert: out[e] = A_e^T B_e, A_e and B_e the rows

@@ -11,10 +11,13 @@
 //                written as [dH | dZ] rows in expert-sorted order for every
 //                slot of the token (A operand of dX and of dW_in / dW_g).
 //  route_bwd     per token: dr_j = <Y(.)G, g_j> = (sum of the Out dgrad's
-//                partial dots) / r_j; with renormalised top-k weights
-//                r = softmax over the selected logits,
-//                  dlogit_j = r_j (dr_j - sum_i r_i dr_i)   (0 off S_t);
-//                dX_t = sum_j dX_{t,j} + sum_j dlogit_j W_r[:, S_j].
+//                partial dots) / r_j; with s = sum_i r_i dr_i,
+//                  dlogit_j = r_j (dr_j - s) on S_t, and off S_t 0 for
+//                  renormalised weights (r = softmax over the selected
+//                  logits) or -p_m s for r = p (the softmax over all E);
+//                dX_t = sum_j dX_{t,j} + sum_m dlogit_m W_r[:, m].
+//  route_probs   p = softmax over all E experts (float32), for the r = p case.
+//  route_wgrad   dW_r = X^T dlogits and dbias = the column sums of dlogits.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -98,15 +101,19 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // One warp per token; W_r^T slice [E][DS] staged in shared memory.
+// probs == nullptr: renormalised weights (dlogit zero off S_t). Otherwise
+// r = p (the softmax over all E experts, probs [T][E]) and every expert m
+// off S_t gets dlogit_m = -p_m sum_i r_i dr_i, which also enters dX.
 __global__ void __launch_bounds__(kRouteBwdThreads)
     route_bwd_kernel(int64_t T, int k, int E, int Dm, const int32_t* __restrict__ topk_idx,
-                     const float* __restrict__ topk_w, const float* __restrict__ dr_part,
-                     int n_parts, const float* __restrict__ dx_slots,
-                     const float* __restrict__ w_r, float* __restrict__ dlogits,
-                     __nv_bfloat16* __restrict__ dx, int DS) {
+                     const float* __restrict__ topk_w, const float* __restrict__ probs,
+                     const float* __restrict__ dr_part, int n_parts,
+                     const float* __restrict__ dx_slots, const float* __restrict__ w_r,
+                     float* __restrict__ dlogits, __nv_bfloat16* __restrict__ dx, int DS) {
   extern __shared__ float sWt[];  // [E][DS]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = kRouteBwdThreads / 32;
+  __shared__ float s_coef[kRouteBwdThreads / 32][kMaxExperts];  // off-S dlogits (probs given)
   for (int D0 = 0; D0 < Dm; D0 += DS) {
     const int dn = min(DS, Dm - D0);
     __syncthreads();
@@ -143,9 +150,21 @@ __global__ void __launch_bounds__(kRouteBwdThreads)
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j)
         if (j < k) dl[j] = rw[j] * (dr[j] - s);
+      if (probs) {
+        // experts off S_t: dlogit_m = -p_m s (0 for the selected ones here;
+        // theirs are dl[j])
+        for (int e = lane; e < E; e += 32) {
+          bool on = false;
+#pragma unroll
+          for (int j = 0; j < kMaxTopK; ++j)
+            if (j < k && sel[j] == e) on = true;
+          s_coef[warp][e] = on ? 0.f : -probs[t * E + e] * s;
+        }
+        __syncwarp();
+      }
       if (D0 == 0 && dlogits) {
         for (int e = lane; e < E; e += 32) {
-          float v = 0.f;
+          float v = probs ? s_coef[warp][e] : 0.f;
 #pragma unroll
           for (int j = 0; j < kMaxTopK; ++j)
             if (j < k && sel[j] == e) v = dl[j];
@@ -172,9 +191,132 @@ __global__ void __launch_bounds__(kRouteBwdThreads)
             acc.w = fmaf(dl[j], w.w, acc.w);
           }
         }
+        if (probs) {
+          for (int e = 0; e < E; ++e) {
+            const float c = s_coef[warp][e];
+            const float4 w = *reinterpret_cast<const float4*>(sWt + e * DS + d);
+            acc.x = fmaf(c, w.x, acc.x);
+            acc.y = fmaf(c, w.y, acc.y);
+            acc.z = fmaf(c, w.z, acc.z);
+            acc.w = fmaf(c, w.w, acc.w);
+          }
+        }
         *reinterpret_cast<uint2*>(dx + t * Dm + D0 + d) =
             make_uint2(pack2(acc.x, acc.y), pack2(acc.z, acc.w));
       }
+      __syncwarp();  // s_coef is rewritten for the warp's next token
+    }
+  }
+}
+
+template <typename InT>
+__device__ __forceinline__ float to_f(InT v);
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+template <>
+__device__ __forceinline__ float to_f<float>(float v) {
+  return v;
+}
+
+// Softmax over all E experts of every token, float32 (the routing weights'
+// full distribution, which the backward needs when r = p is not
+// renormalised). One warp per token: lanes split d_model and accumulate 16
+// experts at a time in feature order, then a butterfly sum.
+template <typename InT>
+__global__ void __launch_bounds__(256)
+    route_probs_kernel(const InT* __restrict__ x, int64_t T, int Dm, const float* __restrict__ w_r,
+                       const float* __restrict__ bias, int E, float* __restrict__ probs) {
+  __shared__ float s_l[8][kMaxExperts];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t t = blockIdx.x * 8ll + warp; t < T; t += static_cast<int64_t>(gridDim.x) * 8) {
+    for (int e0 = 0; e0 < E; e0 += 16) {
+      float acc[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+      for (int d = lane; d < Dm; d += 32) {
+        const float xv = to_f<InT>(x[t * Dm + d]);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (e0 + q < E) acc[q] = fmaf(xv, __ldg(w_r + static_cast<int64_t>(d) * E + e0 + q), acc[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+      }
+      if (lane == 0)
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (e0 + q < E) s_l[warp][e0 + q] = acc[q] + (bias ? __ldg(bias + e0 + q) : 0.f);
+    }
+    __syncwarp();
+    float m = -INFINITY;
+    for (int e = 0; e < E; ++e) m = fmaxf(m, s_l[warp][e]);
+    float den = 0.f;
+    for (int e = 0; e < E; ++e) den += expf(s_l[warp][e] - m);
+    for (int e = lane; e < E; e += 32) probs[t * E + e] = expf(s_l[warp][e] - m) / den;
+    __syncwarp();
+  }
+}
+
+// Router weight gradients: dW_r[d][e] = sum_t x[t][d] dlogit[t][e] and
+// dbias[e] = sum_t dlogit[t][e], in float32, summed over t in order (the
+// result does not depend on the launch). One CTA per 32 features of d_model;
+// tiles of 64 tokens of x and of the logit gradients pass through shared
+// memory; thread (f, g) accumulates feature f for the experts g, g+8, ...
+constexpr int kRwFeat = 32, kRwTok = 64;
+
+template <typename InT>
+__global__ void __launch_bounds__(256)
+    route_wgrad_kernel(const InT* __restrict__ x, int64_t T, int Dm, int E,
+                       const float* __restrict__ dl, float* __restrict__ dw_r,
+                       float* __restrict__ dbias) {
+  __shared__ float sx[kRwTok][kRwFeat + 1];
+  __shared__ float sdl[kRwTok][kMaxExperts + 1];
+  const int tid = threadIdx.x, f = tid & 31, g = tid >> 5;
+  const int d0 = blockIdx.x * kRwFeat;
+  const bool bias_cta = blockIdx.x == 0 && dbias != nullptr;
+  float acc[kMaxExperts / 8], bacc[kMaxExperts / 8];
+#pragma unroll
+  for (int q = 0; q < kMaxExperts / 8; ++q) acc[q] = bacc[q] = 0.f;
+  for (int64_t t0 = 0; t0 < T; t0 += kRwTok) {
+    const int nt = static_cast<int>(T - t0 < kRwTok ? T - t0 : kRwTok);
+    for (int i = tid; i < kRwTok * kRwFeat; i += 256) {
+      const int r = i / kRwFeat, c = i - r * kRwFeat;
+      sx[r][c] = (r < nt && d0 + c < Dm) ? to_f<InT>(x[(t0 + r) * Dm + d0 + c]) : 0.f;
+    }
+    for (int i = tid; i < kRwTok * E; i += 256) {
+      const int r = i / E, e = i - r * E;
+      sdl[r][e] = r < nt ? dl[(t0 + r) * E + e] : 0.f;
+    }
+    __syncthreads();
+    for (int r = 0; r < nt; ++r) {
+      const float xv = sx[r][f];
+#pragma unroll
+      for (int q = 0; q < kMaxExperts / 8; ++q) {
+        const int e = g + 8 * q;
+        if (e < E) {
+          acc[q] = fmaf(xv, sdl[r][e], acc[q]);
+          if (bias_cta && f == 0) bacc[q] += sdl[r][e];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (d0 + f < Dm) {
+#pragma unroll
+    for (int q = 0; q < kMaxExperts / 8; ++q) {
+      const int e = g + 8 * q;
+      if (e < E) dw_r[static_cast<int64_t>(d0 + f) * E + e] = acc[q];
+    }
+  }
+  if (bias_cta && f == 0) {
+#pragma unroll
+    for (int q = 0; q < kMaxExperts / 8; ++q) {
+      const int e = g + 8 * q;
+      if (e < E) dbias[e] = bacc[q];
     }
   }
 }
@@ -204,10 +346,36 @@ cudaError_t launch_gate_bwd(const float* uz, const float* gp, int64_t T, int k, 
   return cudaGetLastError();
 }
 
+cudaError_t launch_route_wgrad(const void* x, bool bf16, int64_t T, int Dm, int E,
+                               const float* dlogits, float* dw_r, float* dbias,
+                               cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>((Dm + kRwFeat - 1) / kRwFeat);
+  if (bf16)
+    route_wgrad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), T, Dm, E, dlogits, dw_r, dbias);
+  else
+    route_wgrad_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), T, Dm, E,
+                                                         dlogits, dw_r, dbias);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_probs(const void* x, bool bf16, int64_t T, int Dm, const float* w_r,
+                               const float* bias, int E, float* probs, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const unsigned grid = grid_for(T, 8);
+  if (bf16)
+    route_probs_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), T, Dm, w_r, bias, E, probs);
+  else
+    route_probs_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), T, Dm, w_r,
+                                                         bias, E, probs);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route_bwd(int64_t T, int k, int E, int Dm, const int32_t* topk_idx,
-                             const float* topk_w, const float* dr_part, int n_parts,
-                             const float* dx_slots, const float* w_r, float* dlogits, void* dx,
-                             cudaStream_t stream) {
+                             const float* topk_w, const float* probs, const float* dr_part,
+                             int n_parts, const float* dx_slots, const float* w_r, float* dlogits,
+                             void* dx, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   // W_r^T slice: all of d_model when E * Dm floats fit in 160 KB.
   const int ds_max = (160 * 1024 / 4 / E) / 128 * 128;
@@ -218,9 +386,9 @@ cudaError_t launch_route_bwd(int64_t T, int k, int E, int Dm, const int32_t* top
   if (err != cudaSuccess) return err;
   const unsigned grid =
       static_cast<unsigned>(std::min<int64_t>((T + 31) / 32, device_sm_count()));
-  route_bwd_kernel<<<grid, kRouteBwdThreads, smem, stream>>>(T, k, E, Dm, topk_idx, topk_w, dr_part,
-                                                     n_parts, dx_slots, w_r, dlogits,
-                                                     static_cast<__nv_bfloat16*>(dx), DS);
+  route_bwd_kernel<<<grid, kRouteBwdThreads, smem, stream>>>(
+      T, k, E, Dm, topk_idx, topk_w, probs, dr_part, n_parts, dx_slots, w_r, dlogits,
+      static_cast<__nv_bfloat16*>(dx), DS);
   return cudaGetLastError();
 }
 

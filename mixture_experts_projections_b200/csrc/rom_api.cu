@@ -101,7 +101,7 @@ const char* rom_status_string(int status) {
   }
 }
 
-int rom_version(void) { return 1; }
+int rom_version(void) { return 2; }
 
 size_t rom_workspace_size(int64_t T, int E) {
   if (T <= 0 || E <= 0) return 0;
@@ -291,20 +291,31 @@ int rom_bwd_dgrad_in(const void* dhz_sorted, int64_t R, int De, const void* w_in
 }
 
 int rom_route_bwd(int64_t T, int k, int E, int Dm, int renorm, const int32_t* topk_idx,
-                  const float* topk_w, const float* dr_part, int n_parts,
+                  const float* topk_w, const float* probs, const float* dr_part, int n_parts,
                   const float* dx_slots, const float* w_r, float* dlogits, void* dx,
                   void* stream) {
   if (T < 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E || k > rom::kMaxTopK || Dm <= 0 ||
       n_parts < 1 || (renorm != 0 && renorm != 1))
     return ROM_ERR_INVALID_ARG;
-  if (renorm != 1 || Dm % 4 != 0) return ROM_ERR_UNSUPPORTED;
+  if (Dm % 4 != 0) return ROM_ERR_UNSUPPORTED;
   if (T == 0) return ROM_OK;
-  if (!topk_idx || !topk_w || !dr_part || !dx_slots || !w_r || !dx) return ROM_ERR_INVALID_ARG;
+  if (!topk_idx || !topk_w || !dr_part || !dx_slots || !w_r || !dx || (renorm == 0 && !probs))
+    return ROM_ERR_INVALID_ARG;
   if (!aligned16(dx_slots) || !aligned16(w_r) || (reinterpret_cast<uintptr_t>(dx) & 7u))
     return ROM_ERR_UNSUPPORTED;
-  return rom::to_status(rom::launch_route_bwd(T, k, E, Dm, topk_idx, topk_w, dr_part, n_parts,
+  return rom::to_status(rom::launch_route_bwd(T, k, E, Dm, topk_idx, topk_w,
+                                              renorm ? nullptr : probs, dr_part, n_parts,
                                               dx_slots, w_r, dlogits, dx,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+int rom_route_probs(const void* x, int dtype, int64_t T, int Dm, const float* w_r,
+                    const float* bias, int E, float* probs, void* stream) {
+  if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
+  if (T < 0 || Dm <= 0 || E < 1 || E > rom::kMaxExperts) return ROM_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !w_r || !probs)) return ROM_ERR_INVALID_ARG;
+  return rom::to_status(rom::launch_route_probs(x, dtype == ROM_BF16, T, Dm, w_r, bias, E, probs,
+                                                static_cast<cudaStream_t>(stream)));
 }
 
 int rom_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int64_t R, int E,
@@ -322,6 +333,15 @@ int rom_bwd_wgrad(const void* a_sorted, int M, const void* b_sorted, int N, int6
   if (!st) return ROM_ERR_CUDA;
   return rom::to_status(rom::launch_bwd_wgrad(a_sorted, M, b_sorted, N, R, E, offsets, m_split,
                                               out0, out1, st, static_cast<cudaStream_t>(stream)));
+}
+
+int rom_route_wgrad(const void* x, int dtype, int64_t T, int Dm, int E, const float* dlogits,
+                    float* dw_r, float* dbias, void* stream) {
+  if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
+  if (T < 0 || Dm <= 0 || E < 1 || E > rom::kMaxExperts) return ROM_ERR_INVALID_ARG;
+  if (!dw_r || (T > 0 && (!x || !dlogits))) return ROM_ERR_INVALID_ARG;
+  return rom::to_status(rom::launch_route_wgrad(x, dtype == ROM_BF16, T, Dm, E, dlogits, dw_r,
+                                                dbias, static_cast<cudaStream_t>(stream)));
 }
 
 int rom_debug_wait_timeout(uint64_t limit_ns, void* stream) {

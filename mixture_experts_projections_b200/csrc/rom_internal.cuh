@@ -111,9 +111,14 @@ cudaError_t launch_scale_gather(const void* dout, int64_t R, int k, int N,
                                 cudaStream_t stream);
 cudaError_t launch_gate_bwd(const float* uz, const float* gp, int64_t T, int k, int De,
                             const int32_t* slot_pos, void* dhz, cudaStream_t stream);
+cudaError_t launch_route_wgrad(const void* x, bool bf16, int64_t T, int Dm, int E,
+                               const float* dlogits, float* dw_r, float* dbias,
+                               cudaStream_t stream);
+cudaError_t launch_route_probs(const void* x, bool bf16, int64_t T, int Dm, const float* w_r,
+                               const float* bias, int E, float* probs, cudaStream_t stream);
 cudaError_t launch_route_bwd(int64_t T, int k, int E, int Dm, const int32_t* topk_idx,
-                             const float* topk_w, const float* dr_part, int n_parts,
-                             const float* dx_slots, const float* w_r, float* dlogits, void* dx,
-                             cudaStream_t stream);
+                             const float* topk_w, const float* probs, const float* dr_part,
+                             int n_parts, const float* dx_slots, const float* w_r, float* dlogits,
+                             void* dx, cudaStream_t stream);
 
 }  // namespace rom

@@ -45,7 +45,9 @@ SIGNATURES = {
     "rom_bwd_dgrad_out": (_I, [_P, _L, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "rom_bwd_gate": (_I, [_P, _P, _L, _I, _I, _P, _P, _P]),
     "rom_bwd_dgrad_in": (_I, [_P, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P]),
-    "rom_route_bwd": (_I, [_L, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
+    "rom_route_bwd": (_I, [_L, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
+    "rom_route_probs": (_I, [_P, _I, _L, _I, _P, _P, _I, _P, _P]),
+    "rom_route_wgrad": (_I, [_P, _I, _L, _I, _I, _P, _P, _P, _P]),
     "rom_bwd_wgrad": (_I, [_P, _I, _P, _I, _L, _I, _P, _I, _P, _P, _P]),
     "rom_ssm_core_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I]),
     "rom_ssm_core_routed_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I, _I]),
@@ -277,12 +279,12 @@ def core_workspace(T, De, seq_len, core, device, k=1):
 class BlockBuffers:
     """Intermediate and output buffers of one RoM block forward."""
 
-    def __init__(self, T, Dm, De, E, k, dtype, device, core=None, seq_len=None):
+    def __init__(self, T, Dm, De, E, k, dtype, device, core=None, seq_len=None, keep_uz=False):
         R = T * k
         self.routing = RoutingBuffers(T, Dm, E, k, dtype, device)
         self.h_sorted = torch.empty((max(R, 1), De), dtype=dtype, device=device)
         self.uz = (torch.empty((2, R, De), dtype=torch.float32, device=device)
-                   if (k > 1 or core is not None) else None)
+                   if (k > 1 or core is not None or keep_uz) else None)
         self.core_ws = (core_workspace(T, De, seq_len or T, core, device, k)
                         if core is not None else None)
         self.hsum = (torch.empty((T, De), dtype=torch.float32, device=device)
@@ -293,19 +295,23 @@ class BlockBuffers:
 
 
 def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=None, stream=None,
-                  core=None, seq_len=None):
+                  core=None, seq_len=None, keep_uz=False):
     """RoM block forward: route, dispatch, Conv+Gate, (gate combine), Out, (sum).
 
     x [T, Dm] (bf16 or float32), w_r [Dm, E] float32, bias [E] float32 or None,
     w_conv, w_gate [E, De, Dm] and w_out [E, Dm, De] in the library layout.
     ``core`` (CoreParams): the dense core runs between the projections, Y =
     core(H), over sequences of ``seq_len`` tokens (all T if None); without it
-    Y = H. Returns the BlockBuffers holding O (``.out``) and the intermediates.
+    Y = H. ``keep_uz`` (top-1): keep the float32 u and z of every token for a
+    backward (the Conv+Gate projection then writes them and the gate combine
+    forms h, instead of the fused u * SiLU(z) epilogue).
+    Returns the BlockBuffers holding O (``.out``) and the intermediates.
     """
     T, Dm = x.shape
     E, De, _ = w_conv.shape
     if bufs is None:
-        bufs = BlockBuffers(T, Dm, De, E, k, x.dtype, x.device, core, seq_len)
+        bufs = BlockBuffers(T, Dm, De, E, k, x.dtype, x.device, core, seq_len,
+                            keep_uz=keep_uz)
     rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs.routing, stream)
     R = T * k
     xs = rb.x_sorted[:R]
@@ -333,7 +339,16 @@ def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=Non
             rom_combine(ROM_COMBINE_SUM, _dtype_code(x), bufs.o_slots, T, k, Dm, None, bufs.out,
                         stream)
         return bufs
-    if k == 1:
+    if k == 1 and keep_uz:
+        if bufs.uz is None:
+            raise RomError("keep_uz needs BlockBuffers made with keep_uz=True")
+        rom_expert_proj(ROM_PROJ_CONV_GATE_SLOTS, xs, w_conv, w_gate, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, bufs.uz, stream)
+        rom_combine(ROM_COMBINE_GATE, _dtype_code(x), bufs.uz, T, k, De, rb.slot_pos,
+                    bufs.h_sorted, stream)
+        rom_expert_proj(ROM_PROJ_OUT, bufs.h_sorted[:R], w_out, None, E, k, rb.offsets,
+                        rb.sorted_slot, rb.topk_w, bufs.out, stream)
+    elif k == 1:
         rom_expert_proj(ROM_PROJ_CONV_GATE, xs, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
                         rb.topk_w, bufs.h_sorted, stream)
         rom_expert_proj(ROM_PROJ_OUT, bufs.h_sorted[:R], w_out, None, E, k, rb.offsets,
@@ -508,10 +523,25 @@ def rom_bwd_dgrad_in(dhz_sorted, w_in, w_g, E, k, offsets, sorted_slot, dx_slots
 
 
 def rom_route_bwd(T, k, E, Dm, renorm, topk_idx, topk_w, dr_part, dx_slots, w_r, dlogits, dx,
-                  stream=None):
+                  stream=None, probs=None):
     _check(load_library().rom_route_bwd(
-        T, k, E, Dm, int(renorm), _ptr(topk_idx), _ptr(topk_w), _ptr(dr_part), dr_part.shape[1],
-        _ptr(dx_slots), _ptr(w_r), _ptr(dlogits), _ptr(dx), _stream(stream)), "rom_route_bwd")
+        T, k, E, Dm, int(renorm), _ptr(topk_idx), _ptr(topk_w), _ptr(probs), _ptr(dr_part),
+        dr_part.shape[1], _ptr(dx_slots), _ptr(w_r), _ptr(dlogits), _ptr(dx), _stream(stream)),
+        "rom_route_bwd")
+
+
+def rom_route_probs(x, w_r, bias, probs, stream=None):
+    T, Dm = x.shape
+    _check(load_library().rom_route_probs(_ptr(x), _dtype_code(x), T, Dm, _ptr(w_r), _ptr(bias),
+                                          w_r.shape[1], _ptr(probs), _stream(stream)),
+           "rom_route_probs")
+
+
+def rom_route_wgrad(x, dlogits, dw_r, dbias, stream=None):
+    T, Dm = x.shape
+    _check(load_library().rom_route_wgrad(_ptr(x), _dtype_code(x), T, Dm, dlogits.shape[1],
+                                          _ptr(dlogits), _ptr(dw_r), _ptr(dbias),
+                                          _stream(stream)), "rom_route_wgrad")
 
 
 def rom_bwd_wgrad(a_sorted, b_sorted, E, offsets, m_split, out0, out1, stream=None):
@@ -538,22 +568,33 @@ class BackwardBuffers:
         self.dw_out = torch.empty((E, Dm, De), dtype=torch.float32, device=device)
         self.dw_conv = torch.empty((E, De, Dm), dtype=torch.float32, device=device)
         self.dw_gate = torch.empty((E, De, Dm), dtype=torch.float32, device=device)
+        self.dw_r = torch.empty((Dm, E), dtype=torch.float32, device=device)
+        self.dbias = torch.empty((E,), dtype=torch.float32, device=device)
+        self.probs = torch.empty((T, E), dtype=torch.float32, device=device)
 
 
-def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None, stream=None):
-    """Backward of the RoM block for top-k > 1 (renormalised weights).
+def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None, stream=None,
+                   x=None, bias=None):
+    """Backward of the RoM block (renormalised weights, or r = p with ``x``).
 
-    fwd: the BlockBuffers of the forward (routing, h_sorted, u/z slot partials);
-    dout [T, Dm] bf16; weights in the library layout. Returns BackwardBuffers
-    with dx [T, Dm] bf16, dlogits [T, E] and dw_conv / dw_gate [E, De, Dm],
+    fwd: the BlockBuffers of the forward (routing, h_sorted, u/z slot
+    partials: for k == 1 the forward must have run with keep_uz=True);
+    dout [T, Dm] bf16; weights in the library layout. With ``x`` (the
+    forward's input) the router weight gradients dw_r [Dm, E] and dbias [E]
+    are computed too; r = p (renorm=False) needs ``x`` (and the forward's
+    ``bias``) for the softmax over all experts. Returns BackwardBuffers with
+    dx [T, Dm] bf16, dlogits [T, E] and dw_conv / dw_gate [E, De, Dm],
     dw_out [E, Dm, De] (float32, the weights' layout).
     """
     rb = fwd.routing
     T, Dm = dout.shape
     E, De, _ = w_conv.shape
     k = rb.k
-    if k < 2:
-        raise RomError("block_backward needs the forward's per-slot u/z partials (top-k > 1)")
+    if fwd.uz is None:
+        raise RomError("block_backward needs the forward's u/z slot partials "
+                       "(top-k > 1, or block_forward(..., keep_uz=True))")
+    if not renorm and x is None:
+        raise RomError("the backward of r = p needs the forward's input x")
     R = T * k
     if bufs is None:
         bufs = BackwardBuffers(T, Dm, De, E, k, dout.device)
@@ -563,8 +604,12 @@ def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None
     rom_bwd_gate(fwd.uz, bufs.g_slots, T, k, De, rb.slot_pos, bufs.dhz_sorted, stream)
     rom_bwd_dgrad_in(bufs.dhz_sorted, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
                      bufs.dx_slots, stream)
+    if not renorm:
+        rom_route_probs(x, w_r, bias, bufs.probs, stream)
     rom_route_bwd(T, k, E, Dm, renorm, rb.topk_idx, rb.topk_w, bufs.dr_part, bufs.dx_slots, w_r,
-                  bufs.dlogits, bufs.dx, stream)
+                  bufs.dlogits, bufs.dx, stream, probs=None if renorm else bufs.probs)
+    if x is not None:
+        rom_route_wgrad(x, bufs.dlogits, bufs.dw_r, bufs.dbias, stream)
     rom_bwd_wgrad(bufs.rdo_sorted, fwd.h_sorted[:R], E, rb.offsets, Dm, bufs.dw_out, None, stream)
     rom_bwd_wgrad(bufs.dhz_sorted, rb.x_sorted[:R], E, rb.offsets, De, bufs.dw_conv, bufs.dw_gate,
                   stream)

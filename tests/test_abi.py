@@ -44,7 +44,7 @@ def test_status_strings_and_version(lib):
     assert lib.rom_status_string(5) == b"ROM_ERR_TIMEOUT"
     assert lib.rom_status_string(6) == b"ROM_ERR_ROUTING"
     assert lib.rom_status_string(99) == b"ROM_ERR_UNKNOWN"
-    assert lib.rom_version() >= 1
+    assert lib.rom_version() >= 2
 
 
 def test_workspace_size(lib):
@@ -171,14 +171,34 @@ def test_bwd_dgrad_in_rejects_bad_arguments(lib, kw, code):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(n_parts=0), 1), (dict(renorm=2), 1), (dict(renorm=0), 2), (dict(Dm=6), 2),
+    (dict(n_parts=0), 1), (dict(renorm=2), 1), (dict(renorm=0, probs=None), 1), (dict(Dm=6), 2),
     (dict(k=9), 1), (dict(w_r=None), 1), (dict(dx=ctypes.c_void_p((1 << 20) + 2)), 2),
 ])
 def test_route_bwd_rejects_bad_arguments(lib, kw, code):
-    a = dict(T=10, k=2, E=8, Dm=64, renorm=1, topk_idx=FAKE, topk_w=FAKE, dr_part=FAKE,
-             n_parts=1, dx_slots=FAKE, w_r=FAKE, dlogits=FAKE, dx=FAKE, stream=None)
+    a = dict(T=10, k=2, E=8, Dm=64, renorm=1, topk_idx=FAKE, topk_w=FAKE, probs=None,
+             dr_part=FAKE, n_parts=1, dx_slots=FAKE, w_r=FAKE, dlogits=FAKE, dx=FAKE, stream=None)
     a.update(kw)
     assert lib.rom_route_bwd(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=3), 1), (dict(E=0), 1), (dict(E=65), 1), (dict(Dm=0), 1), (dict(x=None), 1),
+    (dict(probs=None), 1),
+])
+def test_route_probs_rejects_bad_arguments(lib, kw, code):
+    a = dict(x=FAKE, dtype=1, T=10, Dm=64, w_r=FAKE, bias=None, E=8, probs=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_route_probs(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=3), 1), (dict(E=0), 1), (dict(T=-1), 1), (dict(dw_r=None), 1),
+    (dict(dlogits=None), 1),
+])
+def test_route_wgrad_rejects_bad_arguments(lib, kw, code):
+    a = dict(x=FAKE, dtype=1, T=10, Dm=64, E=8, dlogits=FAKE, dw_r=FAKE, dbias=None, stream=None)
+    a.update(kw)
+    assert lib.rom_route_wgrad(*a.values()) == code
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -118,3 +118,42 @@ def test_top2_workload_full_size_backward():
                      magnitude_scaled_abs=True)
         assert_close(to_np(bwd.dw_out[e]), dW["dW_out"][e].T, "bf16", f"top2 dW_out[{e}]",
                      magnitude_scaled_abs=True)
+
+
+ROUTER_GRAD_CASES = [
+    # T, Dm, De, E, k, renorm, bias
+    (600, 256, 256, 8, 1, False, None),       # top-1, r = p (the formula of Knowl 1)
+    (500, 256, 256, 8, 2, False, None),       # top-2 without renormalisation
+    (700, 256, 512, 8, 1, True, None),        # top-1 renormalised: r = 1, dlogits = 0
+    (400, 512, 256, 16, 2, True, {3: 0.5}),   # with a router bias
+]
+
+
+@pytest.mark.parametrize("T,Dm,De,E,k,renorm,bias", ROUTER_GRAD_CASES)
+def test_backward_without_renormalisation_and_router_weight_gradients(T, Dm, De, E, k, renorm,
+                                                                      bias):
+    """r = p (no renormalisation) through rom_route_probs and rom_route_bwd,
+    top-1 through the forward that keeps u and z, and the router weight
+    gradients dW_r, dbias (rom_route_wgrad), all against the oracle."""
+    b = None
+    if bias is not None:
+        b = np.zeros(E, np.float32)
+        for e, v in bias.items():
+            b[e] = v
+    inp = make_block_inputs(T, Dm, De, E, seed=11 * T + k, router_std=0.05, bias=b,
+                            with_dout=True)
+    d = block_to_dev(inp, "bf16")
+    fwd = rom.block_forward(d["x"], d["w_r"], d["bias"], d["w_conv"], d["w_gate"], d["w_out"],
+                            k=k, renorm=renorm, keep_uz=True)
+    bwd = rom.block_backward(fwd, to_dev(inp["dout"], "bf16"), d["w_r"], d["w_conv"],
+                             d["w_gate"], d["w_out"], renorm=renorm, x=d["x"], bias=d["bias"])
+    torch.cuda.synchronize()
+    assert rom.rom_get_status() == 0
+    ref = orc.block_backward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                             inp["dout"], k=k, bias=inp["bias"], renorm=renorm)
+    assert np.array_equal(fwd.routing.topk_idx.cpu().numpy(), ref["forward"]["topk_idx"])
+    assert_close(to_np(fwd.out), ref["forward"]["O"], "bf16", "O (kept u, z)",
+                 magnitude_scaled_abs=True)
+    check_grads(bwd, ref)
+    assert_close(to_np(bwd.dw_r), ref["dW_r"], "bf16", "dW_r", magnitude_scaled_abs=True)
+    assert_close(to_np(bwd.dbias), ref["dbias"], "bf16", "dbias", magnitude_scaled_abs=True)
