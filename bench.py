@@ -447,14 +447,23 @@ def build_workload(torch, rom, wl, inp):
             dout = to_dev(torch, inp["dout"], bf16)
             in_bytes += dout.numel() * dout.element_size()
             bwd_bufs = rom.BackwardBuffers(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.device)
+            # Data parallel over ranks: every rank trains on its own tokens and
+            # the weight gradients (experts and router) are summed over all.
+            import torch.distributed as dist
+            dp = dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1
+            grad_sync = rom.GradientAllReduce() if dp else None
 
             def ph_bwd():
                 rom.block_backward(bufs, dout, w_r, ws["w_conv"], ws["w_gate"], ws["w_out"],
-                                   renorm=wl.renorm, bufs=bwd_bufs)
+                                   renorm=wl.renorm, bufs=bwd_bufs, x=x, bias=bias,
+                                   grad_sync=grad_sync)
             phases.append(("backward", ph_bwd))
+            # NCCL collectives are not captured into CUDA graphs here: the
+            # data-parallel step is timed as eager launches
+            res["eager_only"] = dp
         res.update(phases=phases, dominant=(ph_p0, "flop", lambda counts: flops["conv_gate"]),
                    out=bufs.out, counts=rb.counts,
-                   launches=4 + (2 if wl.k > 1 else 0) + (7 if wl.backward else 0))
+                   launches=4 + (2 if wl.k > 1 else 0) + (8 if wl.backward else 0))
         if wl.backward:
             res["e2e"] = None  # host copies around one step (below)
         else:
@@ -503,16 +512,24 @@ def measure(args, wl, world, local_rank, with_e2e):
 
     # The step captured once as one CUDA graph (the library's launch sequence
     # is static: its kernels read the expert counts on the device), and each
-    # phase once more on its own for the per-phase breakdown.
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        step()
-    graphs = []
-    for ph in phases:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            ph()
-        graphs.append(g)
+    # phase once more on its own for the per-phase breakdown. A step with a
+    # collective (data-parallel backward) runs as eager launches instead.
+    class _Eager:
+        def __init__(self, fn):
+            self.replay = fn
+    if b.get("eager_only"):
+        g_step = _Eager(step)
+        graphs = [_Eager(ph) for ph in phases]
+    else:
+        g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            step()
+        graphs = []
+        for ph in phases:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                ph()
+            graphs.append(g)
     torch.cuda.synchronize()
 
     def timed_loop(run_phase, n, count):

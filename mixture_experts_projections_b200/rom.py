@@ -552,6 +552,33 @@ def rom_bwd_wgrad(a_sorted, b_sorted, E, offsets, m_split, out0, out1, stream=No
         _ptr(out1), _stream(stream)), "rom_bwd_wgrad")
 
 
+class GradientAllReduce:
+    """Data-parallel exchange of the weight gradients: every rank holds the
+    gradients of its own tokens, and each tensor handed to ``start`` is summed
+    over the ranks of ``group`` (torch.distributed all-reduce: NCCL over
+    NVLink between GPUs, gloo between CPU processes). A transfer is started
+    as soon as the kernel that produces its tensor is enqueued, so it overlaps
+    the rest of the backward; ``finish`` makes the current stream wait for
+    all of them. Every rank must start the same tensors in the same order.
+    The token batch is split across ranks and the expert and router weights
+    are replicated; the tokens themselves are never exchanged."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.pending = []
+
+    def start(self, *tensors):
+        import torch.distributed as dist
+        for t in tensors:
+            self.pending.append(dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group,
+                                                async_op=True))
+
+    def finish(self):
+        for w in self.pending:
+            w.wait()
+        self.pending = []
+
+
 class BackwardBuffers:
     """Device buffers of one backward pass (allocated by torch)."""
 
@@ -574,7 +601,7 @@ class BackwardBuffers:
 
 
 def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None, stream=None,
-                   x=None, bias=None):
+                   x=None, bias=None, grad_sync=None):
     """Backward of the RoM block (renormalised weights, or r = p with ``x``).
 
     fwd: the BlockBuffers of the forward (routing, h_sorted, u/z slot
@@ -585,6 +612,9 @@ def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None
     ``bias``) for the softmax over all experts. Returns BackwardBuffers with
     dx [T, Dm] bf16, dlogits [T, E] and dw_conv / dw_gate [E, De, Dm],
     dw_out [E, Dm, De] (float32, the weights' layout).
+    ``grad_sync`` (a GradientAllReduce): data-parallel training; the weight
+    gradients are summed over its ranks, dW_out while the rest of the
+    backward runs.
     """
     rb = fwd.routing
     T, Dm = dout.shape
@@ -601,6 +631,11 @@ def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None
     rom_bwd_gather(dout, k, rb.sorted_slot, rb.topk_w, bufs.rdo_sorted, stream)
     rom_bwd_dgrad_out(bufs.rdo_sorted, w_out, E, k, rb.offsets, rb.sorted_slot,
                       fwd.h_sorted[:R], bufs.g_slots, bufs.dr_part, stream)
+    if grad_sync is not None:
+        # dW_out first, so that its exchange overlaps the rest of the backward
+        rom_bwd_wgrad(bufs.rdo_sorted, fwd.h_sorted[:R], E, rb.offsets, Dm, bufs.dw_out, None,
+                      stream)
+        grad_sync.start(bufs.dw_out)
     rom_bwd_gate(fwd.uz, bufs.g_slots, T, k, De, rb.slot_pos, bufs.dhz_sorted, stream)
     rom_bwd_dgrad_in(bufs.dhz_sorted, w_conv, w_gate, E, k, rb.offsets, rb.sorted_slot,
                      bufs.dx_slots, stream)
@@ -610,9 +645,16 @@ def block_backward(fwd, dout, w_r, w_conv, w_gate, w_out, renorm=True, bufs=None
                   bufs.dlogits, bufs.dx, stream, probs=None if renorm else bufs.probs)
     if x is not None:
         rom_route_wgrad(x, bufs.dlogits, bufs.dw_r, bufs.dbias, stream)
-    rom_bwd_wgrad(bufs.rdo_sorted, fwd.h_sorted[:R], E, rb.offsets, Dm, bufs.dw_out, None, stream)
+        if grad_sync is not None:
+            grad_sync.start(bufs.dw_r, bufs.dbias)
+    if grad_sync is None:
+        rom_bwd_wgrad(bufs.rdo_sorted, fwd.h_sorted[:R], E, rb.offsets, Dm, bufs.dw_out, None,
+                      stream)
     rom_bwd_wgrad(bufs.dhz_sorted, rb.x_sorted[:R], E, rb.offsets, De, bufs.dw_conv, bufs.dw_gate,
                   stream)
+    if grad_sync is not None:
+        grad_sync.start(bufs.dw_conv, bufs.dw_gate)
+        grad_sync.finish()
     return bufs
 
 

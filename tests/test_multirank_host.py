@@ -88,3 +88,43 @@ def test_metric_names_the_block_and_the_gpu_count():
     assert r.returncode == 0, r.stderr
     line = json.loads([ln for ln in r.stdout.splitlines() if ln.strip()][0])
     assert line["metric"] == "tokens/s and TFLOPS (% bf16 peak) for RoM projection block fwd, 1 B200"
+
+
+def _grad_rank_main(rank, world, port):
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    from mixture_experts_projections_b200 import rom
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # per-rank gradients of different shapes, started in the backward's
+        # order (dW_out first, the router's next, Conv / Gate last)
+        g = {n: torch.full(shape, float(rank + 1)) * (i + 1)
+             for i, (n, shape) in enumerate([("dw_out", (3, 4, 5)), ("dw_r", (4, 2)),
+                                             ("dbias", (2,)), ("dw_conv", (3, 5, 4)),
+                                             ("dw_gate", (3, 5, 4))])}
+        sync = rom.GradientAllReduce()
+        sync.start(g["dw_out"])
+        sync.start(g["dw_r"], g["dbias"])
+        sync.start(g["dw_conv"], g["dw_gate"])
+        sync.finish()
+        assert sync.pending == []
+        total = sum(r + 1 for r in range(world))
+        for i, n in enumerate(["dw_out", "dw_r", "dbias", "dw_conv", "dw_gate"]):
+            assert torch.all(g[n] == total * (i + 1)), (rank, n)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_gradients_are_summed_over_two_gloo_ranks():
+    """The data-parallel gradient exchange of the backward (GradientAllReduce,
+    which rom.block_backward drives with grad_sync): every rank ends with the
+    sum of all ranks' gradients, in the order they were started."""
+    world = 2
+    mp.start_processes(_grad_rank_main, args=(world, _free_port()), nprocs=world,
+                       start_method="spawn", join=True)
