@@ -62,9 +62,6 @@ struct Params {
   int k;
   int n_tiles_n;
   int* status;
-  // swap-AB kernel: the weight stack [E][N][K], for the L2 prefetch it
-  // issues before the routing it depends on is complete (may be null)
-  const void* w_prefetch;
 };
 
 // u * SiLU(z) = u * z / (1 + e^-z), with the fast exp and divide intrinsics:
@@ -484,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Set-up that needs no routing: barriers, TMEM, tensor maps. The kernel is
   // launched as a programmatic dependent of the dispatch, so this overlaps
-  // the router and the dispatch.
+  // the router and the dispatch. (An L2 prefetch of each CTA's first weight
+  // tile here measured no gain on the decode step: 79.9 us either way.)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW_STAGES; ++s) {
       mbar_init(&ctl.full[s], 1);
@@ -505,24 +503,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(&ctl.tmem_base, SW_TMEM_COLS);
     tmem_relinquish();
-  }
-  if (warp == 2 && p.w_prefetch) {
-    // The expert weights do not depend on the routing: bring this CTA's first
-    // weight tile into L2 while the routing is still being computed, taking
-    // the tile order that holds when every expert has one token tile (at
-    // most 64 rows each; a decode batch). If the routing turns out otherwise
-    // the prefetched lines are only unused.
-    const int tile = blockIdx.x;
-    if (tile < E * n_wt) {
-      const int e = tile / n_wt, w_blk = tile - (tile / n_wt) * n_wt;
-      const uint8_t* base = static_cast<const uint8_t*>(p.w_prefetch) +
-                            (static_cast<int64_t>(e) * p.N + static_cast<int64_t>(w_blk) * SW_BM) *
-                                p.K * 2;
-      const uint32_t bytes = static_cast<uint32_t>(SW_BM) * static_cast<uint32_t>(p.K) * 2u;
-      constexpr uint32_t kChunk = 16384;
-      for (uint32_t off = static_cast<uint32_t>(lane) * kChunk; off < bytes; off += 32 * kChunk)
-        bulk_prefetch_l2(base + off, bytes - off < kChunk ? bytes - off : kChunk);
-    }
   }
   pdl_wait();  // the routing (offsets, sorted rows, weights) is complete from here
   for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = offset_of(p, i);
@@ -776,7 +756,6 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
     p.E = E;
     p.k = k;
     p.status = status;
-    p.w_prefetch = w0;
     // Upper bound of the tile count (the exact count depends on the routing,
     // read on the device); every CTA gets ceil(tiles / SMs) tiles.
     const int64_t max_tiles = ((R + SW_BN - 1) / SW_BN + E) * static_cast<int64_t>(N / SW_BM);
@@ -790,7 +769,7 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(kSwapSmemBytes));
     if (err != cudaSuccess) return err;
-    // Programmatic dependent launch: the set-up and the weight prefetch run
+    // Programmatic dependent launch: the set-up runs
     // while the kernel before (the dispatch) finishes.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

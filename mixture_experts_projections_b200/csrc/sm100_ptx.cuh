@@ -120,14 +120,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Hint: bring `bytes` (multiple of 16, 16-byte aligned address) of global
-// memory into L2 without waiting for it.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-               "r"(bytes)
-               : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 // Allocates ncols TMEM columns (power of two >= 32); the base address is

@@ -11,15 +11,17 @@
 //
 // Kernels, in order (all on the caller's stream, no host synchronisation):
 //  1. conv_silu_kernel: causal depthwise convolution (K taps, restart at
-//     every sequence) + bias + SiLU, bf16 X (the A operand of the next GEMM).
+//     every sequence) + bias + SiLU, bf16 X (the A operand of the next GEMM);
+//     one thread per channel walks a chunk of time steps.
 //  2. the x projection, X [T][De] x W_x -> float32 [T][Np] (the tensor-core
 //     grouped GEMM with one expert; W_x stored [Np][De], rows past R + 2N
 //     zero).
 //  3. dt_cast_kernel: the dt columns to bf16 [T][R].
 //  4. the dt projection, dt [T][R] x W_dt -> float32 [T][De] (same GEMM).
 //  5. the scan in chunks of kChunk steps, parallel over channels and chunks:
-//     scan_kernel<false> runs each chunk from a zero state and keeps its final
-//     state and sum of delta; scan_carry_kernel chains the chunks of each
+//     scan_kernel<false> turns dt W_dt into delta = softplus(. + b_dt) in
+//     place and runs each chunk from a zero state, keeping its final state
+//     and sum of delta; scan_carry_kernel chains the chunks of each
 //     sequence (the state entering chunk c+1 is exp(A sum_c delta) times the
 //     state entering chunk c plus chunk c's own final state); scan_kernel<true>
 //     runs every chunk again from its entering state and writes y.
@@ -48,36 +50,52 @@ constexpr int kChunk = 128;        // time steps per scan chunk
 constexpr int kScanThreads = 128;  // channels per scan CTA
 constexpr float kLog2e = 1.4426950408889634f;
 
-__global__ void __launch_bounds__(256)
+// One thread per channel and a chunk of kConvSteps time steps (a CTA holds
+// 128 consecutive channels, so every load and store of a step is one row
+// segment); the K - 1 previous inputs stay in registers, so each input is
+// read once (plus K - 1 at the chunk's start).
+constexpr int kConvSteps = 64;
+
+__global__ void __launch_bounds__(128)
     conv_silu_kernel(const float* __restrict__ h, int64_t T, int De, int L,
                      const float* __restrict__ w, const float* __restrict__ b, int K,
                      __nv_bfloat16* __restrict__ x) {
-  const int nq = De / 4;
-  const int64_t total = T * nq;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / nq;
-    const int d = static_cast<int>(i - t * nq) * 4;
-    const int64_t seq0 = (t / L) * L;  // the convolution restarts at every sequence
-    float acc[4];
+  const int d = blockIdx.x * 128 + threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kConvSteps;
+  if (d >= De) return;
+  float tap[kMaxTaps], win[kMaxTaps];  // win[j] = h_{t-1-j} (0 before the sequence)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[q] = __ldg(b + d + q);
-    // tap K-1 multiplies the current step, tap K-1-j the step j back
-    for (int j = 0; j < K && t - j >= seq0; ++j) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(h + (t - j) * De + d));
-      const float vv[4] = {v.x, v.y, v.z, v.w};
+  for (int j = 0; j < kMaxTaps; ++j) {
+    tap[j] = j < K ? __ldg(w + static_cast<int64_t>(d) * K + j) : 0.f;
+    win[j] = 0.f;
+  }
+  const float bias = __ldg(b + d);
+  int64_t seq0 = (t0 / L) * L;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] = fmaf(__ldg(w + (d + q) * K + (K - 1 - j)), vv[q], acc[q]);
+  for (int j = 0; j < kMaxTaps - 1; ++j)
+    if (j < K - 1 && t0 - 1 - j >= seq0) win[j] = __ldg(h + (t0 - 1 - j) * De + d);
+  const int n = static_cast<int>(T - t0 < kConvSteps ? T - t0 : kConvSteps);
+  int64_t next_seq = seq0 + L;  // the window restarts where the next sequence begins
+  const float* hp = h + t0 * De + d;
+  __nv_bfloat16* xp = x + t0 * De + d;
+  for (int s = 0; s < n; ++s) {
+    if (t0 + s == next_seq) {
+#pragma unroll
+      for (int j = 0; j < kMaxTaps; ++j) win[j] = 0.f;
+      next_seq += L;
     }
-    float s[4];
+    const float cur = __ldg(hp + static_cast<int64_t>(s) * De);
+    // tap K-1 multiplies the current step, tap K-1-j the step j back
+    float acc = fmaf(tap[K - 1], cur, bias);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) s[q] = acc[q] / (1.0f + expf(-acc[q]));
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(s[0], s[1]);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(s[2], s[3]);
-    uint2 o;
-    o.x = *reinterpret_cast<const uint32_t*>(&lo);
-    o.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(x + t * De + d) = o;
+    for (int j = 1; j < kMaxTaps; ++j)
+      if (j < K) acc = fmaf(tap[K - 1 - j], win[j - 1], acc);
+#pragma unroll
+    for (int j = kMaxTaps - 1; j > 0; --j) win[j] = win[j - 1];
+    win[0] = cur;
+    // SiLU with the fast exp and divide (their error is far below the bf16
+    // rounding of X; for acc < -88 the quotient is SiLU's limit 0)
+    xp[static_cast<int64_t>(s) * De] = __float2bfloat16_rn(__fdividef(acc, 1.0f + __expf(-acc)));
   }
 }
 
@@ -109,12 +127,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// softplus(v) = ln(1 + e^v); for v > 20 it equals v in float32.
-__device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(expf(v)); }
+// softplus(v) = ln(1 + e^v), accurate for small results (delta is often
+// ~1e-3); for v > 20 it equals v in float32.
+__device__ __forceinline__ float softplus_f(float v) {
+  return v > 20.f ? v : log1pf(__expf(v));
+}
+
+// 2^v on the special-function unit (relative error ~2^-22; inputs here are
+// <= 0, results underflow to 0 for v < -126).
+__device__ __forceinline__ float ex2_approx(float v) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
 
 struct ScanArgs {
   const __nv_bfloat16* x;  // [T][De]
-  const float* dpre;       // [T][De]: dt W_dt (before the bias and softplus)
+  float* delta;            // [T][De]: dt W_dt on entry; delta = softplus(. + b_dt) after pass 1
   const float* b_dt;       // [De]
   const float* dbc;        // [T][Np]: dt | B | C | zero padding
   const float* a_log;      // [De][N]
@@ -127,20 +156,29 @@ struct ScanArgs {
   int De, L, nc, Np, R, N;
 };
 
-// One chunk of one sequence for 128 channels. kOut = false: from a zero
-// state, record the final state and the sum of delta (the chunk's own part
-// of the recurrence); kOut = true: from the chunk's entering state, write y.
+// One chunk of one sequence for 128 channels.
+// kOut = false: delta = softplus(dt W_dt + b_dt) written over its input, then
+//   (except for a sequence's last chunk, which feeds nothing) the chunk's
+//   own recurrence from a zero state: its final state and sum of delta.
+// kOut = true: the recurrence again from the chunk's entering state, y out.
+// Each step's delta and x are loaded one step ahead of their use.
 template <bool kOut>
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
   __shared__ float sB[kChunk][kMaxState];
   __shared__ float sC[kOut ? kChunk : 1][kMaxState];
   const int cg = blockIdx.y;  // chunk over all sequences
   const int seq = cg / a.nc, c = cg - (cg / a.nc) * a.nc;
-  if (!kOut && c == a.nc - 1) return;  // a sequence's last chunk feeds nothing
+  const bool last = c == a.nc - 1;
   const int d = blockIdx.x * kScanThreads + threadIdx.x;
   const int64_t t0 = static_cast<int64_t>(seq) * a.L + static_cast<int64_t>(c) * kChunk;
   const int len = min(kChunk, a.L - c * kChunk);
   const int N = a.N;
+  float* dp = a.delta + t0 * a.De + d;
+  if (!kOut && last) {
+    const float bd = __ldg(a.b_dt + d);
+    for (int s = 0; s < len; ++s) dp[s * a.De] = softplus_f(dp[s * a.De] + bd);
+    return;
+  }
   for (int i = threadIdx.x; i < len * N; i += kScanThreads) {
     const int s = i / N, n = i - (i / N) * N;
     const float* row = a.dbc + (t0 + s) * a.Np + a.R;
@@ -154,24 +192,35 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
     A2[n] = n < N ? -expf(__ldg(a.a_log + static_cast<int64_t>(d) * N + n)) * kLog2e : 0.f;
     h[n] = (kOut && n < N) ? a.carry[(static_cast<int64_t>(cg) * N + n) * a.De + d] : 0.f;
   }
-  const float bd = __ldg(a.b_dt + d);
+  const float bd = kOut ? 0.f : __ldg(a.b_dt + d);
   const float Dd = kOut ? __ldg(a.d + d) : 0.f;
+  const __nv_bfloat16* xp = a.x + t0 * a.De + d;
+  float* yp = kOut ? a.y + t0 * a.De + d : nullptr;
   float ssum = 0.f;
+  float pre_next = dp[0];
+  float x_next = __bfloat162float(xp[0]);
   for (int s = 0; s < len; ++s) {
-    const int64_t idx = (t0 + s) * a.De + d;
-    const float delta = softplus_f(__ldg(a.dpre + idx) + bd);
-    const float xv = __bfloat162float(a.x[idx]);
+    const float pre = pre_next, xv = x_next;
+    if (s + 1 < len) {
+      pre_next = dp[(s + 1) * a.De];
+      x_next = __bfloat162float(xp[(s + 1) * a.De]);
+    }
+    float delta = pre;
+    if (!kOut) {
+      delta = softplus_f(pre + bd);
+      dp[s * a.De] = delta;
+    }
     const float dx = delta * xv;
     ssum += delta;
     float yv = 0.f;
 #pragma unroll
     for (int n = 0; n < kMaxState; ++n) {
       if (n < N) {
-        h[n] = fmaf(exp2f(delta * A2[n]), h[n], dx * sB[s][n]);
+        h[n] = fmaf(ex2_approx(delta * A2[n]), h[n], dx * sB[s][n]);
         if (kOut) yv = fmaf(h[n], sC[s][n], yv);
       }
     }
-    if (kOut) a.y[idx] = fmaf(Dd, xv, yv);
+    if (kOut) yp[s * a.De] = fmaf(Dd, xv, yv);
   }
   if (!kOut) {
     a.S[static_cast<int64_t>(cg) * a.De + d] = ssum;
@@ -196,7 +245,7 @@ __global__ void __launch_bounds__(256) scan_carry_kernel(const ScanArgs a, int n
       const int64_t cg = static_cast<int64_t>(seq) * a.nc + c;
       a.carry[(cg * a.N + n) * a.De + d] = cin;
       if (c + 1 < a.nc)
-        cin = fmaf(exp2f(a.S[cg * a.De + d] * A2), cin, a.hend[(cg * a.N + n) * a.De + d]);
+        cin = fmaf(ex2_approx(a.S[cg * a.De + d] * A2), cin, a.hend[(cg * a.N + n) * a.De + d]);
     }
   }
 }
@@ -296,8 +345,9 @@ cudaError_t launch_ssm_core(const float* h, int64_t T, int De, int seq_len, cons
                             cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const CoreWs w = core_ws_layout(ws, T, De, seq_len, R, N, Np, k);
-  conv_silu_kernel<<<grid_for(T * (De / 4), 256), 256, 0, stream>>>(h, T, De, seq_len, conv_w,
-                                                                     conv_b, K, w.x);
+  conv_silu_kernel<<<dim3(static_cast<unsigned>(De / 128),
+                         static_cast<unsigned>((T + kConvSteps - 1) / kConvSteps)),
+                    128, 0, stream>>>(h, T, De, seq_len, conv_w, conv_b, K, w.x);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // x projection to [dt | B | C | 0] float32 rows, token order
@@ -312,7 +362,7 @@ cudaError_t launch_ssm_core(const float* h, int64_t T, int De, int seq_len, cons
   if (e != cudaSuccess) return e;
   ScanArgs a;
   a.x = w.x;
-  a.dpre = w.dpre;
+  a.delta = w.dpre;
   a.b_dt = b_dt;
   a.dbc = w.dbc;
   a.a_log = a_log;

@@ -51,7 +51,7 @@ SIGNATURES = {
     "rom_bwd_wgrad": (_I, [_P, _I, _P, _I, _L, _I, _P, _I, _P, _P, _P]),
     "rom_ssm_core_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I]),
     "rom_ssm_core_routed_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I, _I]),
-    "rom_ssm_core_routed": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P,
+    "rom_ssm_core_routed": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P,
                                  _I, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "rom_ssm_core": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                           ctypes.c_size_t, _P]),

@@ -223,3 +223,22 @@ def test_route_dispatch_noalloc_rejects_bad_arguments(lib, kw, code):
              slot_pos=FAKE, x_sorted=FAKE, stream=None)
     a.update(kw)
     assert lib.rom_route_dispatch_noalloc(*a.values()) == code
+
+
+def _declared_arity():
+    """Number of parameters of every function declared in include/rom.h."""
+    text = open(os.path.join(ROOT, "include", "rom.h")).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"(?:int|size_t|const char\*)\s+(rom_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_the_header_arity():
+    from mixture_experts_projections_b200 import rom
+    arity = _declared_arity()
+    assert arity, "no declarations parsed"
+    for name, n in arity.items():
+        assert len(rom.SIGNATURES[name][1]) == n, (name, len(rom.SIGNATURES[name][1]), n)
