@@ -341,6 +341,25 @@ def test_oracle_regression_fixture():
     path = os.path.join(os.path.dirname(__file__), "golden", "oracle_regression.json")
     cases = json.load(open(path))["cases"]
     for name, c in cases.items():
+        if name.startswith("independent"):
+            inp = make_block_inputs(c["T"], c["Dm"], c["De"], c["E"], seed=c["seed"],
+                                    router_std=c["router_std"], extra_routers=True)
+            v = orc.variant_block_forward(inp["x"], inp["w_conv"], inp["w_gate"], inp["w_out"],
+                                          c["k"], {"conv": inp["w_r"], "gate": inp["w_r_gate"],
+                                                   "out": inp["w_r_out"]},
+                                          {"conv": True, "gate": True, "out": True})
+            np.testing.assert_allclose(v["O"], c["O"], rtol=1e-12, atol=1e-14)
+            continue
+        if name.startswith("core"):
+            from mixture_experts_projections_b200.inputs import make_core_params
+            inp = make_block_inputs(c["T"], c["Dm"], c["De"], c["E"], seed=c["seed"],
+                                    router_std=c["router_std"])
+            core = make_core_params(c["De"], c["Dm"], seed=c["seed"], N=c["N"], K=c["K"])
+            r = orc.block_forward(inp["x"], inp["w_r"], inp["w_conv"], inp["w_gate"],
+                                  inp["w_out"], c["k"], core=core, seq_len=c["seq_len"])
+            np.testing.assert_allclose(r["O"], c["O"], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(r["Y"], c["Y"], rtol=1e-12, atol=1e-14)
+            continue
         if name.startswith("inproj"):
             inp = make_inproj_inputs(c["T"], c["Dm"], c["N"], c["E"], seed=c["seed"],
                                      router_std=c["router_std"])
