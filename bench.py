@@ -638,12 +638,32 @@ def workload_config(wl, world):
             **({"projections": wl.variant} if wl.kind == "variant" else {})}
 
 
+SM_COUNT = 148
+SFU_PER_SM_CLK = 16  # special-function results (exp2, log2, ...) per SM per clock
+
+
+def core_roofline(res, wl):
+    """The core's state updates (one exp(delta A) per token, channel and
+    state: T * d_inner * N) per second over the whole core phase (the
+    convolution, the x and dt projections and the scan), against the
+    special-function unit's exp2 rate: 148 SMs x 16 results per clock x the
+    highest SM clock seen."""
+    from mixture_experts_projections_b200.inputs import CORE_STATE
+    t_s = res["part_ms"]["core"] / 1e3
+    mhz = res["clocks"].get("sm_max_mhz") or 1965.0
+    peak = SM_COUNT * SFU_PER_SM_CLK * mhz * 1e6 / 1e9
+    ach = wl.T * wl.De * CORE_STATE / t_s / 1e9
+    return {"bound": "alu", "unit": "G exp2/s", "achieved": ach, "peak": peak,
+            "frac": ach / peak, "kernel": "rom_ssm_core (whole phase)"}
+
+
 def summary_entry(res, peaks, src, world):
     """Per-workload figures of the extra workloads of one bench run."""
     wl = res["wl"]
     tot = sum(block_flops(wl).values())
     step_s = res["step_ms"] / 1e3
-    return {"config": workload_config(wl, world), "l2": res["l2"],
+    extra = {"core_roofline": core_roofline(res, wl)} if wl.core else {}
+    return {**extra, "config": workload_config(wl, world), "l2": res["l2"],
             "step": "forward + backward" if wl.backward else "forward",
             "ms_per_step": res["step_ms"], "tokens_per_s": job_tokens_per_s(wl.T, world,
                                                                             res["step_ms"]),

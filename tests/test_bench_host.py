@@ -57,3 +57,13 @@ def test_clock_summary_skips_lines_that_do_not_parse():
     assert s["samples"] == 1 and s["sm_mhz"] == 1965.0
     empty = bench.summarize_clocks([])
     assert empty["sm_mhz"] is None and empty["sm_max_mhz"] is None and empty["samples"] == 0
+
+
+def test_core_roofline_counts_one_exp_per_state_update():
+    wl = WORKLOADS["prefill_16k_core"]
+    res = {"part_ms": {"core": 1.0}, "clocks": {"sm_max_mhz": 1965.0}}
+    r = bench.core_roofline(res, wl)
+    # 16384 tokens x 4096 channels x 16 states in 1 ms
+    assert r["achieved"] == pytest.approx(16384 * 4096 * 16 / 1e-3 / 1e9)
+    assert r["peak"] == pytest.approx(148 * 16 * 1965e6 / 1e9)
+    assert r["bound"] == "alu" and 0 < r["frac"] < 1
