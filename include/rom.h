@@ -336,8 +336,10 @@ size_t rom_ssm_core_workspace_size(int64_t T, int De, int seq_len, int R, int N,
  *  b_dt    [De], a_log [De][N] (N <= 16), d [De]: float32
  *  y       [T][De] float32 out; may be the same buffer as h
  *  ws      workspace of rom_ssm_core_workspace_size() bytes, 256-byte aligned
- * X and dt are rounded to bf16 for the two projections (tensor cores); the
- * convolution, softplus and the scan run in float32. Requires De % 128 == 0.
+ * The two projections run on the bf16 tensor cores with X and dt split into
+ * two bf16 parts each (hi + lo, so the products are accurate to ~2^-16);
+ * the convolution, softplus and the scan run in float32. Requires
+ * De % 128 == 0.
  */
 int rom_ssm_core(const float* h, int64_t T, int De, int seq_len, const float* conv_w,
                  const float* conv_b, int K, const void* w_x, int R, int N, int Np,
@@ -346,7 +348,7 @@ int rom_ssm_core(const float* h, int64_t T, int De, int seq_len, const float* co
 
 /* Bytes of workspace rom_ssm_core_routed needs (0 for invalid sizes). */
 size_t rom_ssm_core_routed_workspace_size(int64_t T, int De, int seq_len, int R, int N, int Np,
-                                          int k);
+                                          int E, int k);
 
 /*
  * rom_ssm_core_routed -- rom_ssm_core with the x and dt projections

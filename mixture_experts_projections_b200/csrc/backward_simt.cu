@@ -18,12 +18,15 @@
 //                dX_t = sum_j dX_{t,j} + sum_m dlogit_m W_r[:, m].
 //  route_probs   p = softmax over all E experts (float32), for the r = p case.
 //  route_wgrad   dW_r = X^T dlogits and dbias = the column sums of dlogits.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <math.h>
 
 #include <algorithm>
 
 #include "rom_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace rom {
 namespace {
@@ -262,30 +265,46 @@ __global__ void __launch_bounds__(256)
 }
 
 // Router weight gradients: dW_r[d][e] = sum_t x[t][d] dlogit[t][e] and
-// dbias[e] = sum_t dlogit[t][e], in float32, summed over t in order (the
-// result does not depend on the launch). One CTA per 32 features of d_model;
-// tiles of 64 tokens of x and of the logit gradients pass through shared
-// memory; thread (f, g) accumulates feature f for the experts g, g+8, ...
-constexpr int kRwFeat = 32, kRwTok = 64;
+// dbias[e] = sum_t dlogit[t][e], in float32. A cluster of kRwSplit CTAs owns
+// 64 features of d_model; CTA r of the cluster sums the tokens of its slice
+// r of T (tiles of 64 tokens of x and of the logit gradients through shared
+// memory, thread (f, g) accumulating feature f for the experts g, g+4, ...),
+// then CTA 0 adds the kRwSplit partial sums in rank order through
+// distributed shared memory. The order of every sum is fixed, so the result
+// does not depend on the launch.
+constexpr int kRwFeat = 64, kRwTok = 64, kRwSplit = 8;
 
-template <typename InT>
 __global__ void __launch_bounds__(256)
-    route_wgrad_kernel(const InT* __restrict__ x, int64_t T, int Dm, int E,
+    route_wgrad_kernel(const void* __restrict__ xv, bool bf16, int64_t T, int Dm, int E,
                        const float* __restrict__ dl, float* __restrict__ dw_r,
                        float* __restrict__ dbias) {
-  __shared__ float sx[kRwTok][kRwFeat + 1];
+  static_assert(kRwTok == kRwFeat && kRwFeat >= kMaxExperts, "partials reuse the x tile");
+  __shared__ float sx[kRwTok][kRwFeat + 1];  // the x tile; after the loop the partial sums
   __shared__ float sdl[kRwTok][kMaxExperts + 1];
-  const int tid = threadIdx.x, f = tid & 31, g = tid >> 5;
-  const int d0 = blockIdx.x * kRwFeat;
-  const bool bias_cta = blockIdx.x == 0 && dbias != nullptr;
-  float acc[kMaxExperts / 8], bacc[kMaxExperts / 8];
+  __shared__ float s_bias[kMaxExperts];
+  float(*s_part)[kRwFeat + 1] = sx;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int tid = threadIdx.x, f = tid & 63, g = tid >> 6;  // g in 0..3
+  const int d0 = (blockIdx.x / kRwSplit) * kRwFeat;
+  const bool bias_cluster = blockIdx.x / kRwSplit == 0 && dbias != nullptr;
+  const int64_t per = (T + kRwSplit - 1) / kRwSplit;
+  const int64_t ta = rank * per, tb = ta + per < T ? ta + per : T;
+  constexpr int Q = kMaxExperts / 4;
+  float acc[Q], bacc[Q];
 #pragma unroll
-  for (int q = 0; q < kMaxExperts / 8; ++q) acc[q] = bacc[q] = 0.f;
-  for (int64_t t0 = 0; t0 < T; t0 += kRwTok) {
-    const int nt = static_cast<int>(T - t0 < kRwTok ? T - t0 : kRwTok);
+  for (int q = 0; q < Q; ++q) acc[q] = bacc[q] = 0.f;
+  for (int64_t t0 = ta; t0 < tb; t0 += kRwTok) {
+    const int nt = static_cast<int>(tb - t0 < kRwTok ? tb - t0 : kRwTok);
     for (int i = tid; i < kRwTok * kRwFeat; i += 256) {
       const int r = i / kRwFeat, c = i - r * kRwFeat;
-      sx[r][c] = (r < nt && d0 + c < Dm) ? to_f<InT>(x[(t0 + r) * Dm + d0 + c]) : 0.f;
+      float v = 0.f;
+      if (r < nt && d0 + c < Dm) {
+        const int64_t at = (t0 + r) * Dm + d0 + c;
+        v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(xv)[at])
+                 : static_cast<const float*>(xv)[at];
+      }
+      sx[r][c] = v;
     }
     for (int i = tid; i < kRwTok * E; i += 256) {
       const int r = i / E, e = i - r * E;
@@ -293,32 +312,42 @@ __global__ void __launch_bounds__(256)
     }
     __syncthreads();
     for (int r = 0; r < nt; ++r) {
-      const float xv = sx[r][f];
+      const float x = sx[r][f];
 #pragma unroll
-      for (int q = 0; q < kMaxExperts / 8; ++q) {
-        const int e = g + 8 * q;
+      for (int q = 0; q < Q; ++q) {
+        const int e = g + 4 * q;
         if (e < E) {
-          acc[q] = fmaf(xv, sdl[r][e], acc[q]);
-          if (bias_cta && f == 0) bacc[q] += sdl[r][e];
+          acc[q] = fmaf(x, sdl[r][e], acc[q]);
+          if (bias_cluster && f == 0) bacc[q] += sdl[r][e];
         }
       }
     }
     __syncthreads();
   }
-  if (d0 + f < Dm) {
 #pragma unroll
-    for (int q = 0; q < kMaxExperts / 8; ++q) {
-      const int e = g + 8 * q;
-      if (e < E) dw_r[static_cast<int64_t>(d0 + f) * E + e] = acc[q];
+  for (int q = 0; q < Q; ++q) {
+    const int e = g + 4 * q;
+    if (e < E) {
+      s_part[f][e] = acc[q];
+      if (f == 0) s_bias[e] = bacc[q];
     }
   }
-  if (bias_cta && f == 0) {
-#pragma unroll
-    for (int q = 0; q < kMaxExperts / 8; ++q) {
-      const int e = g + 8 * q;
-      if (e < E) dbias[e] = bacc[q];
+  cluster.sync();  // every CTA's partial sums are in its shared memory
+  if (rank == 0) {
+    for (int i = tid; i < kRwFeat * E; i += 256) {
+      const int ff = i / E, e = i - ff * E;
+      float v = 0.f;
+      for (int rr = 0; rr < kRwSplit; ++rr) v += cluster.map_shared_rank(&s_part[ff][e], rr)[0];
+      if (d0 + ff < Dm) dw_r[static_cast<int64_t>(d0 + ff) * E + e] = v;
     }
+    if (bias_cluster)
+      for (int e = tid; e < E; e += 256) {
+        float v = 0.f;
+        for (int rr = 0; rr < kRwSplit; ++rr) v += cluster.map_shared_rank(&s_bias[e], rr)[0];
+        dbias[e] = v;
+      }
   }
+  cluster.sync();  // no CTA exits while CTA 0 still reads its shared memory
 }
 
 unsigned grid_for(int64_t work_items, int per_block) {
@@ -349,14 +378,19 @@ cudaError_t launch_gate_bwd(const float* uz, const float* gp, int64_t T, int k, 
 cudaError_t launch_route_wgrad(const void* x, bool bf16, int64_t T, int Dm, int E,
                                const float* dlogits, float* dw_r, float* dbias,
                                cudaStream_t stream) {
-  const unsigned grid = static_cast<unsigned>((Dm + kRwFeat - 1) / kRwFeat);
-  if (bf16)
-    route_wgrad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), T, Dm, E, dlogits, dw_r, dbias);
-  else
-    route_wgrad_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), T, Dm, E,
-                                                         dlogits, dw_r, dbias);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kRwSplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((Dm + kRwFeat - 1) / kRwFeat * kRwSplit), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, route_wgrad_kernel, x, bf16, T, Dm, E, dlogits, dw_r, dbias);
 }
 
 cudaError_t launch_route_probs(const void* x, bool bf16, int64_t T, int Dm, const float* w_r,

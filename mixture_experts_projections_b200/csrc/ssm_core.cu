@@ -11,13 +11,14 @@
 //
 // Kernels, in order (all on the caller's stream, no host synchronisation):
 //  1. conv_silu_kernel: causal depthwise convolution (K taps, restart at
-//     every sequence) + bias + SiLU, bf16 X (the A operand of the next GEMM);
-//     one thread per channel walks a chunk of time steps.
-//  2. the x projection, X [T][De] x W_x -> float32 [T][Np] (the tensor-core
-//     grouped GEMM with one expert; W_x stored [Np][De], rows past R + 2N
-//     zero).
-//  3. dt_cast_kernel: the dt columns to bf16 [T][R].
-//  4. the dt projection, dt [T][R] x W_dt -> float32 [T][De] (same GEMM).
+//     every sequence) + bias + SiLU; one thread per channel walks a chunk of
+//     time steps. X is kept as two bf16 parts, hi and lo = bf16(X - hi).
+//  2. the x projection, [hi | lo] x [W_x ; W_x] -> float32 [T][Np] (the
+//     tensor-core grouped GEMM with one expert and K = 2 De, so the product
+//     is accurate to ~2^-16 although the tensor cores take bf16; W_x stored
+//     [Np][De], rows past R + 2N zero, doubled along K by dup_k_kernel).
+//  3. dt_split_kernel: the dt columns as two bf16 parts.
+//  4. the dt projection, the same way, K = 2R -> float32 [T][De].
 //  5. the scan in chunks of kChunk steps, parallel over channels and chunks:
 //     scan_kernel<false> turns dt W_dt into delta = softplus(. + b_dt) in
 //     place and runs each chunk from a zero state, keeping its final state
@@ -31,7 +32,8 @@
 // a token's k slots in slot order.
 // One thread owns one channel and all N <= 16 states of it in registers; the
 // 32 lanes of a warp are 32 consecutive channels, so every per-step load of
-// delta and x is one 128-byte row segment, and B_t, C_t (the same for every
+// delta and x is one row segment, issued kBatch steps at a time (enough
+// loads in flight to stream from HBM), and B_t, C_t (the same for every
 // channel) are staged in shared memory per chunk.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -53,13 +55,23 @@ constexpr float kLog2e = 1.4426950408889634f;
 // One thread per channel and a chunk of kConvSteps time steps (a CTA holds
 // 128 consecutive channels, so every load and store of a step is one row
 // segment); the K - 1 previous inputs stay in registers, so each input is
-// read once (plus K - 1 at the chunk's start).
+// read once (plus K - 1 at the chunk's start), and the loads of kBatch steps
+// are issued together. X is written as two bf16 parts per value, hi = bf16(v)
+// in row t, columns [0, De) and lo = bf16(v - hi) in columns [De, 2 De): the
+// x projection multiplies both by W_x (a product accurate to ~2^-16 on the
+// bf16 tensor cores) and the scan reads hi + lo.
 constexpr int kConvSteps = 64;
+constexpr int kBatch = 8;  // time steps whose loads are issued together
+
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(v);
+  lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
 
 __global__ void __launch_bounds__(128)
     conv_silu_kernel(const float* __restrict__ h, int64_t T, int De, int L,
                      const float* __restrict__ w, const float* __restrict__ b, int K,
-                     __nv_bfloat16* __restrict__ x) {
+                     __nv_bfloat16* __restrict__ x2) {
   const int d = blockIdx.x * 128 + threadIdx.x;
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kConvSteps;
   if (d >= De) return;
@@ -70,6 +82,7 @@ __global__ void __launch_bounds__(128)
     win[j] = 0.f;
   }
   const float bias = __ldg(b + d);
+  const float tcur = tap[K - 1];
   int64_t seq0 = (t0 / L) * L;
 #pragma unroll
   for (int j = 0; j < kMaxTaps - 1; ++j)
@@ -77,37 +90,68 @@ __global__ void __launch_bounds__(128)
   const int n = static_cast<int>(T - t0 < kConvSteps ? T - t0 : kConvSteps);
   int64_t next_seq = seq0 + L;  // the window restarts where the next sequence begins
   const float* hp = h + t0 * De + d;
-  __nv_bfloat16* xp = x + t0 * De + d;
-  for (int s = 0; s < n; ++s) {
-    if (t0 + s == next_seq) {
+  __nv_bfloat16* xp = x2 + t0 * (2 * static_cast<int64_t>(De)) + d;
+  for (int s0 = 0; s0 < n; s0 += kBatch) {
+    float cur[kBatch];
 #pragma unroll
-      for (int j = 0; j < kMaxTaps; ++j) win[j] = 0.f;
-      next_seq += L;
+    for (int q = 0; q < kBatch; ++q)
+      cur[q] = s0 + q < n ? __ldg(hp + static_cast<int64_t>(s0 + q) * De) : 0.f;
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int s = s0 + q;
+      if (s >= n) break;
+      if (t0 + s == next_seq) {
+#pragma unroll
+        for (int j = 0; j < kMaxTaps; ++j) win[j] = 0.f;
+        next_seq += L;
+      }
+      // tap K-1 multiplies the current step, tap K-1-j the step j back
+      float acc = fmaf(tcur, cur[q], bias);
+#pragma unroll
+      for (int j = 1; j < kMaxTaps; ++j)
+        if (j < K) acc = fmaf(tap[K - 1 - j], win[j - 1], acc);
+#pragma unroll
+      for (int j = kMaxTaps - 1; j > 0; --j) win[j] = win[j - 1];
+      win[0] = cur[q];
+      // SiLU with the fast exp and divide (relative error ~1e-6; for
+      // acc < -88 the quotient is SiLU's limit 0)
+      __nv_bfloat16 hi, lo;
+      split_bf16(__fdividef(acc, 1.0f + __expf(-acc)), hi, lo);
+      xp[static_cast<int64_t>(s) * 2 * De] = hi;
+      xp[static_cast<int64_t>(s) * 2 * De + De] = lo;
     }
-    const float cur = __ldg(hp + static_cast<int64_t>(s) * De);
-    // tap K-1 multiplies the current step, tap K-1-j the step j back
-    float acc = fmaf(tap[K - 1], cur, bias);
-#pragma unroll
-    for (int j = 1; j < kMaxTaps; ++j)
-      if (j < K) acc = fmaf(tap[K - 1 - j], win[j - 1], acc);
-#pragma unroll
-    for (int j = kMaxTaps - 1; j > 0; --j) win[j] = win[j - 1];
-    win[0] = cur;
-    // SiLU with the fast exp and divide (their error is far below the bf16
-    // rounding of X; for acc < -88 the quotient is SiLU's limit 0)
-    xp[static_cast<int64_t>(s) * De] = __float2bfloat16_rn(__fdividef(acc, 1.0f + __expf(-acc)));
   }
 }
 
+// The dt columns of [dt | B | C] as two bf16 parts: dt2[t] = [hi | lo]
+// (the dt projection multiplies both by W_dt).
 __global__ void __launch_bounds__(256)
-    dt_cast_kernel(const float* __restrict__ dbc, int64_t T, int Np, int R,
-                   __nv_bfloat16* __restrict__ dt) {
+    dt_split_kernel(const float* __restrict__ dbc, int64_t T, int Np, int R,
+                    __nv_bfloat16* __restrict__ dt2) {
   const int64_t total = T * R;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t t = i / R;
     const int r = static_cast<int>(i - t * R);
-    dt[i] = __float2bfloat16_rn(dbc[t * Np + r]);
+    __nv_bfloat16 hi, lo;
+    split_bf16(dbc[t * Np + r], hi, lo);
+    dt2[t * 2 * R + r] = hi;
+    dt2[t * 2 * R + R + r] = lo;
+  }
+}
+
+// w2[row] = [w[row] | w[row]] (rows of K bf16, K % 8 == 0): the weight twice
+// along K, so that one GEMM over [hi | lo] rows adds hi W + lo W.
+__global__ void __launch_bounds__(256)
+    dup_k_kernel(const uint4* __restrict__ w, int64_t rows, int kv, uint4* __restrict__ w2) {
+  const int64_t total = rows * kv;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / kv;
+    const int v = static_cast<int>(i - row * kv);
+    const uint4 val = __ldg(w + i);
+    w2[row * 2 * kv + v] = val;
+    w2[row * 2 * kv + kv + v] = val;
   }
 }
 
@@ -142,7 +186,7 @@ __device__ __forceinline__ float ex2_approx(float v) {
 }
 
 struct ScanArgs {
-  const __nv_bfloat16* x;  // [T][De]
+  const __nv_bfloat16* x2;  // [T][2 De]: hi | lo parts of X
   float* delta;            // [T][De]: dt W_dt on entry; delta = softplus(. + b_dt) after pass 1
   const float* b_dt;       // [De]
   const float* dbc;        // [T][Np]: dt | B | C | zero padding
@@ -161,7 +205,7 @@ struct ScanArgs {
 //   (except for a sequence's last chunk, which feeds nothing) the chunk's
 //   own recurrence from a zero state: its final state and sum of delta.
 // kOut = true: the recurrence again from the chunk's entering state, y out.
-// Each step's delta and x are loaded one step ahead of their use.
+// The loads of kBatch steps' delta and x are issued together.
 template <bool kOut>
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
   __shared__ float sB[kChunk][kMaxState];
@@ -194,33 +238,40 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
   }
   const float bd = kOut ? 0.f : __ldg(a.b_dt + d);
   const float Dd = kOut ? __ldg(a.d + d) : 0.f;
-  const __nv_bfloat16* xp = a.x + t0 * a.De + d;
+  // x = hi + lo of the two bf16 parts written by the convolution
+  const __nv_bfloat16* xp = a.x2 + t0 * (2 * static_cast<int64_t>(a.De)) + d;
   float* yp = kOut ? a.y + t0 * a.De + d : nullptr;
   float ssum = 0.f;
-  float pre_next = dp[0];
-  float x_next = __bfloat162float(xp[0]);
-  for (int s = 0; s < len; ++s) {
-    const float pre = pre_next, xv = x_next;
-    if (s + 1 < len) {
-      pre_next = dp[(s + 1) * a.De];
-      x_next = __bfloat162float(xp[(s + 1) * a.De]);
-    }
-    float delta = pre;
-    if (!kOut) {
-      delta = softplus_f(pre + bd);
-      dp[s * a.De] = delta;
-    }
-    const float dx = delta * xv;
-    ssum += delta;
-    float yv = 0.f;
+  for (int s0 = 0; s0 < len; s0 += kBatch) {
+    float pre[kBatch], xv[kBatch];
 #pragma unroll
-    for (int n = 0; n < kMaxState; ++n) {
-      if (n < N) {
-        h[n] = fmaf(ex2_approx(delta * A2[n]), h[n], dx * sB[s][n]);
-        if (kOut) yv = fmaf(h[n], sC[s][n], yv);
-      }
+    for (int q = 0; q < kBatch; ++q) {
+      const int s = s0 + q < len ? s0 + q : len - 1;
+      pre[q] = dp[s * a.De];
+      xv[q] = __bfloat162float(xp[static_cast<int64_t>(s) * 2 * a.De]) +
+              __bfloat162float(xp[static_cast<int64_t>(s) * 2 * a.De + a.De]);
     }
-    if (kOut) yp[s * a.De] = fmaf(Dd, xv, yv);
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int s = s0 + q;
+      if (s >= len) break;
+      float delta = pre[q];
+      if (!kOut) {
+        delta = softplus_f(pre[q] + bd);
+        dp[s * a.De] = delta;
+      }
+      const float dx = delta * xv[q];
+      ssum += delta;
+      float yv = 0.f;
+#pragma unroll
+      for (int n = 0; n < kMaxState; ++n) {
+        if (n < N) {
+          h[n] = fmaf(ex2_approx(delta * A2[n]), h[n], dx * sB[s][n]);
+          if (kOut) yv = fmaf(h[n], sC[s][n], yv);
+        }
+      }
+      if (kOut) yp[s * a.De] = fmaf(Dd, xv[q], yv);
+    }
   }
   if (!kOut) {
     a.S[static_cast<int64_t>(cg) * a.De + d] = ssum;
@@ -253,24 +304,26 @@ __global__ void __launch_bounds__(256) scan_carry_kernel(const ScanArgs a, int n
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 struct CoreWs {
-  __nv_bfloat16* x;
-  float* dbc;
-  __nv_bfloat16* dt;
-  float* dpre;
+  __nv_bfloat16* x2;   // [T][2 De]: X as hi | lo bf16 parts
+  float* dbc;          // [T][Np]: dt | B | C | 0
+  __nv_bfloat16* dt2;  // [T][2 R]: dt as hi | lo bf16 parts
+  float* dpre;         // [T][De]: dt W_dt, then delta
   float* S;
   float* hend;
   float* carry;
+  __nv_bfloat16* wx2;   // [E][Np][2 De]: W_x twice along K
+  __nv_bfloat16* wdt2;  // [E][De][2 R]: W_dt twice along K
   // expertized x and dt projections (k slots per token)
-  __nv_bfloat16* xs;   // [T*k][De]: X rows in expert order
-  __nv_bfloat16* dts;  // [T*k][R]: dt rows in expert order
+  __nv_bfloat16* xs;   // [T*k][2 De]: X rows in expert order
+  __nv_bfloat16* dts;  // [T*k][2 R]: dt rows in expert order
   float* dbc_slots;    // [T*k][Np] (k > 1; else the token-order buffer)
   float* dpre_slots;   // [T*k][De] (k > 1; else the token-order buffer)
   size_t bytes;
 };
 
-// k == 0: the shared core; k >= 1: expertized x and dt projections.
-CoreWs core_ws_layout(void* base, int64_t T, int De, int seq_len, int R, int N, int Np,
-                      int k = 0) {
+// k == 0: the shared core (E == 1); k >= 1: expertized x and dt projections.
+CoreWs core_ws_layout(void* base, int64_t T, int De, int seq_len, int R, int N, int Np, int E,
+                      int k) {
   const int64_t nchunks = (T / seq_len) * ((seq_len + kChunk - 1) / kChunk);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -279,20 +332,22 @@ CoreWs core_ws_layout(void* base, int64_t T, int De, int seq_len, int R, int N, 
     return static_cast<uint8_t*>(base) + o;
   };
   CoreWs w;
-  w.x = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * De * 2));
+  w.x2 = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * De * 4));
   w.dbc = reinterpret_cast<float*>(take(static_cast<size_t>(T) * Np * 4));
-  w.dt = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * R * 2));
+  w.dt2 = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(T) * R * 4));
   w.dpre = reinterpret_cast<float*>(take(static_cast<size_t>(T) * De * 4));
   w.S = reinterpret_cast<float*>(take(static_cast<size_t>(nchunks) * De * 4));
   w.hend = reinterpret_cast<float*>(take(static_cast<size_t>(nchunks) * N * De * 4));
   w.carry = reinterpret_cast<float*>(take(static_cast<size_t>(nchunks) * N * De * 4));
+  w.wx2 = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(E) * Np * De * 4));
+  w.wdt2 = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(E) * De * R * 4));
   w.xs = w.dts = nullptr;
   w.dbc_slots = w.dbc;
   w.dpre_slots = w.dpre;
   if (k >= 1) {
     const size_t Rs = static_cast<size_t>(T) * k;
-    w.xs = reinterpret_cast<__nv_bfloat16*>(take(Rs * De * 2));
-    w.dts = reinterpret_cast<__nv_bfloat16*>(take(Rs * R * 2));
+    w.xs = reinterpret_cast<__nv_bfloat16*>(take(Rs * De * 4));
+    w.dts = reinterpret_cast<__nv_bfloat16*>(take(Rs * R * 4));
     if (k > 1) {
       w.dbc_slots = reinterpret_cast<float*>(take(Rs * Np * 4));
       w.dpre_slots = reinterpret_cast<float*>(take(Rs * De * 4));
@@ -310,8 +365,9 @@ unsigned grid_for(int64_t total, int threads) {
 
 }  // namespace
 
-size_t ssm_core_workspace_bytes(int64_t T, int De, int seq_len, int R, int N, int Np, int k) {
-  return core_ws_layout(nullptr, T, De, seq_len, R, N, Np, k).bytes;
+size_t ssm_core_workspace_bytes(int64_t T, int De, int seq_len, int R, int N, int Np, int E,
+                                int k) {
+  return core_ws_layout(nullptr, T, De, seq_len, R, N, Np, E, k).bytes;
 }
 
 // One projection of the core, to float32 rows in token order: shared (one
@@ -344,24 +400,34 @@ cudaError_t launch_ssm_core(const float* h, int64_t T, int De, int seq_len, cons
                             const int32_t* sorted_slot, float* y, void* ws, int* status,
                             cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const CoreWs w = core_ws_layout(ws, T, De, seq_len, R, N, Np, k);
-  conv_silu_kernel<<<dim3(static_cast<unsigned>(De / 128),
-                         static_cast<unsigned>((T + kConvSteps - 1) / kConvSteps)),
-                    128, 0, stream>>>(h, T, De, seq_len, conv_w, conv_b, K, w.x);
+  const CoreWs w = core_ws_layout(ws, T, De, seq_len, R, N, Np, E, k);
+  // the projections' weights twice along K (one GEMM then adds hi W + lo W)
+  const int64_t ex = static_cast<int64_t>(E);
+  dup_k_kernel<<<grid_for(ex * Np * (De / 8), 256), 256, 0, stream>>>(
+      static_cast<const uint4*>(w_x), ex * Np, De / 8, reinterpret_cast<uint4*>(w.wx2));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // x projection to [dt | B | C | 0] float32 rows, token order
-  e = core_projection(w.x, T, De, w_x, Np, E, k, offsets, sorted_slot, w.xs, w.dbc_slots, w.dbc,
-                      status, stream);
-  if (e != cudaSuccess) return e;
-  dt_cast_kernel<<<grid_for(T * R, 256), 256, 0, stream>>>(w.dbc, T, Np, R, w.dt);
+  dup_k_kernel<<<grid_for(ex * De * (R / 8), 256), 256, 0, stream>>>(
+      static_cast<const uint4*>(w_dt), ex * De, R / 8, reinterpret_cast<uint4*>(w.wdt2));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = core_projection(w.dt, T, R, w_dt, De, E, k, offsets, sorted_slot, w.dts, w.dpre_slots,
-                      w.dpre, status, stream);
+  conv_silu_kernel<<<dim3(static_cast<unsigned>(De / 128),
+                         static_cast<unsigned>((T + kConvSteps - 1) / kConvSteps)),
+                    128, 0, stream>>>(h, T, De, seq_len, conv_w, conv_b, K, w.x2);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // x projection to [dt | B | C | 0] float32 rows, token order
+  e = core_projection(w.x2, T, 2 * De, w.wx2, Np, E, k, offsets, sorted_slot, w.xs, w.dbc_slots,
+                      w.dbc, status, stream);
+  if (e != cudaSuccess) return e;
+  dt_split_kernel<<<grid_for(T * R, 256), 256, 0, stream>>>(w.dbc, T, Np, R, w.dt2);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = core_projection(w.dt2, T, 2 * R, w.wdt2, De, E, k, offsets, sorted_slot, w.dts,
+                      w.dpre_slots, w.dpre, status, stream);
   if (e != cudaSuccess) return e;
   ScanArgs a;
-  a.x = w.x;
+  a.x2 = w.x2;
   a.delta = w.dpre;
   a.b_dt = b_dt;
   a.dbc = w.dbc;
@@ -416,7 +482,7 @@ int ssm_core_entry(const float* h, int64_t T, int De, int seq_len, const float* 
   if ((reinterpret_cast<uintptr_t>(h) & 15u) || (reinterpret_cast<uintptr_t>(w_x) & 15u) ||
       (reinterpret_cast<uintptr_t>(w_dt) & 15u))
     return ROM_ERR_UNSUPPORTED;
-  if (!ws || ws_bytes < rom::ssm_core_workspace_bytes(T, De, seq_len, R, N, Np, k) ||
+  if (!ws || ws_bytes < rom::ssm_core_workspace_bytes(T, De, seq_len, R, N, Np, k > 0 ? E : 1, k) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return ROM_ERR_WORKSPACE;
   int* st = rom::status_ptr();
@@ -437,13 +503,13 @@ bool core_sizes_ok(int64_t T, int De, int seq_len, int R, int N, int Np) {
 extern "C" size_t rom_ssm_core_workspace_size(int64_t T, int De, int seq_len, int R, int N,
                                               int Np) {
   if (!core_sizes_ok(T, De, seq_len, R, N, Np)) return 0;
-  return rom::ssm_core_workspace_bytes(T, De, seq_len, R, N, Np, 0);
+  return rom::ssm_core_workspace_bytes(T, De, seq_len, R, N, Np, 1, 0);
 }
 
 extern "C" size_t rom_ssm_core_routed_workspace_size(int64_t T, int De, int seq_len, int R, int N,
-                                                     int Np, int k) {
-  if (!core_sizes_ok(T, De, seq_len, R, N, Np) || k < 1) return 0;
-  return rom::ssm_core_workspace_bytes(T, De, seq_len, R, N, Np, k);
+                                                     int Np, int E, int k) {
+  if (!core_sizes_ok(T, De, seq_len, R, N, Np) || k < 1 || E < 1) return 0;
+  return rom::ssm_core_workspace_bytes(T, De, seq_len, R, N, Np, E, k);
 }
 
 extern "C" int rom_ssm_core(const float* h, int64_t T, int De, int seq_len, const float* conv_w,

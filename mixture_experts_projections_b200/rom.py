@@ -50,7 +50,7 @@ SIGNATURES = {
     "rom_route_wgrad": (_I, [_P, _I, _L, _I, _I, _P, _P, _P, _P]),
     "rom_bwd_wgrad": (_I, [_P, _I, _P, _I, _L, _I, _P, _I, _P, _P, _P]),
     "rom_ssm_core_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I]),
-    "rom_ssm_core_routed_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I, _I]),
+    "rom_ssm_core_routed_workspace_size": (ctypes.c_size_t, [_L, _I, _I, _I, _I, _I, _I, _I]),
     "rom_ssm_core_routed": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P,
                                  _I, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "rom_ssm_core": (_I, [_P, _L, _I, _I, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P,
@@ -270,7 +270,7 @@ def rom_ssm_core(h, seq_len, core, y, ws, stream=None, routing=None):
 def core_workspace(T, De, seq_len, core, device, k=1):
     if core.routed:
         n = int(load_library().rom_ssm_core_routed_workspace_size(T, De, seq_len, core.R, core.N,
-                                                                  core.Np, k))
+                                                                  core.Np, core.E, k))
     else:
         n = rom_ssm_core_workspace_size(T, De, seq_len, core.R, core.N, core.Np)
     return torch.empty((max(n, 256),), dtype=torch.uint8, device=device)
