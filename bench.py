@@ -6,7 +6,8 @@
 One step = one pass of the whole block over one batch of synthetic input:
 route -> dispatch -> Conv+Gate grouped GEMM (+ gate combine for top-k > 1)
 -> Out grouped GEMM (+ slot sum for top-k > 1); for the Swimba decode
-workload: route -> dispatch -> routed in-projection. Inputs are resident in
+workload: route -> routed in-projection (a decode batch of at most 64 tokens
+needs no dispatch). Inputs are resident in
 HBM when the timed region starts. Between timed steps the L2 is flushed (a
 256 MiB write, outside the step's events), except where the step's inputs
 (tokens and weights) exceed twice the L2: then every step streams them from
@@ -326,21 +327,34 @@ def build_workload(torch, rom, wl, inp):
         slots = (torch.empty((R, wl.De), dtype=torch.float32, device=x.device)
                  if wl.k > 1 else None)
 
+        # a decode-sized batch takes the projection without a dispatch
+        dense = bf16 and wl.T <= rom.DENSE_SMALL_MAX_TOKENS
+
         def ph_route():
-            rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, bufs)
+            if dense:
+                rom.rom_route(x, w_r, bias, wl.k, wl.renorm, bufs.topk_idx, bufs.topk_w,
+                              bufs.counts, bufs.ws)
+            else:
+                rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, bufs)
 
         def ph_p0():
-            rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
-                                bufs.offsets, bufs.sorted_slot, bufs.topk_w,
-                                out if wl.k == 1 else slots)
+            if dense:
+                rom.rom_expert_proj_dense(rom.ROM_PROJ_INPROJ, x, w, wl.E, wl.k, bufs.topk_idx,
+                                          bufs.topk_w, out if wl.k == 1 else slots)
+            else:
+                rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
+                                    bufs.offsets, bufs.sorted_slot, bufs.topk_w,
+                                    out if wl.k == 1 else slots)
 
         def ph_p1():
             if wl.k > 1:
                 rom.rom_combine(rom.ROM_COMBINE_SUM, dt, slots, wl.T, wl.k, wl.De, None, out)
-        res.update(phases=[("route_dispatch", ph_route), ("proj0", ph_p0), ("proj1", ph_p1)],
+        res.update(phases=[("route" if dense else "route_dispatch", ph_route), ("proj0", ph_p0),
+                           ("proj1", ph_p1)],
                    dominant=(ph_p0, "byte",
                              lambda counts: inproj_bytes(wl, int(np.count_nonzero(counts)))),
-                   out=out, counts=bufs.counts, launches=3 + (1 if wl.k > 1 else 0))
+                   out=out, counts=bufs.counts,
+                   launches=(2 if dense else 3) + (1 if wl.k > 1 else 0))
         pipe = rom.HostPipeline(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
         res["e2e"] = (pipe, lambda hx, ho: pipe.inproj_forward(hx, w_r, w, ho, renorm=wl.renorm,
                                                                 bias=bias))
@@ -620,7 +634,9 @@ def roofline(res, peaks, src):
     t_k = res["dominant_ms"] / 1e3
     if res["dominant_kind"] == "byte":
         ach = res["dominant_work"] / t_k / 1e9
-        return {"bound": "hbm", "kernel": "rom_expert_proj(INPROJ)", "achieved": ach,
+        kern = ("rom_expert_proj_dense(INPROJ)" if wl.T <= 64 and wl.dtype == "bf16"
+                else "rom_expert_proj(INPROJ)")
+        return {"bound": "hbm", "kernel": kern, "achieved": ach,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
                 "traffic": profiled_traffic(wl.name), "peak_source": f"{src} hbm_gbs"}
     ach = res["dominant_work"] / t_k / 1e12

@@ -173,6 +173,31 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
                     const int32_t* sorted_slot, const float* topk_w, void* out, void* stream);
 
 /*
+ * rom_expert_proj_dense -- the routed projection for a few tokens (T <= 64)
+ * without a dispatch (Swimba page, Extended abstract: s_t = sum_j r_{t,j}
+ * x_t W_{S_j}; RoM page, Knowl 1 for the Out projection). Every expert's
+ * weight tiles meet all T tokens, taken in token order, and the routing
+ * only selects in the epilogue: token t keeps expert e's result exactly when
+ * e is one of its k selected experts. The weights stream once, as in
+ * rom_expert_proj. Nothing before the epilogue depends on the routing, so
+ * the kernel is launched as a programmatic dependent of the kernel before it
+ * on the stream (the router: decode steps need no rom_dispatch) and only its
+ * epilogue waits for that kernel's results.
+ *
+ *  proj      ROM_PROJ_INPROJ or ROM_PROJ_OUT (both weighted by r)
+ *  x         [T][K] bf16, token order (as given to rom_route)
+ *  w         [E][N][K] bf16
+ *  topk_idx, topk_w [T][k] from rom_route
+ *  out       k == 1: [T][N] bf16, token order; k > 1: float32 [T*k][N] in slot
+ *            order (then rom_combine(ROM_COMBINE_SUM))
+ * Requires dtype ROM_BF16, 1 <= T <= 64, K % 8 == 0, N % 128 == 0 and
+ * 16-byte aligned x, w and out.
+ */
+int rom_expert_proj_dense(int proj, int dtype, const void* x, int64_t T, int K, const void* w,
+                          int N, int E, int k, const int32_t* topk_idx, const float* topk_w,
+                          void* out, void* stream);
+
+/*
  * rom_combine -- reduce the k slots of each token in slot order 0..k-1.
  *  ROM_COMBINE_SUM:  in = float32 [T*k][N] (slot order); out = [T][N] dtype,
  *                    out[t] = sum_j in[t*k+j]. slot_pos is unused (may be NULL).

@@ -62,6 +62,8 @@ struct Params {
   int k;
   int n_tiles_n;
   int* status;
+  // the dense small-batch in-projection: every token's experts (else null)
+  const int32_t* topk_idx;
 };
 
 // u * SiLU(z) = u * z / (1 + e^-z), with the fast exp and divide intrinsics:
@@ -466,7 +468,15 @@ __device__ __forceinline__ void swap_token(const Params& p, int64_t prow, bool v
   }
 }
 
-template <int MODE>
+// kDense: the small-batch form without a dispatch (T <= 64 tokens, one token
+// block). Every expert's weight tiles meet all T tokens, which the producer
+// loads in token order; the routing decides only which results are kept: for
+// token t and expert e, the epilogue stores r * acc where e is one of t's
+// selected experts and nothing otherwise. The weights stream once either
+// way (each expert's tiles for its single token block), and since nothing
+// before the epilogue depends on the routing, the kernel is launched as a
+// programmatic dependent of the router and only its epilogue waits for it.
+template <int MODE, bool kDense>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_swap_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmX, const Params p) {
@@ -504,13 +514,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&ctl.tmem_base, SW_TMEM_COLS);
     tmem_relinquish();
   }
-  pdl_wait();  // the routing (offsets, sorted rows, weights) is complete from here
-  for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = offset_of(p, i);
+  if (!kDense) {
+    pdl_wait();  // the routing (offsets, sorted rows, weights) is complete from here
+    for (int i = threadIdx.x; i <= E; i += kThreads) ctl.off[i] = offset_of(p, i);
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = 0;
     for (int e = 0; e < E; ++e) {
-      const int tt = (ctl.off[e + 1] - ctl.off[e] + SW_BN - 1) / SW_BN;
+      // dense: one block of all (<= 64) tokens per expert, in token order
+      const int tt = kDense ? 1 : (ctl.off[e + 1] - ctl.off[e] + SW_BN - 1) / SW_BN;
       ctl.tt[e] = tt;
       ctl.tile_start[e] = run;
       run += tt * n_wt;
@@ -544,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int e, w_blk, t_blk;
         coords(tile, e, w_blk, t_blk);
         const int n0 = w_blk * SW_BM;
-        const int r0 = ctl.off[e] + t_blk * SW_BN;
+        const int r0 = kDense ? 0 : ctl.off[e] + t_blk * SW_BN;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -609,17 +622,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
+    if (kDense) pdl_wait();  // the router's topk_idx / topk_w are complete from here
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       int e, w_blk, t_blk;
       coords(tile, e, w_blk, t_blk);
-      const int n_e = ctl.off[e + 1] - ctl.off[e];
-      const int nv = min(SW_BN, n_e - t_blk * SW_BN);  // valid token columns, >= 1
-      // token info first: its loads overlap the wait for the accumulator
-      const int64_t prow0 = static_cast<int64_t>(ctl.off[e]) + t_blk * SW_BN;
+      int nv;  // token columns of the tile that may be stored
       int orow[2];
       float rw[2];
-      swap_token<MODE>(p, prow0 + lane, lane < nv, orow[0], rw[0]);
-      swap_token<MODE>(p, prow0 + 32 + lane, 32 + lane < nv, orow[1], rw[1]);
+      bool keep[2] = {true, true};
+      if (kDense) {
+        nv = static_cast<int>(p.R < SW_BN ? p.R : SW_BN);  // all T tokens, one block
+        // column c*32 + lane is token t; kept where e is one of its experts
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int t = 32 * c + lane;
+          keep[c] = false;
+          orow[c] = 0;
+          rw[c] = 0.f;
+          if (t < nv)
+            for (int j = 0; j < p.k; ++j) {
+              const int64_t slot = static_cast<int64_t>(t) * p.k + j;
+              if (p.topk_idx[slot] == e) {
+                keep[c] = true;
+                rw[c] = p.topk_w[slot];
+                orow[c] = MODE == kEpiScaleToken ? t : static_cast<int>(slot);
+              }
+            }
+        }
+      } else {
+        const int n_e = ctl.off[e + 1] - ctl.off[e];
+        nv = min(SW_BN, n_e - t_blk * SW_BN);  // valid token columns, >= 1
+        // token info first: its loads overlap the wait for the accumulator
+        const int64_t prow0 = static_cast<int64_t>(ctl.off[e]) + t_blk * SW_BN;
+        swap_token<MODE>(p, prow0 + lane, lane < nv, orow[0], rw[0]);
+        swap_token<MODE>(p, prow0 + 32 + lane, 32 + lane < nv, orow[1], rw[1]);
+      }
       if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t t_row =
@@ -636,11 +673,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (32 * c + j < nv) {  // warp-uniform
               const int o = __shfl_sync(0xffffffffu, orow[c], j);
               const float v = __shfl_sync(0xffffffffu, rw[c], j) * __uint_as_float(a[j]);
+              const bool kept = __shfl_sync(0xffffffffu, keep[c] ? 1 : 0, j) != 0;
               const int64_t i = static_cast<int64_t>(o) * p.N + n;
-              if (MODE == kEpiScaleToken)
-                static_cast<__nv_bfloat16*>(p.out)[i] = __float2bfloat16_rn(v);
-              else
-                static_cast<float*>(p.out)[i] = v;
+              if (kept) {
+                if (MODE == kEpiScaleToken)
+                  static_cast<__nv_bfloat16*>(p.out)[i] = __float2bfloat16_rn(v);
+                else
+                  static_cast<float*>(p.out)[i] = v;
+              }
             }
           }
         }
@@ -764,8 +804,8 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
     const int64_t sms = device_sm_count();
     const int64_t per_cta = (tiles_ub + sms - 1) / sms;
     const int grid = static_cast<int>(std::min<int64_t>(sms, (tiles_ub + per_cta - 1) / per_cta));
-    auto kern = (mode == kEpiScaleToken) ? tc_swap_gemm_kernel<kEpiScaleToken>
-                                         : tc_swap_gemm_kernel<kEpiScaleSlots>;
+    auto kern = (mode == kEpiScaleToken) ? tc_swap_gemm_kernel<kEpiScaleToken, false>
+                                         : tc_swap_gemm_kernel<kEpiScaleSlots, false>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(kSwapSmemBytes));
     if (err != cudaSuccess) return err;
@@ -821,6 +861,49 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
         return cudaErrorInvalidValue;
     }
   }
+}
+
+cudaError_t launch_tc_dense_small(int mode, const void* x, int64_t T, int K, const void* w, int N,
+                                  int E, int k, const int32_t* topk_idx, const float* topk_w,
+                                  void* out, int* status, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  if (T > SW_BN || N % SW_BM != 0 || K % 8 != 0 || E > kMaxExperts) return cudaErrorInvalidValue;
+  CUtensorMap tw, tx;
+  if (!make_map(&tw, w, K, N, E, SW_BM)) return cudaErrorInvalidValue;
+  if (!make_map(&tx, x, K, T, 0, SW_BN)) return cudaErrorInvalidValue;
+  Params p{};
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  p.out = out;
+  p.R = T;  // token rows (in token order)
+  p.K = K;
+  p.N = N;
+  p.E = E;
+  p.k = k;
+  p.status = status;
+  // every CTA gets the same number of tiles (E x N/128 tiles in all)
+  const int64_t tiles = static_cast<int64_t>(E) * (N / SW_BM);
+  const int64_t sms = device_sm_count();
+  const int64_t per_cta = (tiles + sms - 1) / sms;
+  const int grid = static_cast<int>(std::min<int64_t>(sms, (tiles + per_cta - 1) / per_cta));
+  auto kern = (mode == kEpiScaleToken) ? tc_swap_gemm_kernel<kEpiScaleToken, true>
+                                       : tc_swap_gemm_kernel<kEpiScaleSlots, true>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSwapSmemBytes));
+  if (err != cudaSuccess) return err;
+  // a programmatic dependent of the router: the weight streaming and the
+  // MMAs run while the router finishes; the epilogue waits for it
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSwapSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
 }
 
 }  // namespace rom

@@ -201,6 +201,25 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
                                                     offsets, sorted_slot, topk_w, out, st, s));
 }
 
+int rom_expert_proj_dense(int proj, int dtype, const void* x, int64_t T, int K, const void* w,
+                          int N, int E, int k, const int32_t* topk_idx, const float* topk_w,
+                          void* out, void* stream) {
+  if (proj != ROM_PROJ_OUT && proj != ROM_PROJ_INPROJ) return ROM_ERR_INVALID_ARG;
+  if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
+  if (T < 0 || K <= 0 || N <= 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E ||
+      k > rom::kMaxTopK)
+    return ROM_ERR_INVALID_ARG;
+  if (dtype != ROM_BF16 || T > 64 || K % 8 != 0 || N % 128 != 0) return ROM_ERR_UNSUPPORTED;
+  if (T == 0) return ROM_OK;
+  if (!x || !w || !topk_idx || !topk_w || !out) return ROM_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return ROM_ERR_UNSUPPORTED;
+  int* st = rom::status_ptr();
+  if (!st) return ROM_ERR_CUDA;
+  return rom::to_status(rom::launch_tc_dense_small(
+      k == 1 ? rom::kEpiScaleToken : rom::kEpiScaleSlots, x, T, K, w, N, E, k, topk_idx, topk_w,
+      out, st, static_cast<cudaStream_t>(stream)));
+}
+
 int rom_combine(int mode, int dtype, const void* in, int64_t T, int k, int N,
                 const int32_t* slot_pos, void* out, void* stream) {
   if (mode != ROM_COMBINE_SUM && mode != ROM_COMBINE_GATE && mode != ROM_COMBINE_GATE_DENSE)

@@ -81,6 +81,12 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
                                    const float* topk_w, void* out, int* status,
                                    cudaStream_t stream);
 
+// Small-batch (T <= 64) routed projection without a dispatch: x in token
+// order, the router's topk_idx / topk_w read only by the epilogue.
+cudaError_t launch_tc_dense_small(int mode, const void* x, int64_t T, int K, const void* w, int N,
+                                  int E, int k, const int32_t* topk_idx, const float* topk_w,
+                                  void* out, int* status, cudaStream_t stream);
+
 // float32 SIMT grouped GEMM (same semantics as the tensor-core one).
 cudaError_t launch_simt_grouped_gemm(int mode, const float* a_sorted, int64_t R, int K,
                                      const float* w0, const float* w1, int N, int E, int k,

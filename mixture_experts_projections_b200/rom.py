@@ -37,6 +37,7 @@ SIGNATURES = {
     "rom_dispatch": (_I, [_P, _I, _L, _I, _I, _I, _P, _P, ctypes.c_size_t, _P, _P, _P, _P, _P]),
     "rom_expert_proj": (_I, [_I, _I, _P, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "rom_combine": (_I, [_I, _I, _P, _L, _I, _I, _P, _P, _P]),
+    "rom_expert_proj_dense": (_I, [_I, _I, _P, _L, _I, _P, _I, _I, _I, _P, _P, _P, _P]),
     "rom_get_status": (_I, [_P, ctypes.POINTER(ctypes.c_int32)]),
     "rom_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "rom_route_dispatch_noalloc": (_I, [_P, _I, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
@@ -144,6 +145,19 @@ def rom_expert_proj(proj, a_sorted, w0, w1, E, k, offsets, sorted_slot, topk_w, 
         proj, _dtype_code(a_sorted), _ptr(a_sorted), R, K, _ptr(w0), _ptr(w1), N, E, k,
         _ptr(offsets), _ptr(sorted_slot), _ptr(topk_w), _ptr(out), _stream(stream)),
         "rom_expert_proj")
+
+
+def rom_expert_proj_dense(proj, x, w, E, k, topk_idx, topk_w, out, stream=None):
+    T, K = x.shape
+    N = w.shape[1]
+    _check(load_library().rom_expert_proj_dense(
+        proj, _dtype_code(x), _ptr(x), T, K, _ptr(w), N, E, k, _ptr(topk_idx), _ptr(topk_w),
+        _ptr(out), _stream(stream)), "rom_expert_proj_dense")
+
+
+# Few tokens: the routed projection reads x in token order and needs no
+# dispatch (rom_expert_proj_dense).
+DENSE_SMALL_MAX_TOKENS = 64
 
 
 def rom_combine(mode, dtype_code, inp, T, k, N, slot_pos, out, stream=None):
@@ -366,14 +380,33 @@ def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=Non
 
 
 def inproj_forward(x, w_r, w, k=1, renorm=False, bias=None, bufs=None, out=None, slots=None,
-                   stream=None):
-    """Swimba routed in-projection: s_t = sum_j r_{t,j} x_t W_{S_j} (W as [E, N, Dm])."""
+                   stream=None, dense_small=True):
+    """Swimba routed in-projection: s_t = sum_j r_{t,j} x_t W_{S_j} (W as [E, N, Dm]).
+
+    A bf16 batch of at most DENSE_SMALL_MAX_TOKENS tokens (a decode step)
+    takes the projection without a dispatch (rom_expert_proj_dense) unless
+    ``dense_small`` is False."""
     T, Dm = x.shape
     E, N, _ = w.shape
-    rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs, stream)
+    R = T * k
     if out is None:
         out = torch.empty((T, N), dtype=x.dtype, device=x.device)
-    R = T * k
+    if dense_small and x.dtype == torch.bfloat16 and 0 < T <= DENSE_SMALL_MAX_TOKENS:
+        if bufs is None:
+            bufs = RoutingBuffers(T, Dm, E, k, x.dtype, x.device)
+        rom_route(x, w_r, bias, k, renorm, bufs.topk_idx, bufs.topk_w, bufs.counts, bufs.ws,
+                  stream)
+        if k == 1:
+            rom_expert_proj_dense(ROM_PROJ_INPROJ, x, w, E, k, bufs.topk_idx, bufs.topk_w, out,
+                                  stream)
+        else:
+            if slots is None:
+                slots = torch.empty((R, N), dtype=torch.float32, device=x.device)
+            rom_expert_proj_dense(ROM_PROJ_INPROJ, x, w, E, k, bufs.topk_idx, bufs.topk_w, slots,
+                                  stream)
+            rom_combine(ROM_COMBINE_SUM, _dtype_code(x), slots, T, k, N, None, out, stream)
+        return out, bufs
+    rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs, stream)
     if k == 1:
         rom_expert_proj(ROM_PROJ_INPROJ, rb.x_sorted[:R], w, None, E, k, rb.offsets,
                         rb.sorted_slot, rb.topk_w, out, stream)

@@ -242,3 +242,15 @@ def test_binding_signatures_match_the_header_arity():
     assert arity, "no declarations parsed"
     for name, n in arity.items():
         assert len(rom.SIGNATURES[name][1]) == n, (name, len(rom.SIGNATURES[name][1]), n)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(proj=0), 1), (dict(dtype=5), 1), (dict(E=0), 1), (dict(k=3, E=2), 1),
+    (dict(T=65), 2), (dict(dtype=0), 2), (dict(N=200), 2), (dict(K=12), 2),
+    (dict(topk_idx=None), 1), (dict(out=ctypes.c_void_p((1 << 20) + 4)), 2),
+])
+def test_expert_proj_dense_rejects_bad_arguments(lib, kw, code):
+    a = dict(proj=2, dtype=1, x=FAKE, T=64, K=64, w=FAKE, N=256, E=4, k=1, topk_idx=FAKE,
+             topk_w=FAKE, out=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_expert_proj_dense(*a.values()) == code

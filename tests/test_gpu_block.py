@@ -194,3 +194,27 @@ def test_host_pipeline_inproj_matches_single_call(T, Dm, N, E, k, renorm):
     orc_ref = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=k, renorm=renorm)
     assert_close(out_h.float().numpy().astype(np.float64), orc_ref["S"], "bf16", "S (pipelined)",
                  magnitude_scaled_abs=True)
+
+@pytest.mark.parametrize("T,Dm,N,E,k,renorm", [
+    (64, 512, 1280, 4, 1, False),
+    (37, 1024, 512, 8, 1, False),
+    (1, 256, 256, 4, 1, False),
+    (50, 256, 768, 4, 2, True),
+    (64, 1024, 1024, 16, 2, False),
+])
+def test_inproj_without_dispatch_for_small_batches(T, Dm, N, E, k, renorm):
+    """rom_expert_proj_dense (every expert's weights meet all tokens, the
+    routing selects in the epilogue, launched as a dependent of the router)
+    against the oracle and against the dispatched path on the same inputs."""
+    inp = make_inproj_inputs(T, Dm, N, E, seed=3 * T + N + k, router_std=0.05)
+    ref = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=k, renorm=renorm)
+    args = (to_dev(inp["x"], "bf16"), to_dev(inp["w_r"], "f32"), weights_to_dev(inp["w"], "bf16"))
+    dense, rb = rom.inproj_forward(*args, k=k, renorm=renorm)
+    sparse, _ = rom.inproj_forward(*args, k=k, renorm=renorm, dense_small=False)
+    torch.cuda.synchronize()
+    assert rom.rom_get_status() == 0
+    assert_routing_matches(rb.topk_idx.cpu().numpy(), rb.topk_w.cpu().numpy().astype(np.float64),
+                           ref, x=inp["x"], w_r=inp["w_r"])
+    assert_close(to_np(dense), ref["S"], "bf16", "S (no dispatch)", magnitude_scaled_abs=True)
+    assert_close(to_np(dense), to_np(sparse), "bf16", "no dispatch vs dispatched",
+                 magnitude_scaled_abs=True)
