@@ -266,70 +266,93 @@ __global__ void __launch_bounds__(256)
 
 // Router weight gradients: dW_r[d][e] = sum_t x[t][d] dlogit[t][e] and
 // dbias[e] = sum_t dlogit[t][e], in float32. A cluster of kRwSplit CTAs owns
-// 64 features of d_model; CTA r of the cluster sums the tokens of its slice
-// r of T (tiles of 64 tokens of x and of the logit gradients through shared
-// memory, thread (f, g) accumulating feature f for the experts g, g+4, ...),
-// then CTA 0 adds the kRwSplit partial sums in rank order through
-// distributed shared memory. The order of every sum is fixed, so the result
-// does not depend on the launch.
-constexpr int kRwFeat = 64, kRwTok = 64, kRwSplit = 8;
+// 64 features of d_model; CTA r of the cluster sums the tokens of its slice r
+// of T. The CTA walks its slice in chunks of 128 tokens: the chunk's logit
+// gradients are staged in shared memory (coalesced), and warp w takes tokens
+// 16w .. 16w+15 of the chunk, each lane two features for all experts: the 16
+// tokens' x loads are issued together, then per token and expert one packed
+// FMA updates the lane's two feature sums (the gradient row read as
+// broadcast float4s). The 8 warps' sums are added in warp order, then CTA 0
+// adds the kRwSplit partial sums in rank order through distributed shared
+// memory. The order of every sum is fixed, so the result does not depend on
+// the launch.
+constexpr int kRwFeat = 64, kRwSplit = 8, kRwChunk = 128, kRwTokPerWarp = 16;
 
+template <int EB, typename InT>
 __global__ void __launch_bounds__(256)
-    route_wgrad_kernel(const void* __restrict__ xv, bool bf16, int64_t T, int Dm, int E,
+    route_wgrad_kernel(const InT* __restrict__ x, int64_t T, int Dm, int E,
                        const float* __restrict__ dl, float* __restrict__ dw_r,
                        float* __restrict__ dbias) {
-  static_assert(kRwTok == kRwFeat && kRwFeat >= kMaxExperts, "partials reuse the x tile");
-  __shared__ float sx[kRwTok][kRwFeat + 1];  // the x tile; after the loop the partial sums
-  __shared__ float sdl[kRwTok][kMaxExperts + 1];
-  __shared__ float s_bias[kMaxExperts];
-  float(*s_part)[kRwFeat + 1] = sx;
+  static_assert(kRwChunk * EB >= kRwFeat * EB && kRwChunk == 8 * kRwTokPerWarp, "layout");
+  constexpr int kGroups = 256 / EB;  // bias: token groups per expert
+  __shared__ __align__(16) float s_dl[kRwChunk][EB];  // after the loop: the partial sums
+  __shared__ float s_bsum[256];
+  __shared__ float s_bias[EB];
+  float(*s_part)[EB] = reinterpret_cast<float(*)[EB]>(&s_dl[0][0]);  // [kRwFeat][EB]
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int tid = threadIdx.x, f = tid & 63, g = tid >> 6;  // g in 0..3
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d0 = (blockIdx.x / kRwSplit) * kRwFeat;
+  const int da = d0 + 2 * lane, db = da + 1;  // this lane's features
   const bool bias_cluster = blockIdx.x / kRwSplit == 0 && dbias != nullptr;
   const int64_t per = (T + kRwSplit - 1) / kRwSplit;
   const int64_t ta = rank * per, tb = ta + per < T ? ta + per : T;
-  constexpr int Q = kMaxExperts / 4;
-  float acc[Q], bacc[Q];
+  float2 acc[EB];
 #pragma unroll
-  for (int q = 0; q < Q; ++q) acc[q] = bacc[q] = 0.f;
-  for (int64_t t0 = ta; t0 < tb; t0 += kRwTok) {
-    const int nt = static_cast<int>(tb - t0 < kRwTok ? tb - t0 : kRwTok);
-    for (int i = tid; i < kRwTok * kRwFeat; i += 256) {
-      const int r = i / kRwFeat, c = i - r * kRwFeat;
-      float v = 0.f;
-      if (r < nt && d0 + c < Dm) {
-        const int64_t at = (t0 + r) * Dm + d0 + c;
-        v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(xv)[at])
-                 : static_cast<const float*>(xv)[at];
-      }
-      sx[r][c] = v;
+  for (int e = 0; e < EB; ++e) acc[e] = make_float2(0.f, 0.f);
+  float bacc = 0.f;  // bias: expert tid % EB over token group tid / EB
+  for (int64_t t0 = ta; t0 < tb; t0 += kRwChunk) {
+    const int nt = static_cast<int>(tb - t0 < kRwChunk ? tb - t0 : kRwChunk);
+    // x of this warp's 16 tokens first: their loads overlap the staging
+    float2 xv[kRwTokPerWarp];
+#pragma unroll
+    for (int u = 0; u < kRwTokPerWarp; ++u) {
+      const int r = kRwTokPerWarp * warp + u;
+      const InT* row = x + (t0 + r) * Dm;
+      const bool ok = r < nt;
+      xv[u].x = (ok && da < Dm) ? static_cast<float>(row[da]) : 0.f;
+      xv[u].y = (ok && db < Dm) ? static_cast<float>(row[db]) : 0.f;
     }
-    for (int i = tid; i < kRwTok * E; i += 256) {
-      const int r = i / E, e = i - r * E;
-      sdl[r][e] = r < nt ? dl[(t0 + r) * E + e] : 0.f;
+    for (int i = tid; i < kRwChunk * EB; i += 256) {
+      const int r = i / EB, e = i - r * EB;
+      s_dl[r][e] = (r < nt && e < E) ? dl[(t0 + r) * E + e] : 0.f;
     }
     __syncthreads();
-    for (int r = 0; r < nt; ++r) {
-      const float x = sx[r][f];
 #pragma unroll
-      for (int q = 0; q < Q; ++q) {
-        const int e = g + 4 * q;
-        if (e < E) {
-          acc[q] = fmaf(x, sdl[r][e], acc[q]);
-          if (bias_cluster && f == 0) bacc[q] += sdl[r][e];
-        }
+    for (int u = 0; u < kRwTokPerWarp; ++u) {
+      const float4* g4 = reinterpret_cast<const float4*>(&s_dl[kRwTokPerWarp * warp + u][0]);
+#pragma unroll
+      for (int e4 = 0; e4 < EB / 4; ++e4) {
+        const float4 g = g4[e4];
+        acc[4 * e4] = __ffma2_rn(xv[u], make_float2(g.x, g.x), acc[4 * e4]);
+        acc[4 * e4 + 1] = __ffma2_rn(xv[u], make_float2(g.y, g.y), acc[4 * e4 + 1]);
+        acc[4 * e4 + 2] = __ffma2_rn(xv[u], make_float2(g.z, g.z), acc[4 * e4 + 2]);
+        acc[4 * e4 + 3] = __ffma2_rn(xv[u], make_float2(g.w, g.w), acc[4 * e4 + 3]);
+      }
+    }
+    if (bias_cluster)
+      for (int r = tid / EB; r < kRwChunk; r += kGroups) bacc += s_dl[r][tid % EB];
+    __syncthreads();
+  }
+  // the warps' sums, added in warp order
+#pragma unroll 1
+  for (int w = 0; w < 8; ++w) {
+    if (warp == w) {
+#pragma unroll
+      for (int e = 0; e < EB; ++e) {
+        s_part[2 * lane][e] = (w == 0) ? acc[e].x : s_part[2 * lane][e] + acc[e].x;
+        s_part[2 * lane + 1][e] = (w == 0) ? acc[e].y : s_part[2 * lane + 1][e] + acc[e].y;
       }
     }
     __syncthreads();
   }
-#pragma unroll
-  for (int q = 0; q < Q; ++q) {
-    const int e = g + 4 * q;
-    if (e < E) {
-      s_part[f][e] = acc[q];
-      if (f == 0) s_bias[e] = bacc[q];
+  if (bias_cluster) {
+    s_bsum[tid] = bacc;
+    __syncthreads();
+    if (tid < EB) {
+      float v = s_bsum[tid];
+      for (int g = 1; g < kGroups; ++g) v += s_bsum[g * EB + tid];
+      s_bias[tid] = v;
     }
   }
   cluster.sync();  // every CTA's partial sums are in its shared memory
@@ -390,7 +413,23 @@ cudaError_t launch_route_wgrad(const void* x, bool bf16, int64_t T, int Dm, int 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, route_wgrad_kernel, x, bf16, T, Dm, E, dlogits, dw_r, dbias);
+  // experts rounded up to 4, 8, 16, 32 or 64 (the padded columns are zero)
+  const int eb = E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64;
+#define ROM_RWG_CASE(EBV)                                                                      \
+  if (eb == EBV)                                                                               \
+    return bf16 ? cudaLaunchKernelEx(&cfg, route_wgrad_kernel<EBV, __nv_bfloat16>,             \
+                                     static_cast<const __nv_bfloat16*>(x), T, Dm, E, dlogits,  \
+                                     dw_r, dbias)                                              \
+                : cudaLaunchKernelEx(&cfg, route_wgrad_kernel<EBV, float>,                     \
+                                     static_cast<const float*>(x), T, Dm, E, dlogits, dw_r,    \
+                                     dbias);
+  ROM_RWG_CASE(4)
+  ROM_RWG_CASE(8)
+  ROM_RWG_CASE(16)
+  ROM_RWG_CASE(32)
+  ROM_RWG_CASE(64)
+#undef ROM_RWG_CASE
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_route_probs(const void* x, bool bf16, int64_t T, int Dm, const float* w_r,

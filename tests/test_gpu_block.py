@@ -98,6 +98,8 @@ INPROJ_CASES = [
     (300, 1024, 768, 4, 2, True),
     # ragged last K block (K = 1000), partial token tiles of both 32-column halves
     (700, 1000, 512, 4, 1, False),
+    # more weight tiles than SMs (several tiles per CTA)
+    (300, 1024, 2560, 8, 2, True),
 ]
 
 
@@ -201,6 +203,9 @@ def test_host_pipeline_inproj_matches_single_call(T, Dm, N, E, k, renorm):
     (1, 256, 256, 4, 1, False),
     (50, 256, 768, 4, 2, True),
     (64, 1024, 1024, 16, 2, False),
+    # more weight tiles than SMs (several tiles per CTA), ragged K = 1000
+    (50, 1000, 5120, 4, 1, False),
+    (64, 2048, 2560, 8, 2, True),
 ])
 def test_inproj_without_dispatch_for_small_batches(T, Dm, N, E, k, renorm):
     """rom_expert_proj_dense (every expert's weights meet all tokens, the
@@ -218,3 +223,35 @@ def test_inproj_without_dispatch_for_small_batches(T, Dm, N, E, k, renorm):
     assert_close(to_np(dense), ref["S"], "bf16", "S (no dispatch)", magnitude_scaled_abs=True)
     assert_close(to_np(dense), to_np(sparse), "bf16", "no dispatch vs dispatched",
                  magnitude_scaled_abs=True)
+
+
+@pytest.mark.parametrize("dense_small", [True, False])
+def test_few_token_inproj_graph_replays_match_eager(dense_small):
+    """The few-token projection over more weight tiles than SMs, captured in a
+    CUDA graph and replayed: every replay must reproduce the eager bits."""
+    T, Dm, N, E = 64, 4096, 5120, 4  # 160 weight tiles
+    inp = make_inproj_inputs(T, Dm, N, E, seed=11, router_std=0.05)
+    x, w_r, w = (to_dev(inp["x"], "bf16"), to_dev(inp["w_r"], "f32"),
+                 weights_to_dev(inp["w"], "bf16"))
+    eager, bufs = rom.inproj_forward(x, w_r, w, k=1, renorm=False, dense_small=dense_small)
+    eager = eager.clone()
+    out = torch.empty_like(eager)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        rom.inproj_forward(x, w_r, w, k=1, renorm=False, bufs=bufs, out=out,
+                           dense_small=dense_small)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        rom.inproj_forward(x, w_r, w, k=1, renorm=False, bufs=bufs, out=out,
+                           dense_small=dense_small)
+    for _ in range(4):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert rom.rom_get_status() == 0
+        assert torch.equal(out, eager)
+    ref = orc.inproj_forward(inp["x"], inp["w_r"], inp["w"], k=1, renorm=False)
+    assert_close(to_np(eager), ref["S"], "bf16", "S (160 weight tiles)", magnitude_scaled_abs=True)
+    del g

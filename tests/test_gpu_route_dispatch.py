@@ -28,6 +28,10 @@ ROUTE_CASES = [
     (1500, 512, 16, 2, True, "bf16", 0.02),
     (1300, 256, 4, 1, False, "bf16", 0.1),
     (1200, 256, 8, 2, False, "f32", 0.05),
+    # more 128-token tiles than SMs: CTAs of the streaming router take a second
+    # tile (the weight norms come from the first)
+    (20000, 192, 16, 2, True, "bf16", 0.05),
+    (19001, 128, 4, 1, False, "bf16", 0.1),
     # small batches with 16 experts, float32 data, a 64-token decode shape
     (64, 4096, 4, 1, False, "bf16", 0.02),
     (333, 512, 16, 2, True, "f32", 0.05),
