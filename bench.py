@@ -327,20 +327,24 @@ def build_workload(torch, rom, wl, inp):
         slots = (torch.empty((R, wl.De), dtype=torch.float32, device=x.device)
                  if wl.k > 1 else None)
 
-        # a decode-sized batch takes the projection without a dispatch
+        # a decode-sized batch takes the projection without a dispatch, over
+        # the weights in the tile-major layout (packed once, here)
         dense = bf16 and wl.T <= rom.DENSE_SMALL_MAX_TOKENS
+        w_tiled = rom.pack_expert_weights(w) if dense else None
 
         def ph_route():
             if dense:
-                rom.rom_route(x, w_r, bias, wl.k, wl.renorm, bufs.topk_idx, bufs.topk_w,
-                              bufs.counts, bufs.ws)
+                # no dispatch follows: neither counts nor chunk histograms
+                rom.rom_route(x, w_r, bias, wl.k, wl.renorm, bufs.topk_idx, bufs.topk_w, None,
+                              None)
             else:
                 rom.route_and_dispatch(x, w_r, bias, wl.E, wl.k, wl.renorm, bufs)
 
         def ph_p0():
             if dense:
-                rom.rom_expert_proj_dense(rom.ROM_PROJ_INPROJ, x, w, wl.E, wl.k, bufs.topk_idx,
-                                          bufs.topk_w, out if wl.k == 1 else slots)
+                rom.rom_expert_proj_dense(rom.ROM_PROJ_INPROJ, x, w_tiled, wl.E, wl.k,
+                                          bufs.topk_idx, bufs.topk_w,
+                                          out if wl.k == 1 else slots, tiled=True)
             else:
                 rom.rom_expert_proj(rom.ROM_PROJ_INPROJ, bufs.x_sorted[:R], w, None, wl.E, wl.k,
                                     bufs.offsets, bufs.sorted_slot, bufs.topk_w,
@@ -353,11 +357,14 @@ def build_workload(torch, rom, wl, inp):
                            ("proj1", ph_p1)],
                    dominant=(ph_p0, "byte",
                              lambda counts: inproj_bytes(wl, int(np.count_nonzero(counts)))),
-                   out=out, counts=bufs.counts,
+                   out=out,
+                   counts=((lambda: torch.bincount(bufs.topk_idx.reshape(-1).long(),
+                                                   minlength=wl.E).int())
+                           if dense else bufs.counts),
                    launches=(2 if dense else 3) + (1 if wl.k > 1 else 0))
         pipe = rom.HostPipeline(wl.T, wl.Dm, wl.De, wl.E, wl.k, x.dtype, x.device)
         res["e2e"] = (pipe, lambda hx, ho: pipe.inproj_forward(hx, w_r, w, ho, renorm=wl.renorm,
-                                                                bias=bias))
+                                                                bias=bias, w_tiled=w_tiled))
     elif wl.kind == "variant":
         routers, weighted = variant_spec(wl, inp)
         d_r = {}
@@ -580,7 +587,7 @@ def measure(args, wl, world, local_rank, with_e2e):
     # host ahead of the GPU (no graph-launch latency in its duration).
     dom_fn, dom_kind, dom_work = b["dominant"]
     dom_ms = timed_loop(lambda j: dom_fn(), args.steps, 1)[:, 0]
-    counts = b["counts"].cpu().numpy()
+    counts = (b["counts"]() if callable(b["counts"]) else b["counts"]).cpu().numpy()
     t_total_ms = float(step_ms.sum())
 
     # ---------------------------------------------- e2e through host buffers
@@ -648,10 +655,14 @@ def roofline(res, peaks, src):
 
 
 def workload_config(wl, world):
+    from mixture_experts_projections_b200 import rom
     return {"workload": wl.name, "tokens": wl.T, "d_model": wl.Dm,
             ("d_out" if wl.kind == "inproj" else "d_inner"): wl.De, "experts": wl.E,
             "top_k": wl.k, "renorm": wl.renorm, "parallelism": f"replicas x{world}",
-            **({"projections": wl.variant} if wl.kind == "variant" else {})}
+            **({"projections": wl.variant} if wl.kind == "variant" else {}),
+            **({"weights": "tile-major (rom_pack_expert_weights, once, before timing)"}
+               if wl.kind == "inproj" and wl.dtype == "bf16" and wl.T <= rom.DENSE_SMALL_MAX_TOKENS
+               else {})}
 
 
 SM_COUNT = 148

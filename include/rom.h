@@ -63,6 +63,10 @@ typedef enum {
   ROM_PROJ_CONV_GATE_SLOTS = 4 /* Conv and Gate to float32 u, z slot rows for any k */
 } rom_proj;
 
+/* Flag OR'd into `proj` of rom_expert_proj_dense: the weights are in the
+ * tile-major layout written by rom_pack_expert_weights. */
+#define ROM_W_TILED 0x100
+
 typedef enum {
   ROM_COMBINE_SUM = 0,       /* out[t] = sum_j in[t*k+j]                     */
   ROM_COMBINE_GATE = 1,      /* h_t = (sum_j u_{t,j}) * SiLU(sum_j z_{t,j}) */
@@ -96,7 +100,9 @@ size_t rom_workspace_size(int64_t T, int E);
  *  counts   [E]       out, int32 per-expert slot count, or NULL (not written)
  *  ws, ws_bytes       workspace of at least rom_workspace_size(T, E) bytes;
  *                     rom_dispatch() must receive the same workspace, unchanged,
- *                     on the same stream, after this call.
+ *                     on the same stream, after this call. NULL when no
+ *                     rom_dispatch follows (rom_expert_proj_dense): the per-chunk
+ *                     histograms are then not formed.
  *
  * Precision: logits are accumulated in float32 in a fixed order together with
  * a rigorous bound on their rounding error; a token whose top-k decision is
@@ -184,9 +190,13 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
  * on the stream (the router: decode steps need no rom_dispatch) and only its
  * epilogue waits for that kernel's results.
  *
- *  proj      ROM_PROJ_INPROJ or ROM_PROJ_OUT (both weighted by r)
+ *  proj      ROM_PROJ_INPROJ or ROM_PROJ_OUT (both weighted by r), optionally
+ *            | ROM_W_TILED
  *  x         [T][K] bf16, token order (as given to rom_route)
- *  w         [E][N][K] bf16
+ *  w         [E][N][K] bf16, or with ROM_W_TILED the same weights in the
+ *            tile-major layout of rom_pack_expert_weights (which requires
+ *            K % 64 == 0); the results are identical, the tiled weights
+ *            stream as whole 16 KB blocks
  *  topk_idx, topk_w [T][k] from rom_route
  *  out       k == 1: [T][N] bf16, token order; k > 1: float32 [T*k][N] in slot
  *            order (then rom_combine(ROM_COMBINE_SUM))
@@ -196,6 +206,22 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
 int rom_expert_proj_dense(int proj, int dtype, const void* x, int64_t T, int K, const void* w,
                           int N, int E, int k, const int32_t* topk_idx, const float* topk_w,
                           void* out, void* stream);
+
+/*
+ * rom_pack_expert_weights -- a one-time copy of expert weights into the
+ * tile-major layout that rom_expert_proj_dense takes with ROM_W_TILED: the
+ * 128 x 64 weight tiles the projection's kernel reads (128 output rows, 64
+ * contraction elements) stored one after another, 16 KB each, so that every
+ * tile is one contiguous read. No counterpart in the source pages: it is a
+ * storage layout of the same W, not part of the method.
+ *  w         [E][N][K] bf16 (as for rom_expert_proj_dense)
+ *  w_tiled   out, E*N*K bf16 elements: element (e, n, c) at
+ *            ((((e * N/128 + n/128) * K/64 + c/64) * 128 + n % 128) * 64 + c % 64)
+ * Requires dtype ROM_BF16, N % 128 == 0, K % 64 == 0, 16-byte aligned
+ * pointers and w_tiled not overlapping w.
+ */
+int rom_pack_expert_weights(int dtype, const void* w, int E, int N, int K, void* w_tiled,
+                            void* stream);
 
 /*
  * rom_combine -- reduce the k slots of each token in slot order 0..k-1.

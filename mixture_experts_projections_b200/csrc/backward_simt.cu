@@ -23,6 +23,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "rom_internal.cuh"
 
@@ -265,93 +266,131 @@ __global__ void __launch_bounds__(256)
 }
 
 // Router weight gradients: dW_r[d][e] = sum_t x[t][d] dlogit[t][e] and
-// dbias[e] = sum_t dlogit[t][e], in float32. A cluster of kRwSplit CTAs owns
-// 64 features of d_model; CTA r of the cluster sums the tokens of its slice r
-// of T. The CTA walks its slice in chunks of 128 tokens: the chunk's logit
-// gradients are staged in shared memory (coalesced), and warp w takes tokens
-// 16w .. 16w+15 of the chunk, each lane two features for all experts: the 16
-// tokens' x loads are issued together, then per token and expert one packed
-// FMA updates the lane's two feature sums (the gradient row read as
-// broadcast float4s). The 8 warps' sums are added in warp order, then CTA 0
-// adds the kRwSplit partial sums in rank order through distributed shared
-// memory. The order of every sum is fixed, so the result does not depend on
-// the launch.
-constexpr int kRwFeat = 64, kRwSplit = 8, kRwChunk = 128, kRwTokPerWarp = 16;
+// dbias[e] = sum_t dlogit[t][e], in float32. A cluster of `split` CTAs (sized
+// at launch so that the grid fits the SMs in one wave) owns 64 features of
+// d_model; CTA r of the cluster sums the tokens of its slice r of T. Warp w
+// of a CTA takes the 16-token groups w, w + 8, ... of the slice on its own
+// (no block-wide barrier in the loop): each lane holds two features for all
+// experts, the group's logit gradients go through the warp's own shared
+// buffer and are read back as broadcast float4s, one packed FMA per token and
+// expert updates the lane's two sums, and the next group's x and gradient
+// loads are in flight while the current group is computed. The 8 warps' sums
+// are added in warp order, then CTA 0 of the cluster adds the `split` partial
+// sums in rank order through distributed shared memory. The order of every
+// sum is fixed for a given launch shape, so the result is deterministic.
+constexpr int kRwFeat = 64, kRwMaxSplit = 8, kRwGroup = 16;
+
+// x[da], x[da + 1] of one row (zero past d_model or for a token past the
+// slice), kept packed until use: bf16 as one 32-bit word, float32 as a pair.
+// `pair` (uniform): the two values are one aligned 4- or 8-byte load.
+__device__ __forceinline__ uint32_t load_pair(const __nv_bfloat16* row, int da, int Dm, bool ok,
+                                              bool pair) {
+  if (!ok) return 0u;
+  if (pair && da + 1 < Dm) return __ldg(reinterpret_cast<const unsigned int*>(row + da));
+  const uint32_t lo = da < Dm ? __bfloat16_as_ushort(row[da]) : 0u;
+  const uint32_t hi = da + 1 < Dm ? __bfloat16_as_ushort(row[da + 1]) : 0u;
+  return lo | (hi << 16);
+}
+__device__ __forceinline__ float2 load_pair(const float* row, int da, int Dm, bool ok, bool pair) {
+  if (!ok) return make_float2(0.f, 0.f);
+  if (pair && da + 1 < Dm) return __ldg(reinterpret_cast<const float2*>(row + da));
+  return make_float2(da < Dm ? row[da] : 0.f, da + 1 < Dm ? row[da + 1] : 0.f);
+}
+__device__ __forceinline__ float2 unpack_pair(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+__device__ __forceinline__ float2 unpack_pair(float2 v) { return v; }
 
 template <int EB, typename InT>
 __global__ void __launch_bounds__(256)
     route_wgrad_kernel(const InT* __restrict__ x, int64_t T, int Dm, int E,
                        const float* __restrict__ dl, float* __restrict__ dw_r,
-                       float* __restrict__ dbias) {
-  static_assert(kRwChunk * EB >= kRwFeat * EB && kRwChunk == 8 * kRwTokPerWarp, "layout");
-  constexpr int kGroups = 256 / EB;  // bias: token groups per expert
-  __shared__ __align__(16) float s_dl[kRwChunk][EB];  // after the loop: the partial sums
-  __shared__ float s_bsum[256];
+                       float* __restrict__ dbias, bool pair) {
+  using Packed = typename std::conditional<std::is_same<InT, float>::value, float2, uint32_t>::type;
+  constexpr int kPer = kRwGroup * EB / 32;  // gradient values a lane stages per group
+  static_assert(kPer >= 1 && 8 * kRwGroup >= kRwFeat, "layout");
+  __shared__ __align__(16) float s_dl[8][kRwGroup][EB];  // after the loop: s_part
+  __shared__ float s_bsum[8][EB];
   __shared__ float s_bias[EB];
-  float(*s_part)[EB] = reinterpret_cast<float(*)[EB]>(&s_dl[0][0]);  // [kRwFeat][EB]
+  float(*s_part)[kRwFeat + 1] = reinterpret_cast<float(*)[kRwFeat + 1]>(&s_dl[0][0][0]);  // [EB][65]
+  static_assert(EB * (kRwFeat + 1) <= 8 * kRwGroup * EB, "partials fit the staging buffer");
   cg::cluster_group cluster = cg::this_cluster();
+  const int split = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int d0 = (blockIdx.x / kRwSplit) * kRwFeat;
-  const int da = d0 + 2 * lane, db = da + 1;  // this lane's features
-  const bool bias_cluster = blockIdx.x / kRwSplit == 0 && dbias != nullptr;
-  const int64_t per = (T + kRwSplit - 1) / kRwSplit;
+  const int d0 = (blockIdx.x / split) * kRwFeat;
+  const int da = d0 + 2 * lane;  // this lane's features da, da + 1
+  const bool bias_cluster = blockIdx.x / split == 0 && dbias != nullptr;
+  const int64_t per = (T + split - 1) / split;
   const int64_t ta = rank * per, tb = ta + per < T ? ta + per : T;
   float2 acc[EB];
 #pragma unroll
   for (int e = 0; e < EB; ++e) acc[e] = make_float2(0.f, 0.f);
-  float bacc = 0.f;  // bias: expert tid % EB over token group tid / EB
-  for (int64_t t0 = ta; t0 < tb; t0 += kRwChunk) {
-    const int nt = static_cast<int>(tb - t0 < kRwChunk ? tb - t0 : kRwChunk);
-    // x of this warp's 16 tokens first: their loads overlap the staging
-    float2 xv[kRwTokPerWarp];
+  float bacc = 0.f;  // bias (lane < EB): expert `lane` over this warp's tokens
+  float(*buf)[EB] = s_dl[warp];
+
+  // loads of one group (tokens g0 .. g0+15 of the slice) into registers
+  Packed xn[kRwGroup];
+  float dn[kPer];
+  auto fetch = [&](int64_t g0) {
+    const InT* row = x + g0 * Dm;
 #pragma unroll
-    for (int u = 0; u < kRwTokPerWarp; ++u) {
-      const int r = kRwTokPerWarp * warp + u;
-      const InT* row = x + (t0 + r) * Dm;
-      const bool ok = r < nt;
-      xv[u].x = (ok && da < Dm) ? static_cast<float>(row[da]) : 0.f;
-      xv[u].y = (ok && db < Dm) ? static_cast<float>(row[db]) : 0.f;
-    }
-    for (int i = tid; i < kRwChunk * EB; i += 256) {
-      const int r = i / EB, e = i - r * EB;
-      s_dl[r][e] = (r < nt && e < E) ? dl[(t0 + r) * E + e] : 0.f;
-    }
-    __syncthreads();
+    for (int u = 0; u < kRwGroup; ++u, row += Dm) xn[u] = load_pair(row, da, Dm, g0 + u < tb, pair);
 #pragma unroll
-    for (int u = 0; u < kRwTokPerWarp; ++u) {
-      const float4* g4 = reinterpret_cast<const float4*>(&s_dl[kRwTokPerWarp * warp + u][0]);
+    for (int j = 0; j < kPer; ++j) {
+      const int i = lane + 32 * j, u = i / EB, e = i - u * EB;
+      const int64_t t = g0 + u;
+      dn[j] = (t < tb && e < E) ? __ldg(dl + t * E + e) : 0.f;
+    }
+  };
+  int64_t g0 = ta + static_cast<int64_t>(warp) * kRwGroup;
+  if (g0 < tb) fetch(g0);
+  for (; g0 < tb; g0 += 8 * kRwGroup) {
+    Packed xc[kRwGroup];
+#pragma unroll
+    for (int u = 0; u < kRwGroup; ++u) xc[u] = xn[u];
+    __syncwarp();  // the previous group's reads of buf are done
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) (&buf[0][0])[lane + 32 * j] = dn[j];
+    __syncwarp();
+    if (g0 + 8 * kRwGroup < tb) fetch(g0 + 8 * kRwGroup);  // in flight during the FMAs
+#pragma unroll
+    for (int u = 0; u < kRwGroup; ++u) {
+      const float2 xv = unpack_pair(xc[u]);
+      const float4* g4 = reinterpret_cast<const float4*>(&buf[u][0]);
 #pragma unroll
       for (int e4 = 0; e4 < EB / 4; ++e4) {
         const float4 g = g4[e4];
-        acc[4 * e4] = __ffma2_rn(xv[u], make_float2(g.x, g.x), acc[4 * e4]);
-        acc[4 * e4 + 1] = __ffma2_rn(xv[u], make_float2(g.y, g.y), acc[4 * e4 + 1]);
-        acc[4 * e4 + 2] = __ffma2_rn(xv[u], make_float2(g.z, g.z), acc[4 * e4 + 2]);
-        acc[4 * e4 + 3] = __ffma2_rn(xv[u], make_float2(g.w, g.w), acc[4 * e4 + 3]);
+        acc[4 * e4] = __ffma2_rn(xv, make_float2(g.x, g.x), acc[4 * e4]);
+        acc[4 * e4 + 1] = __ffma2_rn(xv, make_float2(g.y, g.y), acc[4 * e4 + 1]);
+        acc[4 * e4 + 2] = __ffma2_rn(xv, make_float2(g.z, g.z), acc[4 * e4 + 2]);
+        acc[4 * e4 + 3] = __ffma2_rn(xv, make_float2(g.w, g.w), acc[4 * e4 + 3]);
       }
     }
     if (bias_cluster)
-      for (int r = tid / EB; r < kRwChunk; r += kGroups) bacc += s_dl[r][tid % EB];
-    __syncthreads();
+      for (int e = lane; e < EB; e += 32)
+#pragma unroll
+        for (int u = 0; u < kRwGroup; ++u) bacc += buf[u][e];
   }
-  // the warps' sums, added in warp order
+  __syncthreads();  // every warp is done with its staging buffer
+  // the warps' sums, added in warp order (s_part[e][f]: lanes 2 floats apart)
 #pragma unroll 1
   for (int w = 0; w < 8; ++w) {
     if (warp == w) {
 #pragma unroll
       for (int e = 0; e < EB; ++e) {
-        s_part[2 * lane][e] = (w == 0) ? acc[e].x : s_part[2 * lane][e] + acc[e].x;
-        s_part[2 * lane + 1][e] = (w == 0) ? acc[e].y : s_part[2 * lane + 1][e] + acc[e].y;
+        s_part[e][2 * lane] = (w == 0) ? acc[e].x : s_part[e][2 * lane] + acc[e].x;
+        s_part[e][2 * lane + 1] = (w == 0) ? acc[e].y : s_part[e][2 * lane + 1] + acc[e].y;
       }
     }
     __syncthreads();
   }
   if (bias_cluster) {
-    s_bsum[tid] = bacc;
+    if (lane < EB) s_bsum[warp][lane] = bacc;
     __syncthreads();
     if (tid < EB) {
-      float v = s_bsum[tid];
-      for (int g = 1; g < kGroups; ++g) v += s_bsum[g * EB + tid];
+      float v = s_bsum[0][tid];
+      for (int w = 1; w < 8; ++w) v += s_bsum[w][tid];
       s_bias[tid] = v;
     }
   }
@@ -360,13 +399,13 @@ __global__ void __launch_bounds__(256)
     for (int i = tid; i < kRwFeat * E; i += 256) {
       const int ff = i / E, e = i - ff * E;
       float v = 0.f;
-      for (int rr = 0; rr < kRwSplit; ++rr) v += cluster.map_shared_rank(&s_part[ff][e], rr)[0];
+      for (int rr = 0; rr < split; ++rr) v += cluster.map_shared_rank(&s_part[e][ff], rr)[0];
       if (d0 + ff < Dm) dw_r[static_cast<int64_t>(d0 + ff) * E + e] = v;
     }
     if (bias_cluster)
       for (int e = tid; e < E; e += 256) {
         float v = 0.f;
-        for (int rr = 0; rr < kRwSplit; ++rr) v += cluster.map_shared_rank(&s_bias[e], rr)[0];
+        for (int rr = 0; rr < split; ++rr) v += cluster.map_shared_rank(&s_bias[e], rr)[0];
         dbias[e] = v;
       }
   }
@@ -401,28 +440,47 @@ cudaError_t launch_gate_bwd(const float* uz, const float* gp, int64_t T, int k, 
 cudaError_t launch_route_wgrad(const void* x, bool bf16, int64_t T, int Dm, int E,
                                const float* dlogits, float* dw_r, float* dbias,
                                cudaStream_t stream) {
+  // experts rounded up to 4, 8, 16, 32 or 64 (the padded columns are zero)
+  const int eb = E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64;
+  // Token split (the cluster size): as many CTAs as are resident on the SMs
+  // at once (one wave), at most kRwMaxSplit per 64-feature block.
+  const int blocks = (Dm + kRwFeat - 1) / kRwFeat;
+  // x[da], x[da + 1] as one aligned load: even d_model and an aligned base
+  const size_t esz = bf16 ? 2 : 4;
+  const bool pair = Dm % 2 == 0 && (reinterpret_cast<uintptr_t>(x) % (2 * esz)) == 0;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kRwSplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((Dm + kRwFeat - 1) / kRwFeat * kRwSplit), 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // experts rounded up to 4, 8, 16, 32 or 64 (the padded columns are zero)
-  const int eb = E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : E <= 32 ? 32 : 64;
-#define ROM_RWG_CASE(EBV)                                                                      \
-  if (eb == EBV)                                                                               \
-    return bf16 ? cudaLaunchKernelEx(&cfg, route_wgrad_kernel<EBV, __nv_bfloat16>,             \
-                                     static_cast<const __nv_bfloat16*>(x), T, Dm, E, dlogits,  \
-                                     dw_r, dbias)                                              \
-                : cudaLaunchKernelEx(&cfg, route_wgrad_kernel<EBV, float>,                     \
-                                     static_cast<const float*>(x), T, Dm, E, dlogits, dw_r,    \
-                                     dbias);
+  auto go = [&](auto kern, auto xp) -> cudaError_t {
+    // the largest split whose clusters (one per feature block) are all
+    // resident at once
+    int split = 1;
+    for (int sp = kRwMaxSplit; sp > 1; --sp) {
+      attr[0].val.clusterDim.x = static_cast<unsigned>(sp);
+      cfg.gridDim = dim3(static_cast<unsigned>(blocks * sp), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= blocks) {
+        split = sp;
+        break;
+      }
+    }
+    (void)cudaGetLastError();  // a refused query leaves no error behind
+    attr[0].val.clusterDim.x = static_cast<unsigned>(split);
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks * split), 1, 1);
+    return cudaLaunchKernelEx(&cfg, kern, xp, T, Dm, E, dlogits, dw_r, dbias, pair);
+  };
+#define ROM_RWG_CASE(EBV)                                                              \
+  if (eb == EBV)                                                                       \
+    return bf16 ? go(route_wgrad_kernel<EBV, __nv_bfloat16>,                           \
+                     static_cast<const __nv_bfloat16*>(x))                             \
+                : go(route_wgrad_kernel<EBV, float>, static_cast<const float*>(x));
   ROM_RWG_CASE(4)
   ROM_RWG_CASE(8)
   ROM_RWG_CASE(16)

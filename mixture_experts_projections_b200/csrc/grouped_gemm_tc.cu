@@ -64,6 +64,9 @@ struct Params {
   int* status;
   // the dense small-batch in-projection: every token's experts (else null)
   const int32_t* topk_idx;
+  // dense small-batch kernel: weights in the tile-major layout
+  // [E][N/128][K/64][128][64] (one 16 KB block per weight tile)
+  int w_tiled;
 };
 
 // u * SiLU(z) = u * z / (1 + e^-z), with the fast exp and divide intrinsics:
@@ -565,7 +568,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sa = smem + stage * SW_STAGE_BYTES;
           mbar_arrive_expect_tx(&ctl.full[stage], SW_STAGE_BYTES);
-          tma_load_3d(sa, &tmW, &ctl.full[stage], kb * BK, n0, e);
+          if (kDense && p.w_tiled)
+            tma_load_5d(sa, &tmW, &ctl.full[stage], 0, 0, kb, w_blk, e);
+          else
+            tma_load_3d(sa, &tmW, &ctl.full[stage], kb * BK, n0, e);
           tma_load_2d(sa + SW_A_BYTES, &tmX, &ctl.full[stage], kb * BK, r0);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -865,14 +871,34 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
 
 cudaError_t launch_tc_dense_small(int mode, const void* x, int64_t T, int K, const void* w, int N,
                                   int E, int k, const int32_t* topk_idx, const float* topk_w,
-                                  void* out, int* status, cudaStream_t stream) {
+                                  void* out, bool w_tiled, int* status, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   if (T > SW_BN || N % SW_BM != 0 || K % 8 != 0 || E > kMaxExperts) return cudaErrorInvalidValue;
+  if (w_tiled && K % BK != 0) return cudaErrorInvalidValue;
   CUtensorMap tw, tx;
-  if (!make_map(&tw, w, K, N, E, SW_BM)) return cudaErrorInvalidValue;
+  if (w_tiled) {
+    // [E][N/128][K/64][128][64]: a box of one whole 128 x 64 tile (16 KB)
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    const cuuint64_t kb = static_cast<cuuint64_t>(K / BK), nt = static_cast<cuuint64_t>(N / SW_BM);
+    const cuuint64_t tile_bytes = static_cast<cuuint64_t>(SW_BM) * BK * 2;
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(BK), static_cast<cuuint64_t>(SW_BM), kb, nt,
+                          static_cast<cuuint64_t>(E)};
+    cuuint64_t strides[4] = {static_cast<cuuint64_t>(BK) * 2, tile_bytes, tile_bytes * kb,
+                             tile_bytes * kb * nt};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(SW_BM), 1, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (fn(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(w), dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else if (!make_map(&tw, w, K, N, E, SW_BM)) {
+    return cudaErrorInvalidValue;
+  }
   if (!make_map(&tx, x, K, T, 0, SW_BN)) return cudaErrorInvalidValue;
   Params p{};
   p.topk_idx = topk_idx;
+  p.w_tiled = w_tiled ? 1 : 0;
   p.topk_w = topk_w;
   p.out = out;
   p.R = T;  // token rows (in token order)

@@ -122,7 +122,7 @@ int rom_route(const void* x, int dtype, int64_t T, int Dm, const float* w_r, con
   if (T > 0) {
     if (!x || !w_r || !topk_idx || !topk_w) return ROM_ERR_INVALID_ARG;
     if (!aligned16(x)) return ROM_ERR_UNSUPPORTED;
-    if (!ws || ws_bytes < rom_workspace_size(T, E)) return ROM_ERR_WORKSPACE;
+    if (ws && ws_bytes < rom_workspace_size(T, E)) return ROM_ERR_WORKSPACE;
   }
   if (counts) {
     const cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
@@ -204,12 +204,15 @@ int rom_expert_proj(int proj, int dtype, const void* a_sorted, int64_t R, int K,
 int rom_expert_proj_dense(int proj, int dtype, const void* x, int64_t T, int K, const void* w,
                           int N, int E, int k, const int32_t* topk_idx, const float* topk_w,
                           void* out, void* stream) {
+  const bool w_tiled = (proj & ROM_W_TILED) != 0;
+  proj &= ~ROM_W_TILED;
   if (proj != ROM_PROJ_OUT && proj != ROM_PROJ_INPROJ) return ROM_ERR_INVALID_ARG;
   if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
   if (T < 0 || K <= 0 || N <= 0 || E < 1 || E > rom::kMaxExperts || k < 1 || k > E ||
       k > rom::kMaxTopK)
     return ROM_ERR_INVALID_ARG;
   if (dtype != ROM_BF16 || T > 64 || K % 8 != 0 || N % 128 != 0) return ROM_ERR_UNSUPPORTED;
+  if (w_tiled && K % 64 != 0) return ROM_ERR_UNSUPPORTED;
   if (T == 0) return ROM_OK;
   if (!x || !w || !topk_idx || !topk_w || !out) return ROM_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return ROM_ERR_UNSUPPORTED;
@@ -217,7 +220,21 @@ int rom_expert_proj_dense(int proj, int dtype, const void* x, int64_t T, int K, 
   if (!st) return ROM_ERR_CUDA;
   return rom::to_status(rom::launch_tc_dense_small(
       k == 1 ? rom::kEpiScaleToken : rom::kEpiScaleSlots, x, T, K, w, N, E, k, topk_idx, topk_w,
-      out, st, static_cast<cudaStream_t>(stream)));
+      out, w_tiled, st, static_cast<cudaStream_t>(stream)));
+}
+
+int rom_pack_expert_weights(int dtype, const void* w, int E, int N, int K, void* w_tiled,
+                            void* stream) {
+  if (dtype != ROM_F32 && dtype != ROM_BF16) return ROM_ERR_INVALID_ARG;
+  if (E < 1 || N <= 0 || K <= 0) return ROM_ERR_INVALID_ARG;
+  if (dtype != ROM_BF16 || N % 128 != 0 || K % 64 != 0) return ROM_ERR_UNSUPPORTED;
+  if (!w || !w_tiled) return ROM_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(w_tiled)) return ROM_ERR_UNSUPPORTED;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(w), b = reinterpret_cast<uintptr_t>(w_tiled);
+  const uintptr_t bytes = static_cast<uintptr_t>(E) * N * K * 2;
+  if (a < b + bytes && b < a + bytes) return ROM_ERR_INVALID_ARG;  // overlapping
+  return rom::to_status(rom::launch_pack_expert_weights(w, E, N, K, w_tiled,
+                                                        static_cast<cudaStream_t>(stream)));
 }
 
 int rom_combine(int mode, int dtype, const void* in, int64_t T, int k, int N,

@@ -85,7 +85,10 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
 // order, the router's topk_idx / topk_w read only by the epilogue.
 cudaError_t launch_tc_dense_small(int mode, const void* x, int64_t T, int K, const void* w, int N,
                                   int E, int k, const int32_t* topk_idx, const float* topk_w,
-                                  void* out, int* status, cudaStream_t stream);
+                                  void* out, bool w_tiled, int* status, cudaStream_t stream);
+// [E][N][K] bf16 -> the tile-major [E][N/128][K/64][128][64] (pack.cu)
+cudaError_t launch_pack_expert_weights(const void* w, int E, int N, int K, void* w_tiled,
+                                       cudaStream_t stream);
 
 // float32 SIMT grouped GEMM (same semantics as the tensor-core one).
 cudaError_t launch_simt_grouped_gemm(int mode, const float* a_sorted, int64_t R, int K,

@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(kRouterThreads)
     }
     __syncthreads();
     for (int e = tid; e < E; e += kRouterThreads) {
-      chunk_hist[c * E + e] = s_hist[e];
+      if (chunk_hist) chunk_hist[c * E + e] = s_hist[e];
       if (counts && s_hist[e]) atomicAdd(counts + e, s_hist[e]);
     }
     __syncthreads();

@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int j = 0; j < k; ++j) {
       topk_idx[t * k + j] = sel[j];
       topk_w[t * k + j] = expf(s_l[sel[j]] - m) / den;
-      atomicAdd(chunk_hist + chunk * EB + sel[j], 1);
+      if (chunk_hist) atomicAdd(chunk_hist + chunk * EB + sel[j], 1);
       if (counts) atomicAdd(counts + sel[j], 1);
     }
   }
@@ -227,9 +227,11 @@ cudaError_t launch_eb(const void* x, int64_t T, int Dm, const float* w_r, const 
                       int k, int renorm, int32_t* topk_idx, float* topk_w, int32_t* counts,
                       int32_t* chunk_hist, cudaStream_t stream) {
   constexpr int kPiece = 16 / static_cast<int>(sizeof(InT));
-  cudaError_t err =
-      cudaMemsetAsync(chunk_hist, 0, sizeof(int32_t) * num_chunks(T) * EB, stream);
-  if (err != cudaSuccess) return err;
+  if (chunk_hist) {
+    const cudaError_t err =
+        cudaMemsetAsync(chunk_hist, 0, sizeof(int32_t) * num_chunks(T) * EB, stream);
+    if (err != cudaSuccess) return err;
+  }
   // Longest rounding chain of a logit: the features of one thread, the warp
   // butterfly, the sum over the warps, the bias (+1 spare); 1 % slack covers
   // the norms.

@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence_block();
       for (int e = lane; e < E; e += 32) {
         const int v = atomicExch(&ctl.hist[e], 0);
-        chunk_hist[tile * E + e] = v;
+        if (chunk_hist) chunk_hist[tile * E + e] = v;
         if (counts && v) atomicAdd(counts + e, v);
       }
       if (lane == 0) ctl.done = 0;

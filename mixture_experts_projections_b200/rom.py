@@ -24,6 +24,7 @@ ROM_F32, ROM_BF16 = 0, 1
 ROM_PROJ_CONV_GATE, ROM_PROJ_OUT, ROM_PROJ_INPROJ, ROM_PROJ_SLOTS, ROM_PROJ_CONV_GATE_SLOTS = \
     0, 1, 2, 3, 4
 ROM_COMBINE_SUM, ROM_COMBINE_GATE, ROM_COMBINE_GATE_DENSE = 0, 1, 2
+ROM_W_TILED = 0x100  # rom_expert_proj_dense: weights in the tile-major layout
 
 # Every exported symbol of include/rom.h with its ctypes signature.
 _P = ctypes.c_void_p
@@ -38,6 +39,7 @@ SIGNATURES = {
     "rom_expert_proj": (_I, [_I, _I, _P, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "rom_combine": (_I, [_I, _I, _P, _L, _I, _I, _P, _P, _P]),
     "rom_expert_proj_dense": (_I, [_I, _I, _P, _L, _I, _P, _I, _I, _I, _P, _P, _P, _P]),
+    "rom_pack_expert_weights": (_I, [_I, _P, _I, _I, _I, _P, _P]),
     "rom_get_status": (_I, [_P, ctypes.POINTER(ctypes.c_int32)]),
     "rom_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "rom_route_dispatch_noalloc": (_I, [_P, _I, _L, _I, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P,
@@ -147,12 +149,27 @@ def rom_expert_proj(proj, a_sorted, w0, w1, E, k, offsets, sorted_slot, topk_w, 
         "rom_expert_proj")
 
 
-def rom_expert_proj_dense(proj, x, w, E, k, topk_idx, topk_w, out, stream=None):
+def rom_expert_proj_dense(proj, x, w, E, k, topk_idx, topk_w, out, stream=None, tiled=False):
+    """``tiled``: ``w`` holds the weights in the tile-major layout of
+    pack_expert_weights (the same [E, N, K] shape and values, stored by tile)."""
     T, K = x.shape
     N = w.shape[1]
     _check(load_library().rom_expert_proj_dense(
-        proj, _dtype_code(x), _ptr(x), T, K, _ptr(w), N, E, k, _ptr(topk_idx), _ptr(topk_w),
-        _ptr(out), _stream(stream)), "rom_expert_proj_dense")
+        proj | (ROM_W_TILED if tiled else 0), _dtype_code(x), _ptr(x), T, K, _ptr(w), N, E, k,
+        _ptr(topk_idx), _ptr(topk_w), _ptr(out), _stream(stream)), "rom_expert_proj_dense")
+
+
+def pack_expert_weights(w, stream=None):
+    """A copy of the expert weights w [E, N, K] (bf16) in the tile-major layout
+    (each 128 x 64 weight tile one contiguous 16 KB block) that
+    rom_expert_proj_dense reads with ``tiled=True``. Returned with the shape
+    [E, N, K]; its elements are in tile order, not row order."""
+    _need(w, "w")
+    E, N, K = w.shape
+    out = torch.empty_like(w)
+    _check(load_library().rom_pack_expert_weights(_dtype_code(w), _ptr(w), E, N, K, _ptr(out),
+                                                  _stream(stream)), "rom_pack_expert_weights")
+    return out
 
 
 # Few tokens: the routed projection reads x in token order and needs no
@@ -380,12 +397,15 @@ def block_forward(x, w_r, bias, w_conv, w_gate, w_out, k, renorm=False, bufs=Non
 
 
 def inproj_forward(x, w_r, w, k=1, renorm=False, bias=None, bufs=None, out=None, slots=None,
-                   stream=None, dense_small=True):
+                   stream=None, dense_small=True, w_tiled=None):
     """Swimba routed in-projection: s_t = sum_j r_{t,j} x_t W_{S_j} (W as [E, N, Dm]).
 
     A bf16 batch of at most DENSE_SMALL_MAX_TOKENS tokens (a decode step)
     takes the projection without a dispatch (rom_expert_proj_dense) unless
-    ``dense_small`` is False."""
+    ``dense_small`` is False; the router then forms neither the per-expert
+    counts nor the per-chunk histograms (``bufs.counts`` is left as it was),
+    which only a dispatch needs. ``w_tiled`` (pack_expert_weights(w)), when
+    given, is what that path reads instead of ``w``."""
     T, Dm = x.shape
     E, N, _ = w.shape
     R = T * k
@@ -394,16 +414,17 @@ def inproj_forward(x, w_r, w, k=1, renorm=False, bias=None, bufs=None, out=None,
     if dense_small and x.dtype == torch.bfloat16 and 0 < T <= DENSE_SMALL_MAX_TOKENS:
         if bufs is None:
             bufs = RoutingBuffers(T, Dm, E, k, x.dtype, x.device)
-        rom_route(x, w_r, bias, k, renorm, bufs.topk_idx, bufs.topk_w, bufs.counts, bufs.ws,
-                  stream)
+        rom_route(x, w_r, bias, k, renorm, bufs.topk_idx, bufs.topk_w, None, None, stream)
+        wd = w if w_tiled is None else w_tiled
+        tiled = w_tiled is not None
         if k == 1:
-            rom_expert_proj_dense(ROM_PROJ_INPROJ, x, w, E, k, bufs.topk_idx, bufs.topk_w, out,
-                                  stream)
+            rom_expert_proj_dense(ROM_PROJ_INPROJ, x, wd, E, k, bufs.topk_idx, bufs.topk_w, out,
+                                  stream, tiled)
         else:
             if slots is None:
                 slots = torch.empty((R, N), dtype=torch.float32, device=x.device)
-            rom_expert_proj_dense(ROM_PROJ_INPROJ, x, w, E, k, bufs.topk_idx, bufs.topk_w, slots,
-                                  stream)
+            rom_expert_proj_dense(ROM_PROJ_INPROJ, x, wd, E, k, bufs.topk_idx, bufs.topk_w, slots,
+                                  stream, tiled)
             rom_combine(ROM_COMBINE_SUM, _dtype_code(x), slots, T, k, N, None, out, stream)
         return out, bufs
     rb = route_and_dispatch(x, w_r, bias, E, k, renorm, bufs, stream)
@@ -805,7 +826,7 @@ class HostPipeline:
         self._launch(key, T, body)
         return out_host
 
-    def inproj_forward(self, x_host, w_r, w, out_host, renorm=False, bias=None):
+    def inproj_forward(self, x_host, w_r, w, out_host, renorm=False, bias=None, w_tiled=None):
         """x_host [T, Dm], out_host [T, N_out]: pinned host tensors."""
         T = x_host.shape[0]
         for a, b in self._chunks(T):
@@ -819,10 +840,12 @@ class HostPipeline:
             bufs = self.bufs[j] if b - a == self.chunk else self._tail[b - a]
             od = self.out[j][: b - a]
             sl = None if self.slots[j] is None else self.slots[j][: (b - a) * self.k]
-            inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s)
+            inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s,
+                           w_tiled=w_tiled)
             out_host[a:b].copy_(od, non_blocking=True)
 
         key = ("inproj", T, x_host.data_ptr(), out_host.data_ptr(), w_r.data_ptr(), w.data_ptr(),
-               0 if bias is None else bias.data_ptr(), bool(renorm))
+               0 if bias is None else bias.data_ptr(), bool(renorm),
+               0 if w_tiled is None else w_tiled.data_ptr())
         self._launch(key, T, body)
         return out_host

@@ -61,7 +61,8 @@ FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced by these 
 @pytest.mark.parametrize("kw,code", [
     (dict(dtype=7), 1), (dict(E=0), 1), (dict(E=65), 1), (dict(k=9, E=16), 1), (dict(k=3, E=2), 1),
     (dict(renorm=2), 1), (dict(Dm=0), 1), (dict(T=-1), 1), (dict(Dm=12), 2), (dict(x=None), 1),
-    (dict(ws=None), 3), (dict(ws_bytes=4), 3), (dict(x=ctypes.c_void_p((1 << 20) + 2)), 2),
+    # a NULL workspace is accepted (no chunk histograms); a short one is not
+    (dict(ws_bytes=4), 3), (dict(x=ctypes.c_void_p((1 << 20) + 2)), 2),
 ])
 def test_route_rejects_bad_arguments(lib, kw, code):
     a = dict(x=FAKE, dtype=1, T=256, Dm=64, w_r=FAKE, bias=None, E=8, k=1, renorm=0,
@@ -254,3 +255,28 @@ def test_expert_proj_dense_rejects_bad_arguments(lib, kw, code):
              topk_w=FAKE, out=FAKE, stream=None)
     a.update(kw)
     assert lib.rom_expert_proj_dense(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    # the tile-major weights (ROM_W_TILED) need whole 64-element K blocks
+    (dict(proj=2 | 0x100, K=96), 2), (dict(proj=1 | 0x100, K=72), 2), (dict(proj=0 | 0x100), 1),
+    (dict(proj=2 | 0x200), 1),
+])
+def test_expert_proj_dense_tiled_flag(lib, kw, code):
+    a = dict(proj=2, dtype=1, x=FAKE, T=64, K=64, w=FAKE, N=256, E=4, k=1, topk_idx=FAKE,
+             topk_w=FAKE, out=FAKE, stream=None)
+    a.update(kw)
+    assert lib.rom_expert_proj_dense(*a.values()) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), 1), (dict(E=0), 1), (dict(N=0), 1), (dict(K=-64), 1),
+    (dict(dtype=0), 2), (dict(N=192), 2), (dict(K=96), 2), (dict(w=None), 1),
+    (dict(w_tiled=ctypes.c_void_p((1 << 22) + 8)), 2),
+    # the copy must not overlap its source
+    (dict(w_tiled=ctypes.c_void_p((1 << 20) + 4096)), 1),
+])
+def test_pack_expert_weights_rejects_bad_arguments(lib, kw, code):
+    a = dict(dtype=1, w=FAKE, E=2, N=128, K=64, w_tiled=ctypes.c_void_p(1 << 22), stream=None)
+    a.update(kw)
+    assert lib.rom_pack_expert_weights(*a.values()) == code

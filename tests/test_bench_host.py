@@ -67,3 +67,14 @@ def test_core_roofline_counts_one_exp_per_state_update():
     assert r["achieved"] == pytest.approx(16384 * 4096 * 16 / 1e-3 / 1e9)
     assert r["peak"] == pytest.approx(148 * 16 * 1965e6 / 1e9)
     assert r["bound"] == "alu" and 0 < r["frac"] < 1
+
+
+def test_workload_config_of_every_workload():
+    """The config dict each JSON line carries: the workload's name and sizes;
+    the decode-sized in-projection says its weights are tile-major."""
+    for name, wl in WORKLOADS.items():
+        cfg = bench.workload_config(wl, 1)
+        assert cfg["workload"] == name and cfg["tokens"] == wl.T and cfg["experts"] == wl.E
+        assert cfg["parallelism"] == "replicas x1"
+        tiled = wl.kind == "inproj" and wl.dtype == "bf16" and wl.T <= 64
+        assert ("weights" in cfg) == tiled, name
