@@ -93,20 +93,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 // Epilogue of one accumulator tile for one warp: thread i reads TMEM lane
 // t_row.lane + i, i.e. sorted row `prow` (stored only when `valid`), output
-// columns n0 .. n0 + (128 for the gate modes, 256 otherwise) - 1. The
+// columns n0 .. n0 + w - 1 (w = 128 for the gate modes, whose z columns
+// follow the w u columns in TMEM, 256 otherwise; half of that for the half
+// tiles of a last wave). The
 // float32 outputs (per-slot partials) go row by row through the warp's
 // staging tile `stg` (row-coalesced stores); the bf16 rows, half as wide,
 // are stored directly in 16-byte pieces, which measured faster for them.
 template <int MODE>
 __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, bool valid,
-                                              int64_t prow, int n0, float* stg) {
+                                              int64_t prow, int n0, int w, float* stg) {
   if (MODE == kEpiGateH) {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < w / 32; ++c) {
       uint32_t u[32], z[32];
       tmem_ld32(t_row + c * 32, u);
-      tmem_ld32(t_row + 128 + c * 32, z);
+      tmem_ld32(t_row + w + c * 32, z);
       tmem_ld_wait();
       if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(out + prow * p.N + n0 + c * 32);
@@ -129,10 +131,10 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
     float* out = static_cast<float*>(p.out);
     const int64_t slot = valid ? slot_of(p, prow) : 0;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < w / 32; ++c) {
       uint32_t u[32], z[32];
       tmem_ld32(t_row + c * 32, u);
-      tmem_ld32(t_row + 128 + c * 32, z);
+      tmem_ld32(t_row + w + c * 32, z);
       tmem_ld_wait();
       float f[32];
 #pragma unroll
@@ -147,7 +149,7 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t t_row, b
     // no routing weights passed: r = 1
     const float r = valid ? (p.topk_w ? p.topk_w[slot] : 1.f) : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < w / 32; ++c) {
       if (n0 + c * 32 >= p.N) break;  // partial last tile (N % 256 == 128)
       uint32_t a[32];
       tmem_ld32(t_row + c * 32, a);
@@ -233,7 +235,9 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1, const Params p) {
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ CUtensorMap tmB0h,
+                        const __grid_constant__ CUtensorMap tmB1h, const Params p) {
   constexpr bool kGate = (MODE == kEpiGateH || MODE == kEpiGateSlots);
   constexpr int kTileN = kGate ? 128 : 256;  // output columns per tile
   constexpr int P_STAGES = PairGeo<MODE>::kStages;
@@ -295,21 +299,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     n_blk = local / ctl.mt[e];
     m_blk = local - n_blk * ctl.mt[e];
   };
+  // Work items of this pair: its whole tiles pair, pair + npairs, ... of the
+  // full waves, then its item of the last wave. When the last wave holds at
+  // most npairs / 2 tiles, each of them is cut into two halves of N / 2
+  // columns (pair 2i and 2i + 1 take tile i's halves), so that wave keeps
+  // every pair busy for half a tile's time instead of some pairs for a
+  // whole one. half: -1 for a whole tile, else 0 or 1.
+  const int full_waves = total / npairs;
+  const int rem = total - full_waves * npairs;
+  const bool halve = rem > 0 && 2 * rem <= npairs;
+  auto item = [&](int j, int& tile, int& half) -> bool {
+    if (j < full_waves) {
+      tile = pair + j * npairs;
+      half = -1;
+      return true;
+    }
+    if (j > full_waves) return false;
+    if (halve) {
+      if (pair >= 2 * rem) return false;
+      tile = full_waves * npairs + pair / 2;
+      half = pair & 1;
+      return true;
+    }
+    if (pair >= rem) return false;
+    tile = full_waves * npairs + pair;
+    half = -1;
+    return true;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
       const CUtensorMap* tmB = (kGate && !leader) ? &tmB1 : &tmB0;
+      const CUtensorMap* tmBh = (kGate && !leader) ? &tmB1h : &tmB0h;
       const uint32_t full0 = mapa_shared(smem_u32(&ctl.full[0]), 0);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;
       bool ok = true;
-      for (int tile = pair; tile < total && ok; tile += npairs) {
+      int tile, half;
+      for (int j = 0; ok && item(j, tile, half); ++j) {
         int e, m_blk, n_blk;
         coords(tile, e, m_blk, n_blk);
         const int row0 = ctl.off[e] + m_blk * PM + static_cast<int>(rank) * BM;
-        const int brow0 = kGate ? n_blk * 128 : n_blk * 256 + static_cast<int>(rank) * 128;
+        // B rows of this CTA: whole tile 128 (Conv+Gate: the tile's 128 W_in
+        // or W_g rows; Out: its half of the 256 columns), half tile 64
+        const int r = static_cast<int>(rank);
+        const int brow0 = half < 0 ? (kGate ? n_blk * 128 : n_blk * 256 + r * 128)
+                                   : (kGate ? n_blk * 128 + half * 64
+                                            : n_blk * 256 + half * 128 + r * 64);
+        const CUtensorMap* mb = half < 0 ? tmB : tmBh;
+        const uint32_t bytes =
+            half < 0 ? 2u * P_STAGE_BYTES : 2u * (P_A_BYTES + P_B_BYTES / 2);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -317,9 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sa = smem + stage * P_STAGE_BYTES;
           const uint32_t fb = full0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
-          if (leader) mbar_arrive_expect_tx(&ctl.full[stage], 2 * P_STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&ctl.full[stage], bytes);
           tma_load_2d_pair(sa, &tmA, fb, kb * BK, row0);
-          tma_load_3d_pair(sa + P_A_BYTES, tmB, fb, kb * BK, brow0, e);
+          tma_load_3d_pair(sa + P_A_BYTES, mb, fb, kb * BK, brow0, e);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == P_STAGES) {
@@ -344,13 +385,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------ MMA issuer (CTA 0)
-      const uint32_t idesc = idesc_bf16_f32(PM, UMMA_N);
+      const uint32_t idesc_whole = idesc_bf16_f32(PM, UMMA_N);
+      const uint32_t idesc_half = idesc_bf16_f32(PM, UMMA_N / 2);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; tile < total && ok; tile += npairs) {
+      int tile, half;
+      for (int j = 0; ok && item(j, tile, half); ++j) {
+        const uint32_t idesc = half < 0 ? idesc_whole : idesc_half;
         if (!mbar_wait(&ctl.tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * UMMA_N);
@@ -391,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (warp - 2) * kStageFloats;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < total; tile += npairs) {
+    int tile, half;
+    for (int j = 0; item(j, tile, half); ++j) {
       int e, m_blk, n_blk;
       coords(tile, e, m_blk, n_blk);
       if (!mbar_wait(&ctl.tfull[acc], acc_phase, abort_flag, p.status)) break;
@@ -401,7 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t prow = static_cast<int64_t>(ctl.off[e]) + row_local;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * UMMA_N);
-      epilogue_rows<MODE>(p, t_row, valid, prow, n_blk * kTileN, stg);
+      const int w = half < 0 ? kTileN : kTileN / 2;
+      epilogue_rows<MODE>(p, t_row, valid, prow, n_blk * kTileN + (half < 0 ? 0 : half * w), w,
+                          stg);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -741,7 +788,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int exp
 
 template <int MODE>
 cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                             const Params& p, int64_t max_tiles, cudaStream_t stream) {
+                             const CUtensorMap& b0h, const CUtensorMap& b1h, const Params& p,
+                             int64_t max_tiles, cudaStream_t stream) {
   auto kern = tc_pair_gemm_kernel<MODE>;
   constexpr size_t kPairSmemBytes = pair_smem_bytes<MODE>();
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -773,7 +821,7 @@ cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const 
   }
   const int64_t n = std::min<int64_t>(pairs, max_tiles);
   cfg.gridDim = dim3(static_cast<unsigned>(2 * n), 1, 1);
-  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, p);
+  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, b0h, b1h, p);
 }
 
 }  // namespace
@@ -832,14 +880,18 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
   if (K % 8 != 0 || N % 128 != 0 || E > kMaxExperts || R >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
   if (R == 0) return cudaSuccess;
-  CUtensorMap ta, tb0, tb1;
+  CUtensorMap ta, tb0, tb1, tb0h, tb1h;
   {
+    // B maps: boxes of 128 rows (whole tiles) and 64 rows (half tiles)
     if (!make_map(&ta, a_sorted, K, R, 0, BM)) return cudaErrorInvalidValue;
     if (!make_map(&tb0, w0, K, N, E, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&tb0h, w0, K, N, E, 64)) return cudaErrorInvalidValue;
     if (gate) {
       if (!make_map(&tb1, w1, K, N, E, 128)) return cudaErrorInvalidValue;
+      if (!make_map(&tb1h, w1, K, N, E, 64)) return cudaErrorInvalidValue;
     } else {
       tb1 = tb0;
+      tb1h = tb0h;
     }
     Params p{};
     p.offsets = offsets;
@@ -856,13 +908,13 @@ cudaError_t launch_tc_grouped_gemm(int mode, const void* a_sorted, int64_t R, in
     const int64_t max_tiles = ((R + PM - 1) / PM + E) * static_cast<int64_t>(p.n_tiles_n);
     switch (mode) {
       case kEpiGateH:
-        return launch_pair_mode<kEpiGateH>(ta, tb0, tb1, p, max_tiles, stream);
+        return launch_pair_mode<kEpiGateH>(ta, tb0, tb1, tb0h, tb1h, p, max_tiles, stream);
       case kEpiGateSlots:
-        return launch_pair_mode<kEpiGateSlots>(ta, tb0, tb1, p, max_tiles, stream);
+        return launch_pair_mode<kEpiGateSlots>(ta, tb0, tb1, tb0h, tb1h, p, max_tiles, stream);
       case kEpiScaleToken:
-        return launch_pair_mode<kEpiScaleToken>(ta, tb0, tb1, p, max_tiles, stream);
+        return launch_pair_mode<kEpiScaleToken>(ta, tb0, tb1, tb0h, tb1h, p, max_tiles, stream);
       case kEpiScaleSlots:
-        return launch_pair_mode<kEpiScaleSlots>(ta, tb0, tb1, p, max_tiles, stream);
+        return launch_pair_mode<kEpiScaleSlots>(ta, tb0, tb1, tb0h, tb1h, p, max_tiles, stream);
       default:
         return cudaErrorInvalidValue;
     }
