@@ -232,6 +232,13 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int64_t T, int Dm, int E, 
       std::max<int64_t>(1, std::min<int64_t>({want, 16, (row_bytes / 16) / 32})));
   // Programmatic dependent launch: the CTAs may start (and be resident)
   // while the router finishes; they wait for it before reading its outputs.
+  // The projection after it is a programmatic dependent too and needs most
+  // of an SM's shared memory; an SM whose shared-memory carve-out was set
+  // small for this kernel would take none of its CTAs until this kernel's
+  // CTAs left, so these CTAs ask for the largest carve-out.
+  const cudaError_t ce = cudaFuncSetAttribute(
+      dispatch_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (ce != cudaSuccess) return ce;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;

@@ -227,9 +227,9 @@ cudaError_t launch_eb(const void* x, int64_t T, int Dm, const float* w_r, const 
                       int k, int renorm, int32_t* topk_idx, float* topk_w, int32_t* counts,
                       int32_t* chunk_hist, cudaStream_t stream) {
   constexpr int kPiece = 16 / static_cast<int>(sizeof(InT));
+  cudaError_t err = cudaSuccess;
   if (chunk_hist) {
-    const cudaError_t err =
-        cudaMemsetAsync(chunk_hist, 0, sizeof(int32_t) * num_chunks(T) * EB, stream);
+    err = cudaMemsetAsync(chunk_hist, 0, sizeof(int32_t) * num_chunks(T) * EB, stream);
     if (err != cudaSuccess) return err;
   }
   // Longest rounding chain of a logit: the features of one thread, the warp
@@ -240,6 +240,15 @@ cudaError_t launch_eb(const void* x, int64_t T, int Dm, const float* w_r, const 
   const double n = m + 5.0 + kWarps + 2.0;
   const double u = 1.0 / 16777216.0;
   const float gamma = static_cast<float>(1.01 * n * u / (1.0 - n * u));
+  // The kernel after this one (the projection, or the dispatch) starts as a
+  // programmatic dependent while these CTAs run, and it needs most of an SM's
+  // shared memory: an SM whose shared-memory carve-out was set small for
+  // this kernel could take none of its CTAs until this one left. So these
+  // CTAs ask for the largest carve-out.
+  err = cudaFuncSetAttribute(router_small_kernel<InT, EB>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess) return err;
   router_small_kernel<InT, EB><<<static_cast<unsigned>(T), kThreads, 0, stream>>>(
       static_cast<const InT*>(x), Dm, w_r, bias, k, renorm, topk_idx, topk_w, counts, chunk_hist,
       gamma);
