@@ -52,14 +52,17 @@ constexpr int kChunk = 128;        // time steps per scan chunk
 constexpr int kScanThreads = 128;  // channels per scan CTA
 constexpr float kLog2e = 1.4426950408889634f;
 
-// One thread per channel and a chunk of kConvSteps time steps (a CTA holds
-// 128 consecutive channels, so every load and store of a step is one row
-// segment); the K - 1 previous inputs stay in registers, so each input is
-// read once (plus K - 1 at the chunk's start), and the loads of kBatch steps
-// are issued together. X is written as two bf16 parts per value, hi = bf16(v)
-// in row t, columns [0, De) and lo = bf16(v - hi) in columns [De, 2 De): the
-// x projection multiplies both by W_x (a product accurate to ~2^-16 on the
-// bf16 tensor cores) and the scan reads hi + lo.
+// One thread per 4 adjacent channels and a chunk of kConvSteps time steps (a
+// CTA holds 512 consecutive channels, so every load and store of a step is
+// one row segment: 16-byte loads, 8-byte stores); the K - 1 previous inputs
+// stay in registers, so each input is read once (plus K - 1 at the chunk's
+// start), and the loads of kBatch steps are issued together. The tap count is
+// a template parameter, which keeps taps and windows in few registers: many
+// resident warps and wide loads keep enough bytes in flight (the kernel is
+// bound by HBM latency otherwise). X is written as two bf16 parts per value,
+// hi = bf16(v) in row t, columns [0, De) and lo = bf16(v - hi) in columns
+// [De, 2 De): the x projection multiplies both by W_x (a product accurate to
+// ~2^-16 on the bf16 tensor cores) and the scan reads hi + lo.
 constexpr int kConvSteps = 64;
 constexpr int kBatch = 8;  // time steps whose loads are issued together
 
@@ -68,57 +71,81 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16& hi, __nv_bflo
   lo = __float2bfloat16_rn(v - __bfloat162float(hi));
 }
 
+__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat16 a, __nv_bfloat16 b) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) |
+         (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
+}
+
+template <int K>
 __global__ void __launch_bounds__(128)
     conv_silu_kernel(const float* __restrict__ h, int64_t T, int De, int L,
-                     const float* __restrict__ w, const float* __restrict__ b, int K,
+                     const float* __restrict__ w, const float* __restrict__ b,
                      __nv_bfloat16* __restrict__ x2) {
-  const int d = blockIdx.x * 128 + threadIdx.x;
+  const int d0 = (blockIdx.x * 128 + threadIdx.x) * 4;  // channels d0 .. d0 + 3
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kConvSteps;
-  if (d >= De) return;
-  float tap[kMaxTaps], win[kMaxTaps];  // win[j] = h_{t-1-j} (0 before the sequence)
+  if (d0 >= De) return;
+  float tap[4][K], win[4][K];  // win[c][j] = h_{t-1-j} of channel d0 + c (0 before the sequence)
+  float bias[4];
 #pragma unroll
-  for (int j = 0; j < kMaxTaps; ++j) {
-    tap[j] = j < K ? __ldg(w + static_cast<int64_t>(d) * K + j) : 0.f;
-    win[j] = 0.f;
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      tap[c][j] = __ldg(w + static_cast<int64_t>(d0 + c) * K + j);
+      win[c][j] = 0.f;
+    }
+    bias[c] = __ldg(b + d0 + c);
   }
-  const float bias = __ldg(b + d);
-  const float tcur = tap[K - 1];
   int64_t seq0 = (t0 / L) * L;
 #pragma unroll
-  for (int j = 0; j < kMaxTaps - 1; ++j)
-    if (j < K - 1 && t0 - 1 - j >= seq0) win[j] = __ldg(h + (t0 - 1 - j) * De + d);
+  for (int j = 0; j < K - 1; ++j)
+    if (t0 - 1 - j >= seq0) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(h + (t0 - 1 - j) * De + d0));
+      win[0][j] = v.x;
+      win[1][j] = v.y;
+      win[2][j] = v.z;
+      win[3][j] = v.w;
+    }
   const int n = static_cast<int>(T - t0 < kConvSteps ? T - t0 : kConvSteps);
-  int64_t next_seq = seq0 + L;  // the window restarts where the next sequence begins
-  const float* hp = h + t0 * De + d;
-  __nv_bfloat16* xp = x2 + t0 * (2 * static_cast<int64_t>(De)) + d;
+  int64_t next_seq = seq0 + L;  // the windows restart where the next sequence begins
+  const float* hp = h + t0 * De + d0;
+  uint2* xp = reinterpret_cast<uint2*>(x2 + t0 * (2 * static_cast<int64_t>(De)) + d0);
+  const int64_t row2 = (2 * static_cast<int64_t>(De)) / 4;  // one X row in uint2 (4 bf16)
+  const int64_t lo_off = De / 4;
   for (int s0 = 0; s0 < n; s0 += kBatch) {
-    float cur[kBatch];
+    float4 cur[kBatch];
 #pragma unroll
     for (int q = 0; q < kBatch; ++q)
-      cur[q] = s0 + q < n ? __ldg(hp + static_cast<int64_t>(s0 + q) * De) : 0.f;
+      cur[q] = s0 + q < n ? __ldg(reinterpret_cast<const float4*>(hp + static_cast<int64_t>(s0 + q) * De))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {
       const int s = s0 + q;
       if (s >= n) break;
       if (t0 + s == next_seq) {
 #pragma unroll
-        for (int j = 0; j < kMaxTaps; ++j) win[j] = 0.f;
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < K; ++j) win[c][j] = 0.f;
         next_seq += L;
       }
-      // tap K-1 multiplies the current step, tap K-1-j the step j back
-      float acc = fmaf(tcur, cur[q], bias);
+      const float cv[4] = {cur[q].x, cur[q].y, cur[q].z, cur[q].w};
+      __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
-      for (int j = 1; j < kMaxTaps; ++j)
-        if (j < K) acc = fmaf(tap[K - 1 - j], win[j - 1], acc);
+      for (int c = 0; c < 4; ++c) {
+        // tap K-1 multiplies the current step, tap K-1-j the step j back
+        float acc = fmaf(tap[c][K - 1], cv[c], bias[c]);
 #pragma unroll
-      for (int j = kMaxTaps - 1; j > 0; --j) win[j] = win[j - 1];
-      win[0] = cur[q];
-      // SiLU with the fast exp and divide (relative error ~1e-6; for
-      // acc < -88 the quotient is SiLU's limit 0)
-      __nv_bfloat16 hi, lo;
-      split_bf16(__fdividef(acc, 1.0f + __expf(-acc)), hi, lo);
-      xp[static_cast<int64_t>(s) * 2 * De] = hi;
-      xp[static_cast<int64_t>(s) * 2 * De + De] = lo;
+        for (int j = 1; j < K; ++j) acc = fmaf(tap[c][K - 1 - j], win[c][j - 1], acc);
+#pragma unroll
+        for (int j = K - 1; j > 0; --j) win[c][j] = win[c][j - 1];
+        win[c][0] = cv[c];
+        // SiLU with the fast exp and divide (relative error ~1e-6; for
+        // acc < -88 the quotient is SiLU's limit 0)
+        split_bf16(__fdividef(acc, 1.0f + __expf(-acc)), hi[c], lo[c]);
+      }
+      uint2* dst = xp + static_cast<int64_t>(s) * row2;
+      dst[0] = make_uint2(bf16x2_bits(hi[0], hi[1]), bf16x2_bits(hi[2], hi[3]));
+      dst[lo_off] = make_uint2(bf16x2_bits(lo[0], lo[1]), bf16x2_bits(lo[2], lo[3]));
     }
   }
 }
@@ -205,11 +232,16 @@ struct ScanArgs {
 //   (except for a sequence's last chunk, which feeds nothing) the chunk's
 //   own recurrence from a zero state: its final state and sum of delta.
 // kOut = true: the recurrence again from the chunk's entering state, y out.
-// The loads of kBatch steps' delta and x are issued together.
-template <bool kOut>
+// NP: the state count rounded up to 4, 8 or 16 (the padded states have
+// A = 0, B = C = 0 and stay 0). The states are updated in pairs with packed
+// float32 arithmetic (one multiply for both exponents' arguments, one for
+// both inputs, one fused multiply-add for both states, one for y's two
+// partial sums), B and C are read from shared memory as float4 rows, and the
+// loads of kBatch steps' delta and x are issued together.
+template <bool kOut, int NP>
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
-  __shared__ float sB[kChunk][kMaxState];
-  __shared__ float sC[kOut ? kChunk : 1][kMaxState];
+  __shared__ __align__(16) float sB[kChunk][NP];
+  __shared__ __align__(16) float sC[kOut ? kChunk : 1][NP];
   const int cg = blockIdx.y;  // chunk over all sequences
   const int seq = cg / a.nc, c = cg - (cg / a.nc) * a.nc;
   const bool last = c == a.nc - 1;
@@ -223,18 +255,25 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
     for (int s = 0; s < len; ++s) dp[s * a.De] = softplus_f(dp[s * a.De] + bd);
     return;
   }
-  for (int i = threadIdx.x; i < len * N; i += kScanThreads) {
-    const int s = i / N, n = i - (i / N) * N;
+  for (int i = threadIdx.x; i < len * NP; i += kScanThreads) {
+    const int s = i / NP, n = i - (i / NP) * NP;
     const float* row = a.dbc + (t0 + s) * a.Np + a.R;
-    sB[s][n] = row[n];
-    if (kOut) sC[s][n] = row[N + n];
+    sB[s][n] = n < N ? row[n] : 0.f;
+    if (kOut) sC[s][n] = n < N ? row[N + n] : 0.f;
   }
   __syncthreads();
-  float A2[kMaxState], h[kMaxState];
+  float2 A2[NP / 2], h[NP / 2];
 #pragma unroll
-  for (int n = 0; n < kMaxState; ++n) {
-    A2[n] = n < N ? -expf(__ldg(a.a_log + static_cast<int64_t>(d) * N + n)) * kLog2e : 0.f;
-    h[n] = (kOut && n < N) ? a.carry[(static_cast<int64_t>(cg) * N + n) * a.De + d] : 0.f;
+  for (int q = 0; q < NP / 2; ++q) {
+    float av[2], hv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int n = 2 * q + u;
+      av[u] = n < N ? -expf(__ldg(a.a_log + static_cast<int64_t>(d) * N + n)) * kLog2e : 0.f;
+      hv[u] = (kOut && n < N) ? a.carry[(static_cast<int64_t>(cg) * N + n) * a.De + d] : 0.f;
+    }
+    A2[q] = make_float2(av[0], av[1]);
+    h[q] = make_float2(hv[0], hv[1]);
   }
   const float bd = kOut ? 0.f : __ldg(a.b_dt + d);
   const float Dd = kOut ? __ldg(a.d + d) : 0.f;
@@ -262,22 +301,38 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const ScanArgs a) {
       }
       const float dx = delta * xv[q];
       ssum += delta;
-      float yv = 0.f;
+      const float2 dd = make_float2(delta, delta), dx2 = make_float2(dx, dx);
+      float2 y2 = make_float2(0.f, 0.f);
+      const float4* b4 = reinterpret_cast<const float4*>(&sB[s][0]);
+      const float4* c4 = reinterpret_cast<const float4*>(&sC[kOut ? s : 0][0]);
 #pragma unroll
-      for (int n = 0; n < kMaxState; ++n) {
-        if (n < N) {
-          h[n] = fmaf(ex2_approx(delta * A2[n]), h[n], dx * sB[s][n]);
-          if (kOut) yv = fmaf(h[n], sC[s][n], yv);
+      for (int g = 0; g < NP / 4; ++g) {
+        const float4 bq = b4[g];
+        float4 cq;
+        if (kOut) cq = c4[g];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int q2 = 2 * g + u;
+          const float2 arg = __fmul2_rn(dd, A2[q2]);
+          const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+          const float2 bv = u == 0 ? make_float2(bq.x, bq.y) : make_float2(bq.z, bq.w);
+          h[q2] = __ffma2_rn(e, h[q2], __fmul2_rn(dx2, bv));
+          if (kOut) {
+            const float2 cv = u == 0 ? make_float2(cq.x, cq.y) : make_float2(cq.z, cq.w);
+            y2 = __ffma2_rn(h[q2], cv, y2);
+          }
         }
       }
-      if (kOut) yp[s * a.De] = fmaf(Dd, xv[q], yv);
+      if (kOut) yp[s * a.De] = fmaf(Dd, xv[q], y2.x + y2.y);
     }
   }
   if (!kOut) {
     a.S[static_cast<int64_t>(cg) * a.De + d] = ssum;
 #pragma unroll
-    for (int n = 0; n < kMaxState; ++n)
-      if (n < N) a.hend[(static_cast<int64_t>(cg) * N + n) * a.De + d] = h[n];
+    for (int q = 0; q < NP / 2; ++q) {
+      if (2 * q < N) a.hend[(static_cast<int64_t>(cg) * N + 2 * q) * a.De + d] = h[q].x;
+      if (2 * q + 1 < N) a.hend[(static_cast<int64_t>(cg) * N + 2 * q + 1) * a.De + d] = h[q].y;
+    }
   }
 }
 
@@ -411,9 +466,27 @@ cudaError_t launch_ssm_core(const float* h, int64_t T, int De, int seq_len, cons
       static_cast<const uint4*>(w_dt), ex * De, R / 8, reinterpret_cast<uint4*>(w.wdt2));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  conv_silu_kernel<<<dim3(static_cast<unsigned>(De / 128),
-                         static_cast<unsigned>((T + kConvSteps - 1) / kConvSteps)),
-                    128, 0, stream>>>(h, T, De, seq_len, conv_w, conv_b, K, w.x2);
+  {
+    const dim3 grid(static_cast<unsigned>((De + 511) / 512),
+                    static_cast<unsigned>((T + kConvSteps - 1) / kConvSteps));
+    switch (K) {
+#define ROM_CONV_CASE(KV)                                                                    \
+  case KV:                                                                                   \
+    conv_silu_kernel<KV><<<grid, 128, 0, stream>>>(h, T, De, seq_len, conv_w, conv_b, w.x2); \
+    break;
+      ROM_CONV_CASE(1)
+      ROM_CONV_CASE(2)
+      ROM_CONV_CASE(3)
+      ROM_CONV_CASE(4)
+      ROM_CONV_CASE(5)
+      ROM_CONV_CASE(6)
+      ROM_CONV_CASE(7)
+      ROM_CONV_CASE(8)
+#undef ROM_CONV_CASE
+      default:
+        return cudaErrorInvalidValue;
+    }
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // x projection to [dt | B | C | 0] float32 rows, token order
@@ -447,14 +520,20 @@ cudaError_t launch_ssm_core(const float* h, int64_t T, int De, int seq_len, cons
   const int nseq = static_cast<int>(T / seq_len);
   const dim3 grid(static_cast<unsigned>(De / kScanThreads),
                   static_cast<unsigned>(static_cast<int64_t>(nseq) * a.nc));
-  scan_kernel<false><<<grid, kScanThreads, 0, stream>>>(a);
+  // states padded to 4, 8 or 16
+  const int np = N <= 4 ? 4 : N <= 8 ? 8 : 16;
+  if (np == 4) scan_kernel<false, 4><<<grid, kScanThreads, 0, stream>>>(a);
+  else if (np == 8) scan_kernel<false, 8><<<grid, kScanThreads, 0, stream>>>(a);
+  else scan_kernel<false, 16><<<grid, kScanThreads, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   scan_carry_kernel<<<grid_for(static_cast<int64_t>(nseq) * N * De, 256), 256, 0, stream>>>(
       a, nseq);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  scan_kernel<true><<<grid, kScanThreads, 0, stream>>>(a);
+  if (np == 4) scan_kernel<true, 4><<<grid, kScanThreads, 0, stream>>>(a);
+  else if (np == 8) scan_kernel<true, 8><<<grid, kScanThreads, 0, stream>>>(a);
+  else scan_kernel<true, 16><<<grid, kScanThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
