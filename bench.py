@@ -684,6 +684,26 @@ def core_roofline(res, wl):
             "frac": ach / peak, "kernel": "rom_ssm_core (whole phase)"}
 
 
+def phase_figures(wl, part_ms, hbm_gbs, world):
+    """Figures of single phases: the route + dispatch phase's HBM rate (the
+    router reads X once, the dispatch reads and writes the R = T*k routed
+    rows: algorithmic bytes / the phase's device time, against the measured
+    HBM copy rate), and for a training step the forward's token rate (its
+    phases' device times summed)."""
+    out = {}
+    elt = 2 if wl.dtype == "bf16" else 4
+    if "route_dispatch" in part_ms and part_ms["route_dispatch"] > 0:
+        routings = 3 if wl.kind == "variant" and wl.variant == "independent" else 1
+        nbytes = routings * (wl.T * wl.Dm * elt + 2 * wl.T * wl.k * wl.Dm * elt)
+        gbs = nbytes / (part_ms["route_dispatch"] / 1e3) / 1e9
+        out["route_dispatch_hbm"] = {"bytes": nbytes, "achieved_gbs": gbs,
+                                     "frac": gbs / hbm_gbs}
+    if wl.backward:
+        fwd_ms = sum(v for n, v in part_ms.items() if n != "backward")
+        out["forward_tokens_per_s"] = job_tokens_per_s(wl.T, world, fwd_ms)
+    return out
+
+
 def summary_entry(res, peaks, src, world):
     """Per-workload figures of the extra workloads of one bench run."""
     wl = res["wl"]
@@ -695,6 +715,7 @@ def summary_entry(res, peaks, src, world):
             "ms_per_step": res["step_ms"], "tokens_per_s": job_tokens_per_s(wl.T, world,
                                                                             res["step_ms"]),
             "block_tflops": tot / step_s / 1e12, "roofline": roofline(res, peaks, src),
+            **phase_figures(wl, res["part_ms"], peaks["hbm_gbs"], world),
             "kernels_ms": res["part_ms"], "kernels_ms_eager": res["part_ms_eager"],
             "clocks": res["clocks"], "gpu_launches": res["launches"],
             "expert_load": (res["counts"] / max(1, res["counts"].sum())).round(4).tolist()}
@@ -806,6 +827,7 @@ def main():
                 "config": config, "l2": res["l2"], "roofline": roofline(res, peaks, src),
                 "block_tflops": tot_flops / step_s / 1e12,
                 "block_frac_of_bf16_peak": tot_flops / step_s / 1e12 / peaks["bf16_tflops"],
+                **phase_figures(wl, res["part_ms"], peaks["hbm_gbs"], world),
                 "kernels_ms": res["part_ms"], "kernels_ms_eager": res["part_ms_eager"],
                 "eager_ms_per_step": res["eager_ms"],
                 "step": "forward + backward" if wl.backward else "forward",

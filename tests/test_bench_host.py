@@ -78,3 +78,21 @@ def test_workload_config_of_every_workload():
         assert cfg["parallelism"] == "replicas x1"
         tiled = wl.kind == "inproj" and wl.dtype == "bf16" and wl.T <= 64
         assert ("weights" in cfg) == tiled, name
+
+
+def test_phase_figures():
+    """The route + dispatch phase's algorithmic bytes (X read by the router,
+    the T*k routed rows read and written by the dispatch) over its time, and
+    a training step's forward token rate."""
+    wl = WORKLOADS["prefill_16k"]
+    f = bench.phase_figures(wl, {"route_dispatch": 0.05, "proj0": 0.3, "proj1": 0.2}, 6500.0, 1)
+    nbytes = 16384 * 2048 * 2 * 3
+    assert f["route_dispatch_hbm"]["bytes"] == nbytes
+    assert abs(f["route_dispatch_hbm"]["achieved_gbs"] - nbytes / 5e-5 / 1e9) < 1e-6
+    assert "forward_tokens_per_s" not in f
+    wl = WORKLOADS["top2_fwd_bwd"]
+    f = bench.phase_figures(wl, {"route_dispatch": 0.3, "proj0": 2.5, "proj1": 2.2,
+                                 "backward": 11.0}, 6500.0, 1)
+    assert f["route_dispatch_hbm"]["bytes"] == 32768 * 2560 * 2 * (1 + 2 * 2)
+    assert abs(f["forward_tokens_per_s"] - 32768 / 5.0e-3) < 1e-3
+    assert bench.phase_figures(WORKLOADS["decode_swimba_inproj"], {"route": 0.01}, 6500.0, 1) == {}
