@@ -719,11 +719,16 @@ class HostPipeline:
     """Forward of the block (or the Swimba in-projection) on HOST tensors.
 
     Tokens are independent, so the batch is cut into chunks (multiples of the
-    128-token routing chunk) that cycle over `nstreams` CUDA streams: the
-    host-to-device copy of one chunk, the kernels of another and the
-    device-to-host copy of a third run at the same time. Each token's result
-    is the one a single call on the whole batch gives. Device buffers are
-    allocated once per stream (torch); the kernels are the library's.
+    128-token routing chunk) that go through three stages, each on streams of
+    its own: the host-to-device copies on one stream, the kernels on two
+    (a chunk of a few thousand tokens leaves the GPU room for a second one),
+    the device-to-host copies on one, chained by events. The input copy of one
+    chunk, the kernels of the previous ones and the output copy of an earlier
+    one run at the same time, and the two copy directions overlap on the
+    link. `nstreams` device buffer sets rotate over the chunks; a set takes a
+    new chunk once its last chunk's output copy has completed. Each token's
+    result is the one a single call on the whole batch gives. Device buffers
+    are allocated once (torch); the kernels are the library's.
 
     With ``graph=True`` the second call with the same host buffers, weights
     and size captures the whole multi-stream sequence (copies and kernels)
@@ -741,7 +746,10 @@ class HostPipeline:
         # Chunks of at least 2048 tokens (smaller ones cost more in launches
         # and stream switches than the overlap saves), at most the batch.
         self.chunk = min(max(2048, -(-per // 128) * 128), max(128, -(-T // 128) * 128))
-        self.streams = [torch.cuda.Stream(device=device) for _ in range(nstreams)]
+        self.nbuf = nstreams
+        self.s_in = torch.cuda.Stream(device=device)
+        self.s_out = torch.cuda.Stream(device=device)
+        self.s_comp = [torch.cuda.Stream(device=device) for _ in range(2)]
         self.x = [torch.empty((self.chunk, Dm), dtype=dtype, device=device) for _ in range(nstreams)]
         if De is not None:  # RoM block
             self.bufs = [BlockBuffers(self.chunk, Dm, De, E, k, dtype, device) for _ in range(nstreams)]
@@ -756,27 +764,44 @@ class HostPipeline:
         return [(i, min(T, i + self.chunk)) for i in range(0, T, self.chunk)]
 
     def _run(self, T, body):
-        """body(j, a, b, stream) for every chunk [a, b); one chunk runs on
-        the current stream, several cycle over the pipeline's streams."""
+        """body = (copy_in, compute, copy_out), each called (j, a, b, stream)
+        for every chunk [a, b) with buffer set j: one chunk runs on the
+        current stream, several go through the staged streams."""
+        copy_in, compute, copy_out = body
         cur = torch.cuda.current_stream()
         chunks = self._chunks(T)
         if len(chunks) == 1:
-            body(0, 0, T, cur)
+            for f in body:
+                f(0, 0, T, cur)
             return
         start = torch.cuda.Event()
         start.record(cur)
-        used = []
+        streams = [self.s_in, self.s_out] + self.s_comp
+        for s in streams:
+            s.wait_event(start)
+        free = [None] * self.nbuf  # buffer set j: its last output copy
         for n, (a, b) in enumerate(chunks):
-            j = n % len(self.streams)
-            s = self.streams[j]
-            if j not in used:
-                s.wait_event(start)
-                used.append(j)
-            with torch.cuda.stream(s):
-                body(j, a, b, s)
-        for j in used:
+            j = n % self.nbuf
+            with torch.cuda.stream(self.s_in):
+                if free[j] is not None:
+                    self.s_in.wait_event(free[j])
+                copy_in(j, a, b, self.s_in)
+                e_in = torch.cuda.Event()
+                e_in.record(self.s_in)
+            sc = self.s_comp[n % len(self.s_comp)]
+            with torch.cuda.stream(sc):
+                sc.wait_event(e_in)
+                compute(j, a, b, sc)
+                e_c = torch.cuda.Event()
+                e_c.record(sc)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(e_c)
+                copy_out(j, a, b, self.s_out)
+                free[j] = torch.cuda.Event()
+                free[j].record(self.s_out)
+        for s in streams:
             ev = torch.cuda.Event()
-            ev.record(self.streams[j])
+            ev.record(s)
             cur.wait_event(ev)
 
     def _launch(self, key, T, body):
@@ -812,13 +837,20 @@ class HostPipeline:
                 self._tail_bufs(b - a, lambda n: BlockBuffers(n, self.Dm, De, self.E, self.k,
                                                               self.x[0].dtype, self.x[0].device))
 
-        def body(j, a, b, s):
-            xd = self.x[j][: b - a]
-            xd.copy_(x_host[a:b], non_blocking=True)
-            bufs = self.bufs[j] if b - a == self.chunk else self._tail[b - a]
-            blk = block_forward(xd, w_r, bias, w_conv, w_gate, w_out, self.k, renorm, bufs,
-                                stream=s)
-            out_host[a:b].copy_(blk.out, non_blocking=True)
+        def bufs_of(j, a, b):
+            return self.bufs[j] if b - a == self.chunk else self._tail[b - a]
+
+        def copy_in(j, a, b, s):
+            self.x[j][: b - a].copy_(x_host[a:b], non_blocking=True)
+
+        def compute(j, a, b, s):
+            block_forward(self.x[j][: b - a], w_r, bias, w_conv, w_gate, w_out, self.k, renorm,
+                          bufs_of(j, a, b), stream=s)
+
+        def copy_out(j, a, b, s):
+            out_host[a:b].copy_(bufs_of(j, a, b).out, non_blocking=True)
+
+        body = (copy_in, compute, copy_out)
 
         key = ("block", T, x_host.data_ptr(), out_host.data_ptr(), w_r.data_ptr(),
                0 if bias is None else bias.data_ptr(), w_conv.data_ptr(), w_gate.data_ptr(),
@@ -834,15 +866,19 @@ class HostPipeline:
                 self._tail_bufs(b - a, lambda n: RoutingBuffers(n, self.Dm, self.E, self.k,
                                                                 self.x[0].dtype, self.x[0].device))
 
-        def body(j, a, b, s):
-            xd = self.x[j][: b - a]
-            xd.copy_(x_host[a:b], non_blocking=True)
+        def copy_in(j, a, b, s):
+            self.x[j][: b - a].copy_(x_host[a:b], non_blocking=True)
+
+        def compute(j, a, b, s):
             bufs = self.bufs[j] if b - a == self.chunk else self._tail[b - a]
-            od = self.out[j][: b - a]
             sl = None if self.slots[j] is None else self.slots[j][: (b - a) * self.k]
-            inproj_forward(xd, w_r, w, self.k, renorm, bias, bufs, od, sl, stream=s,
-                           w_tiled=w_tiled)
-            out_host[a:b].copy_(od, non_blocking=True)
+            inproj_forward(self.x[j][: b - a], w_r, w, self.k, renorm, bias, bufs,
+                           self.out[j][: b - a], sl, stream=s, w_tiled=w_tiled)
+
+        def copy_out(j, a, b, s):
+            out_host[a:b].copy_(self.out[j][: b - a], non_blocking=True)
+
+        body = (copy_in, compute, copy_out)
 
         key = ("inproj", T, x_host.data_ptr(), out_host.data_ptr(), w_r.data_ptr(), w.data_ptr(),
                0 if bias is None else bias.data_ptr(), bool(renorm),
