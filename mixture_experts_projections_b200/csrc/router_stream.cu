@@ -22,7 +22,8 @@
 // (Cauchy-Schwarz). |w_e| is formed from the streamed weight blocks during a
 // CTA's first tile. A token whose selected logits' lower bounds do not all
 // clear the upper bound of every expert ranked after them is re-decided on
-// float64 logits (warp-cooperative). Equal logits go to the lower expert index.
+// float64 logits, which all 8 compute warps form together (each over an
+// eighth of the features). Equal logits go to the lower expert index.
 // Every wait is bounded; after the set-up the roles meet only on mbarriers.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -47,6 +48,7 @@ constexpr int kFeat = BK / kCompute;    // features per warp per block
 constexpr int TPL = BM / 32;            // tokens per lane
 constexpr int kDecide = BM / kCompute;  // tokens decided per warp
 constexpr int kMaxStages = 8;
+constexpr int kUB = 4;                  // uncertain tokens per float64 batch
 
 template <int EB>
 struct Geo {
@@ -67,7 +69,14 @@ struct SCtl {
   int done;
   int hist[EB];
   float wsq[kCompute][EB];
-  double l64[kCompute][EB];
+  // float64 re-decision of uncertain tokens: their tile rows, and the 8
+  // warps' partial logits of a batch of kUB of them
+  int nunc;
+  int unc_row[BM];
+  uint64_t unc_ready;
+  uint64_t p64_ready;
+  uint64_t p64_free;
+  double p64[kUB][kCompute][EB];
 };
 
 __device__ __forceinline__ uint32_t sw128_off(int n, int k) {
@@ -108,8 +117,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl.part_ready, kCompute);
     mbar_init(&ctl.part_free, kCompute);
+    mbar_init(&ctl.unc_ready, kCompute);
+    mbar_init(&ctl.p64_ready, kCompute);
+    mbar_init(&ctl.p64_free, kCompute);
     ctl.abort = 0;
     ctl.done = 0;
+    ctl.nunc = 0;
     for (int e = 0; e < EB; ++e) ctl.hist[e] = 0;
     fence_barrier_init();
   }
@@ -157,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float nq = 0.f;          // this lane's share of |w_{lane % EB}|^2 over the warp's features
   int stage = 0;
   uint32_t phase = 0;
+  uint32_t p64_phase = 0, p64_free_phase = 0;
   int it = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     float acc[TPL][EB];
@@ -356,78 +370,114 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < EB; ++e)
           if (e < E && !((above >> e) & 1ull) && !(lb > l[e] + err[e])) certain = false;
       }
-    unsigned todo = __ballot_sync(0xffffffffu, valid && !certain);
-    while (todo) {
-      const int src = __ffs(todo) - 1;
-      todo &= todo - 1;
-      const int64_t tr = __shfl_sync(0xffffffffu, tok, src);
-      // float64 logits of token tr: lane i takes the 16-byte pieces i, i + 32,
-      // ... of the row (8 features each), four loads in flight; the weights
-      // come from global memory (L2), E floats per feature.
-      const uint4* xr = reinterpret_cast<const uint4*>(x + tr * Dm);
-      const int npc = Dm / 8;
-      double a[EB];
+    // Tokens whose float32 decision is not certain get float64 logits from
+    // all 8 compute warps together, kUB tokens at a time: warp h sums its
+    // feature slice h*Dm/8 .. (h+1)*Dm/8 - 1 (lane l: the 8-feature pieces
+    // l, l + 32, ... of the slice), the slices meet in shared memory and the
+    // deciding lane adds them in the order h = 0 .. 7 and decides again.
+    const bool unsure = valid && !certain;
+    const unsigned mine = __ballot_sync(0xffffffffu, unsure);
+    int my_idx = 0;
+    {
+      int base = 0;
+      if (lane == 0 && mine) base = atomicAdd(&ctl.nunc, __popc(mine));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      my_idx = base + __popc(mine & ((1u << lane) - 1u));
+      if (unsure) ctl.unc_row[my_idx] = r;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl.unc_ready);
+    if (!__all_sync(0xffffffffu, mbar_wait(&ctl.unc_ready, static_cast<uint32_t>(it) & 1u,
+                                           abort_flag, status)))
+      break;
+    const int nunc = *reinterpret_cast<volatile int*>(&ctl.nunc);
+    bool batch_ok = true;
+    for (int b0 = 0; b0 < nunc && batch_ok; b0 += kUB) {
+      const int nb = min(kUB, nunc - b0);
+      for (int u = 0; u < nb; ++u) {
+        const int64_t tr = tile * BM + ctl.unc_row[b0 + u];
+        const uint4* xr = reinterpret_cast<const uint4*>(x + tr * Dm + h * (Dm / kCompute));
+        double a[EB];
 #pragma unroll
-      for (int e = 0; e < EB; ++e) a[e] = 0.0;
-      for (int pc0 = lane; pc0 < npc; pc0 += 4 * 32) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int pc = pc0 + 32 * u;
-          v[u] = (pc < npc) ? __ldg(xr + pc) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int pc = pc0 + 32 * u;
-          if (pc >= npc) break;
-          const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        for (int e = 0; e < EB; ++e) a[e] = 0.0;
+        for (int pc = lane; pc < Dm / (kCompute * 8); pc += 32) {
+          const uint4 v = __ldg(xr + pc);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          const float* wrow = w_r + (static_cast<int64_t>(h) * (Dm / kCompute) + 8 * pc) * EB;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint32_t bits = (j & 1) ? (w4[j >> 1] & 0xFFFF0000u) : (w4[j >> 1] << 16);
             const double xd = static_cast<double>(__uint_as_float(bits));
-            const float4* wr = reinterpret_cast<const float4*>(w_r + static_cast<int64_t>(pc * 8 + j) * EB);
+            const float4* wq = reinterpret_cast<const float4*>(wrow + j * EB);
 #pragma unroll
             for (int e4 = 0; e4 < EB / 4; ++e4) {
-              const float4 wq = __ldg(wr + e4);
-              a[4 * e4] = fma(xd, static_cast<double>(wq.x), a[4 * e4]);
-              a[4 * e4 + 1] = fma(xd, static_cast<double>(wq.y), a[4 * e4 + 1]);
-              a[4 * e4 + 2] = fma(xd, static_cast<double>(wq.z), a[4 * e4 + 2]);
-              a[4 * e4 + 3] = fma(xd, static_cast<double>(wq.w), a[4 * e4 + 3]);
+              const float4 w = __ldg(wq + e4);
+              a[4 * e4] = fma(xd, static_cast<double>(w.x), a[4 * e4]);
+              a[4 * e4 + 1] = fma(xd, static_cast<double>(w.y), a[4 * e4 + 1]);
+              a[4 * e4 + 2] = fma(xd, static_cast<double>(w.z), a[4 * e4 + 2]);
+              a[4 * e4 + 3] = fma(xd, static_cast<double>(w.w), a[4 * e4 + 3]);
             }
           }
         }
-      }
-#pragma unroll
-      for (int e = 0; e < EB; ++e) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a[e] += __shfl_xor_sync(0xffffffffu, a[e], o);
-      }
-      if (lane == src)
 #pragma unroll
         for (int e = 0; e < EB; ++e)
-          if (e < E) ctl.l64[h][e] = a[e] + (bias ? static_cast<double>(bias[e]) : 0.0);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a[e] += __shfl_xor_sync(0xffffffffu, a[e], o);
+        if (lane == 0)
+#pragma unroll
+          for (int e = 0; e < EB; ++e) ctl.p64[u][h][e] = a[e];
+      }
       __syncwarp();
-      if (lane == src) {
+      if (lane == 0) mbar_arrive(&ctl.p64_ready);
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&ctl.p64_ready, p64_phase, abort_flag, status))) {
+        batch_ok = false;
+        break;
+      }
+      p64_phase ^= 1u;
+      if (unsure && my_idx >= b0 && my_idx < b0 + nb) {
+        const int u = my_idx - b0;
+        double l64[EB];
+#pragma unroll
+        for (int e = 0; e < EB; ++e) {
+          double v = ctl.p64[u][0][e];
+#pragma unroll
+          for (int hh = 1; hh < kCompute; ++hh) v += ctl.p64[u][hh][e];
+          l64[e] = v + (bias && e < E ? static_cast<double>(bias[e]) : 0.0);
+        }
         uint64_t u2 = 0;
+#pragma unroll
         for (int j = 0; j <= kMaxTopK; ++j) {
           sel[j] = -1;
           if (j <= k) {
             int bi = -1;
             double bv = 0.0;
-            for (int e = 0; e < E; ++e)
-              if (!((u2 >> e) & 1ull) && (bi < 0 || ctl.l64[h][e] > bv)) {
+#pragma unroll
+            for (int e = 0; e < EB; ++e)
+              if (e < E && !((u2 >> e) & 1ull) && (bi < 0 || l64[e] > bv)) {
                 bi = e;
-                bv = ctl.l64[h][e];
+                bv = l64[e];
               }
             sel[j] = bi;
             if (bi >= 0) u2 |= 1ull << bi;
           }
         }
 #pragma unroll
-        for (int e = 0; e < EB; ++e) l[e] = (e < E) ? static_cast<float>(ctl.l64[h][e]) : -INFINITY;
+        for (int e = 0; e < EB; ++e) l[e] = (e < E) ? static_cast<float>(l64[e]) : -INFINITY;
       }
-      __syncwarp();
+      if (b0 + kUB < nunc) {
+        // the partials are read before the next batch overwrites them
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.p64_free);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&ctl.p64_free, p64_free_phase, abort_flag, status))) {
+          batch_ok = false;
+          break;
+        }
+        p64_free_phase ^= 1u;
+      }
     }
+    if (!batch_ok) break;
     if (valid) {
       const float m = pick(l, sel[0]);
       float den = 0.f;
@@ -462,7 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (chunk_hist) chunk_hist[tile * E + e] = v;
         if (counts && v) atomicAdd(counts + e, v);
       }
-      if (lane == 0) ctl.done = 0;
+      if (lane == 0) {
+        ctl.done = 0;
+        ctl.nunc = 0;  // every warp read it after unc_ready, before its decisions
+      }
       __threadfence_block();
     }
     __syncwarp();

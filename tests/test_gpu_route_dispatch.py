@@ -72,10 +72,14 @@ def test_route_with_bias_and_empty_expert():
     assert b.counts.cpu().numpy()[3] == 0
 
 
-@pytest.mark.parametrize("k,renorm", [(1, False), (2, False), (2, True)])
-def test_route_zero_router_tie_rule(k, renorm):
+@pytest.mark.parametrize("k,renorm,T,E", [(1, False, 300, 6), (2, False, 300, 6),
+                                           (2, True, 300, 6),
+                                           # the streaming router: every token of every
+                                           # tile is re-decided in float64, in batches
+                                           (1, False, 2100, 8), (2, True, 2100, 16)])
+def test_route_zero_router_tie_rule(k, renorm, T, E):
     """W_r = 0: all logits tie exactly; the lower expert index wins."""
-    T, Dm, E = 300, 128, 6
+    Dm = 128
     inp = make_block_inputs(T, Dm, 1, E, seed=9, zero_router=True)
     b = run_route(to_dev(inp["x"], "bf16"), to_dev(inp["w_r"], "f32"), None, E, k, renorm)
     assert np.array_equal(b.topk_idx.cpu().numpy(), np.tile(np.arange(k), (T, 1)))
