@@ -13,11 +13,13 @@
 // tokens, 4 per lane (tokens lane + 32 j). Per block a lane reads its tokens'
 // 8 features (one 16-byte piece each, conflict-free under the swizzle) and
 // the 8 x E weights as broadcast float4 reads, each of which feeds 4 tokens.
-// Per block and expert it forms a partial over the 8 features (sequential
-// float32 FMA, two experts per packed FMA) and adds it to its running sum.
-// At the end of the tile the 8 warps' sums and |x|^2 meet in shared memory and
-// warp h decides tokens 16h .. 16h+15, adding the parts in order h = 0 .. 7.
-// Each logit therefore goes through at most 8 + d_model/64 + 7 + 1 roundings;
+// Per pair of blocks (per block when E = 16) and expert it forms a partial
+// over its 16 (8) features (sequential float32 FMA, two experts per packed
+// FMA) and adds it to its running sum. At the end of the tile the 8 warps'
+// sums and |x|^2 meet in shared memory and warp h decides tokens
+// 16h .. 16h+15, adding the parts in order h = 0 .. 7. Each logit therefore
+// goes through at most 16 + d_model/128 + 7 + 1 roundings (E = 16:
+// 8 + d_model/64 + 7 + 1);
 // with |x| and |w_e| this bounds its error by gamma_n |x| |w_e|
 // (Cauchy-Schwarz). |w_e| is formed from the streamed weight blocks during a
 // CTA's first tile. A token whose selected logits' lower bounds do not all
@@ -55,6 +57,9 @@ struct Geo {
   static constexpr int kWBytes = BK * EB * 4;
   static constexpr int kStage = X_BYTES + kWBytes;  // a multiple of 1024
   static constexpr int kEG = EB < 8 ? EB : 8;        // experts per register group
+  // blocks per partial sum: two (16 features) when one register group holds
+  // every expert, else one (the partials of both groups would not fit)
+  static constexpr int kPB = EB / kEG == 1 ? 2 : 1;
   static constexpr int kPCols = EB + 4;              // part row: sums, |x|^2, pad
   static constexpr int kNormPerLane = kFeat * EB / 32;
 };
@@ -166,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------- compute warps
   const int h = warp - 1;  // feature slice of every block; decided tokens 16h ..
+  constexpr int PB = G::kPB;
   float wn[EB];            // |w_e|, formed in the first tile
   float nq = 0.f;          // this lane's share of |w_{lane % EB}|^2 over the warp's features
   int stage = 0;
@@ -174,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int it = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     float acc[TPL][EB];
+    float2 p[EB / EG][TPL][EG / 2];  // the current partial sums (PB blocks each)
     float sq[TPL];
 #pragma unroll
     for (int t = 0; t < TPL; ++t) {
@@ -213,13 +220,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < TPL; ++t)
 #pragma unroll
         for (int i = 0; i < kFeat; ++i) sq[t] = fmaf(xv[t][i], xv[t][i], sq[t]);
+      const bool p_first = kb % PB == 0;
+      const bool p_last = kb % PB == PB - 1 || kb == KB - 1;
 #pragma unroll
       for (int g = 0; g < EB / EG; ++g) {
-        float2 p[TPL][EG / 2];
+        if (p_first) {
 #pragma unroll
-        for (int t = 0; t < TPL; ++t)
+          for (int t = 0; t < TPL; ++t)
 #pragma unroll
-          for (int e2 = 0; e2 < EG / 2; ++e2) p[t][e2] = make_float2(0.f, 0.f);
+            for (int e2 = 0; e2 < EG / 2; ++e2) p[g][t][e2] = make_float2(0.f, 0.f);
+        }
 #pragma unroll
         for (int i = 0; i < kFeat; ++i) {
           const float4* wv = reinterpret_cast<const float4*>(sw + i * EB + g * EG);
@@ -230,20 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int t = 0; t < TPL; ++t) {
               const float2 xx = make_float2(xv[t][i], xv[t][i]);
-              p[t][2 * q4] = __ffma2_rn(xx, wa, p[t][2 * q4]);
-              p[t][2 * q4 + 1] = __ffma2_rn(xx, wb, p[t][2 * q4 + 1]);
+              p[g][t][2 * q4] = __ffma2_rn(xx, wa, p[g][t][2 * q4]);
+              p[g][t][2 * q4 + 1] = __ffma2_rn(xx, wb, p[g][t][2 * q4 + 1]);
             }
           }
         }
+        if (p_last) {
 #pragma unroll
-        for (int t = 0; t < TPL; ++t)
+          for (int t = 0; t < TPL; ++t)
 #pragma unroll
-          for (int e2 = 0; e2 < EG / 2; ++e2) {
-            const int e = g * EG + 2 * e2;
-            const float2 a2 = __fadd2_rn(make_float2(acc[t][e], acc[t][e + 1]), p[t][e2]);
-            acc[t][e] = a2.x;
-            acc[t][e + 1] = a2.y;
-          }
+            for (int e2 = 0; e2 < EG / 2; ++e2) {
+              const int e = g * EG + 2 * e2;
+              const float2 a2 = __fadd2_rn(make_float2(acc[t][e], acc[t][e + 1]), p[g][t][e2]);
+              acc[t][e] = a2.x;
+              acc[t][e + 1] = a2.y;
+            }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.empty[stage]);  // done with the stage
@@ -561,9 +573,12 @@ cudaError_t launch_eb(const void* x, int64_t T, int Dm, const float* w_r, const 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // Longest rounding chain of a logit: 8 block FMAs, one add per block, 7
-  // adds of the warps' parts, the bias (+1 spare); 1 % slack covers the norms.
-  const double n = static_cast<double>(kFeat) + static_cast<double>(Dm / BK) +
+  // Longest rounding chain of a logit: the FMAs of one partial sum (8
+  // features per block, G::kPB blocks), one add per partial, 7 adds of the
+  // warps' parts, the bias (+1 spare); 1 % slack covers the norms.
+  const int kb_total = Dm / BK;
+  const double n = static_cast<double>(kFeat * std::min(G::kPB, kb_total)) +
+                   static_cast<double>((kb_total + G::kPB - 1) / G::kPB) +
                    static_cast<double>(kCompute - 1) + 2.0;
   const double u = 1.0 / 16777216.0;
   const float gamma = static_cast<float>(1.01 * n * u / (1.0 - n * u));

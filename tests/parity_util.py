@@ -107,8 +107,9 @@ def routing_weight_rtol(x, w_r, bias=None) -> np.ndarray:
     bias add); a token decided on float64 logits carries at most u |l_e| from
     the final cast. Every router's chain is shorter than
     n = d_model / 32 + 32 (per-token router: features per thread + 5 + 8 + 2;
-    streaming router: 64 / Q + d_model / 64 + Q + 1; register-tiled router:
-    the lane's slice + 7), and gamma_n gets the 1 % slack the kernels use.
+    streaming router: 16 + d_model / 128 + 9, or 8 + d_model / 64 + 9 for
+    16 experts; register-tiled router: the lane's slice + 7), and gamma_n
+    gets the 1 % slack the kernels use.
     ln r = l_j - logsumexp(l), so logit errors move ln r by at most twice the
     largest one. The softmax itself adds at most (E + 8) u (expf within 2 ulp
     per term, the sum of E positive terms, the division) plus u |l - max l|
