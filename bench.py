@@ -197,6 +197,84 @@ class ClockSampler:
 
 
 THROTTLE_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+# NVML clock-event reason bits (nvml.h) of the reasons above
+NVML_REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+                    "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+
+class NvmlSampler:
+    """SM clock and clock-event reasons read through NVML every `period_s`
+    seconds around the timed steps: a short workload's timed region spans
+    only a sample or two of nvidia-smi's 100 ms loop, which then mostly sees
+    the idle moments around it."""
+
+    def __init__(self, gpu_index, period_s=0.002):
+        self.gpu = gpu_index
+        self.period = period_s
+        self.samples = []  # (sm MHz, reason bits)
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.nvml = None
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        except Exception:  # noqa: BLE001
+            return
+        self.nvml = pynvml
+        reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+        def run():
+            while not self.stop_evt.is_set():
+                try:
+                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                         int(reasons(h))))
+                except Exception:  # noqa: BLE001
+                    pass
+                self.stop_evt.wait(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_evt.set()
+        self.thread.join(timeout=2)
+        try:
+            self.nvml.nvmlShutdown()
+        except Exception:  # noqa: BLE001
+            pass
+        return summarize_nvml(self.samples, self.period)
+
+
+def summarize_nvml(samples, period_s):
+    """Median and lowest SM clock and the throttle reasons (of
+    THROTTLE_REASONS) active in any of the (MHz, NVML reason bits) samples."""
+    if not samples:
+        return {"samples": 0}
+    mhz = [float(m) for m, _ in samples]
+    bits = 0
+    for _, b in samples:
+        bits |= b
+    return {"samples": len(samples), "period_ms": period_s * 1e3,
+            "sm_mhz": float(np.median(mhz)), "sm_mhz_min": min(mhz),
+            "reasons": sorted(n for n, b in NVML_REASON_BITS.items() if bits & b)}
+
+
+def merge_clocks(smi, fast):
+    """The reported clocks: nvidia-smi's summary, with the median SM clock
+    and the reasons of the NVML samples taken during the timed steps when
+    there are enough of them (their summary is kept under "nvml")."""
+    out = dict(smi)
+    if fast and fast.get("samples", 0) >= 3:
+        out["sm_mhz"] = fast["sm_mhz"]
+        out["reasons"] = sorted(set(smi.get("reasons") or []) | set(fast["reasons"]))
+        out["nvml"] = fast
+    return out
 
 
 def summarize_clocks(lines):
@@ -576,12 +654,15 @@ def measure(args, wl, world, local_rank, with_e2e):
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
+    fast = NvmlSampler(local_rank)
+    fast.start()
     step_ms = timed_loop(lambda j: g_step.replay(), args.steps, 1)[:, 0]
+    fast_clk = fast.stop()
     ph_ms = timed_loop(lambda j: graphs[j].replay(), args.steps, len(phases))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clk = clocks.stop()
+    clk = merge_clocks(clocks.stop(), fast_clk)
     eager_ms = timed_loop(lambda j: phases[j](), args.steps, len(phases))
     # The dominant kernel alone: one eager launch between two events, the
     # host ahead of the GPU (no graph-launch latency in its duration).

@@ -59,6 +59,25 @@ def test_clock_summary_skips_lines_that_do_not_parse():
     assert empty["sm_mhz"] is None and empty["sm_max_mhz"] is None and empty["samples"] == 0
 
 
+def test_nvml_clock_summary_and_merge():
+    """The NVML samples of the timed steps: median and lowest clock and the
+    throttle reasons among their bits; with at least 3 of them their median
+    and reasons replace nvidia-smi's, which may have seen only idle moments."""
+    fast = bench.summarize_nvml([(1965, 0), (1800, 0x4), (1700, 0x4 | 0x1), (1965, 0)], 0.002)
+    assert fast["samples"] == 4 and fast["sm_mhz"] == 1882.5 and fast["sm_mhz_min"] == 1700
+    assert fast["reasons"] == ["sw_power_cap"]  # the idle bit (0x1) is not a throttle reason
+    assert bench.summarize_nvml([(1965, 0x8 | 0x40)], 0.002)["reasons"] == [
+        "hw_slowdown", "hw_thermal_slowdown"]
+    assert bench.summarize_nvml([], 0.002) == {"samples": 0}
+    smi = bench.summarize_clocks([_line(1965, 1965), _line(1965, 1965)])
+    m = bench.merge_clocks(smi, fast)
+    assert m["sm_mhz"] == 1882.5 and m["sm_max_mhz"] == 1965.0
+    assert m["reasons"] == ["sw_power_cap"] and m["nvml"] is fast and m["samples"] == 2
+    few = bench.summarize_nvml([(1500, 0), (1500, 0)], 0.002)
+    assert bench.merge_clocks(smi, few) == smi
+    assert bench.merge_clocks(smi, None) == smi
+
+
 def test_core_roofline_counts_one_exp_per_state_update():
     wl = WORKLOADS["prefill_16k_core"]
     res = {"part_ms": {"core": 1.0}, "clocks": {"sm_max_mhz": 1965.0}}
