@@ -202,28 +202,41 @@ NVML_REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
                     "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
 
+_NVML = {}
+
+
+def nvml_device(gpu_index):
+    """(pynvml, handle) of a GPU, NVML initialised once per process (its
+    first call is slow), or None without NVML."""
+    if gpu_index not in _NVML:
+        try:
+            import pynvml
+            if not _NVML:
+                pynvml.nvmlInit()
+            _NVML[gpu_index] = (pynvml, pynvml.nvmlDeviceGetHandleByIndex(gpu_index))
+        except Exception:  # noqa: BLE001
+            _NVML[gpu_index] = None
+    return _NVML[gpu_index]
+
+
 class NvmlSampler:
     """SM clock and clock-event reasons read through NVML every `period_s`
     seconds around the timed steps: a short workload's timed region spans
     only a sample or two of nvidia-smi's 100 ms loop, which then mostly sees
     the idle moments around it."""
 
-    def __init__(self, gpu_index, period_s=0.002):
+    def __init__(self, gpu_index, period_s=0.0005):
         self.gpu = gpu_index
         self.period = period_s
         self.samples = []  # (sm MHz, reason bits)
         self.stop_evt = threading.Event()
         self.thread = None
-        self.nvml = None
 
     def start(self):
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
-        except Exception:  # noqa: BLE001
+        dev = nvml_device(self.gpu)
+        if dev is None:
             return
-        self.nvml = pynvml
+        pynvml, h = dev
         reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
 
@@ -244,10 +257,6 @@ class NvmlSampler:
             return None
         self.stop_evt.set()
         self.thread.join(timeout=2)
-        try:
-            self.nvml.nvmlShutdown()
-        except Exception:  # noqa: BLE001
-            pass
         return summarize_nvml(self.samples, self.period)
 
 
@@ -653,6 +662,7 @@ def measure(args, wl, world, local_rank, with_e2e):
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
+    nvml_device(local_rank)  # NVML's slow first call before the timed region
     time.sleep(0.3)
     fast = NvmlSampler(local_rank)
     fast.start()

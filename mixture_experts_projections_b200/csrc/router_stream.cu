@@ -196,17 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint8_t* st = smem + stage * G::kStage;
       const float* sw = reinterpret_cast<const float*>(st + X_BYTES) + kFeat * h * EB;
-      float xv[TPL][kFeat];
+      // the lane's tokens' 8 features of the block, as bf16 pairs (unpacked
+      // where the FMAs use them, which keeps fewer registers live)
+      uint4 xc[TPL];
 #pragma unroll
-      for (int t = 0; t < TPL; ++t) {
-        const uint4 v = *reinterpret_cast<const uint4*>(st + sw128_off(lane + 32 * t, kFeat * h));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          xv[t][2 * i] = __uint_as_float(w[i] << 16);
-          xv[t][2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-      }
+      for (int t = 0; t < TPL; ++t)
+        xc[t] = *reinterpret_cast<const uint4*>(st + sw128_off(lane + 32 * t, kFeat * h));
       if (it == 0) {
         // the warp's 8 x EB weights of the block, lane l taking l, l + 32, ...
         // (all of expert l % EB)
@@ -216,10 +211,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           nq = fmaf(w, w, nq);
         }
       }
-#pragma unroll
-      for (int t = 0; t < TPL; ++t)
-#pragma unroll
-        for (int i = 0; i < kFeat; ++i) sq[t] = fmaf(xv[t][i], xv[t][i], sq[t]);
       const bool p_first = kb % PB == 0;
       const bool p_last = kb % PB == PB - 1 || kb == KB - 1;
 #pragma unroll
@@ -232,6 +223,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int i = 0; i < kFeat; ++i) {
+          // feature i of the lane's tokens, unpacked from the bf16 pieces
+          // where it is used (and |x|^2 formed on the first group's pass)
+          float xi[TPL];
+#pragma unroll
+          for (int t = 0; t < TPL; ++t) {
+            const uint32_t wd = (i >> 1) == 0   ? xc[t].x
+                                : (i >> 1) == 1 ? xc[t].y
+                                : (i >> 1) == 2 ? xc[t].z
+                                                : xc[t].w;
+            xi[t] = __uint_as_float((i & 1) ? (wd & 0xFFFF0000u) : (wd << 16));
+            if (g == 0) sq[t] = fmaf(xi[t], xi[t], sq[t]);
+          }
           const float4* wv = reinterpret_cast<const float4*>(sw + i * EB + g * EG);
 #pragma unroll
           for (int q4 = 0; q4 < EG / 4; ++q4) {
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
 #pragma unroll
             for (int t = 0; t < TPL; ++t) {
-              const float2 xx = make_float2(xv[t][i], xv[t][i]);
+              const float2 xx = make_float2(xi[t], xi[t]);
               p[g][t][2 * q4] = __ffma2_rn(xx, wa, p[g][t][2 * q4]);
               p[g][t][2 * q4 + 1] = __ffma2_rn(xx, wb, p[g][t][2 * q4 + 1]);
             }
