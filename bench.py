@@ -221,9 +221,9 @@ def nvml_device(gpu_index):
 
 class NvmlSampler:
     """SM clock and clock-event reasons read through NVML every `period_s`
-    seconds around the timed steps: a short workload's timed region spans
-    only a sample or two of nvidia-smi's 100 ms loop, which then mostly sees
-    the idle moments around it."""
+    seconds around the timed steps and phases: a short workload's timed
+    region spans only a sample or two of nvidia-smi's 100 ms loop, which then
+    mostly sees the idle moments around it."""
 
     def __init__(self, gpu_index, period_s=0.0005):
         self.gpu = gpu_index
@@ -667,8 +667,8 @@ def measure(args, wl, world, local_rank, with_e2e):
     fast = NvmlSampler(local_rank)
     fast.start()
     step_ms = timed_loop(lambda j: g_step.replay(), args.steps, 1)[:, 0]
-    fast_clk = fast.stop()
     ph_ms = timed_loop(lambda j: graphs[j].replay(), args.steps, len(phases))
+    fast_clk = fast.stop()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
