@@ -29,6 +29,7 @@
 #include <algorithm>
 
 #include "rom_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace rom {
 namespace {
@@ -193,7 +194,9 @@ __global__ void __launch_bounds__(kDispatchThreads)
   }
   __syncthreads();
   // Gather this CTA's column slice [v0, v1) of every slot row: one warp per
-  // row, 16-byte vectors, 4 in flight per lane.
+  // row, 16-byte vectors, 4 in flight per lane. The rows are read for the
+  // last time here (the router kept them in L2): their lines go first.
+  const uint64_t pol = l2_policy_evict_first();
   const int v0 = static_cast<int>(static_cast<int64_t>(row_vec16) * slice / nslices);
   const int v1 = static_cast<int>(static_cast<int64_t>(row_vec16) * (slice + 1) / nslices);
   for (int ls = warp; ls < ns; ls += kDispatchWarps) {
@@ -202,14 +205,14 @@ __global__ void __launch_bounds__(kDispatchThreads)
     uint4* drow = x_sorted + static_cast<int64_t>(s_pos[ls]) * row_vec16;
     int i = v0 + lane;
     for (; i + 96 < v1; i += 128) {
-      const uint4 a = __ldg(srow + i), b = __ldg(srow + i + 32), cc = __ldg(srow + i + 64),
-                  d = __ldg(srow + i + 96);
+      const uint4 a = ld_nc_hint(srow + i, pol), b = ld_nc_hint(srow + i + 32, pol),
+                  cc = ld_nc_hint(srow + i + 64, pol), d = ld_nc_hint(srow + i + 96, pol);
       drow[i] = a;
       drow[i + 32] = b;
       drow[i + 64] = cc;
       drow[i + 96] = d;
     }
-    for (; i < v1; i += 32) drow[i] = __ldg(srow + i);
+    for (; i < v1; i += 32) drow[i] = ld_nc_hint(srow + i, pol);
   }
 }
 

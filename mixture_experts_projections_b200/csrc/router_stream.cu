@@ -138,6 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
+      // X is read again right after this kernel by the dispatch's row copy:
+      // its lines are kept in L2 ahead of other data
+      const uint64_t pol_x = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;
@@ -150,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = smem + stage * G::kStage;
           mbar_arrive_expect_tx(&ctl.full[stage], G::kStage);
-          tma_load_2d(st, &tmX, &ctl.full[stage], kb * BK, static_cast<int>(tile * BM));
+          tma_load_2d_hint(st, &tmX, &ctl.full[stage], kb * BK, static_cast<int>(tile * BM),
+                           pol_x);
           bulk_load(st + X_BYTES, w_r + static_cast<int64_t>(kb) * BK * EB, G::kWBytes,
                     &ctl.full[stage]);
           issued |= 1u << stage;
