@@ -684,7 +684,7 @@ def measure(args, wl, world, local_rank, with_e2e):
     # ---------------------------------------------- e2e through host buffers
     # The public host-buffer call: inputs in pinned host memory, result copied
     # back, copies inside the timed region. Forward-only workloads go through
-    # rom.HostPipeline (chunks over 3 streams: copies overlap the kernels);
+    # rom.HostPipeline (chunks staged over copy-in, kernel and copy-out streams);
     # the others copy x in and O out around one step.
     e2e_total = 0.0
     if with_e2e:

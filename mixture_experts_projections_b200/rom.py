@@ -727,8 +727,14 @@ class HostPipeline:
     one run at the same time, and the two copy directions overlap on the
     link. `nstreams` device buffer sets rotate over the chunks; a set takes a
     new chunk once its last chunk's output copy has completed. Each token's
-    result is the one a single call on the whole batch gives. Device buffers
-    are allocated once (torch); the kernels are the library's.
+    routing is the one a single call on the whole batch gives, and so is its
+    output when the chunk and the batch take the same projection kernels
+    (more than 1024 routed rows each); a short last chunk may take the
+    swap-AB Out GEMM, whose output agrees within the forward's tolerance.
+    Chunks of 2048 tokens and four buffer sets measured best for the prefill
+    batch (smaller chunks cost more GEMM efficiency than the shorter first
+    and last copies save). Device buffers are allocated once (torch); the
+    kernels are the library's.
 
     With ``graph=True`` the second call with the same host buffers, weights
     and size captures the whole multi-stream sequence (copies and kernels)
@@ -737,15 +743,16 @@ class HostPipeline:
     eagerly (it also initialises the library's per-device state).
     """
 
-    def __init__(self, T, Dm, N_out, E, k, dtype, device="cuda", chunks=8, nstreams=3,
-                 De=None, graph=True):
+    def __init__(self, T, Dm, N_out, E, k, dtype, device="cuda", chunks=8, nstreams=4,
+                 De=None, graph=True, min_chunk=2048):
         self.T, self.Dm, self.E, self.k = T, Dm, E, k
         self.graph = graph
         self._graphs, self._seen, self._tail = {}, set(), {}
         per = -(-T // chunks)
-        # Chunks of at least 2048 tokens (smaller ones cost more in launches
-        # and stream switches than the overlap saves), at most the batch.
-        self.chunk = min(max(2048, -(-per // 128) * 128), max(128, -(-T // 128) * 128))
+        # Chunks of at least min_chunk tokens (smaller ones cost more in
+        # launches and stream switches than the overlap saves), at most the
+        # batch.
+        self.chunk = min(max(min_chunk, -(-per // 128) * 128), max(128, -(-T // 128) * 128))
         self.nbuf = nstreams
         self.s_in = torch.cuda.Stream(device=device)
         self.s_out = torch.cuda.Stream(device=device)
