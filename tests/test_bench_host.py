@@ -115,3 +115,17 @@ def test_phase_figures():
     assert f["route_dispatch_hbm"]["bytes"] == 32768 * 2560 * 2 * (1 + 2 * 2)
     assert abs(f["forward_tokens_per_s"] - 32768 / 5.0e-3) < 1e-3
     assert bench.phase_figures(WORKLOADS["decode_swimba_inproj"], {"route": 0.01}, 6500.0, 1) == {}
+
+
+def test_tensor_roofline_gives_the_sustained_peak_only_under_the_power_cap():
+    """The dominant GEMM's fraction is of the burst peak; when the clocks of
+    its run show sw_power_cap, the fraction of the sustained peak is added."""
+    wl = WORKLOADS["top2_fwd_bwd"]
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    res = {"wl": wl, "dominant_ms": 2.0, "dominant_kind": "flop", "dominant_work": 2.8e12,
+           "clocks": {"reasons": ["sw_power_cap"]}}
+    r = bench.roofline(res, peaks, "measured")
+    assert abs(r["achieved"] - 1400.0) < 1e-9 and abs(r["frac"] - 0.875) < 1e-12
+    assert abs(r["sustained"]["frac"] - 1.0) < 1e-12 and r["sustained"]["peak"] == 1400.0
+    res["clocks"] = {"reasons": []}
+    assert "sustained" not in bench.roofline(res, peaks, "measured")
