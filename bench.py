@@ -213,7 +213,12 @@ def nvml_device(gpu_index):
             import pynvml
             if not _NVML:
                 pynvml.nvmlInit()
-            _NVML[gpu_index] = (pynvml, pynvml.nvmlDeviceGetHandleByIndex(gpu_index))
+            h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            # the first queries of a device are slow: made here, before any timed region
+            pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+             or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)(h)
+            _NVML[gpu_index] = (pynvml, h)
         except Exception:  # noqa: BLE001
             _NVML[gpu_index] = None
     return _NVML[gpu_index]
