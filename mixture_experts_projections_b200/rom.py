@@ -749,9 +749,9 @@ class HostPipeline:
         self.graph = graph
         self._graphs, self._seen, self._tail = {}, set(), {}
         per = -(-T // chunks)
-        # Chunks of at least min_chunk tokens (smaller ones cost more in
-        # launches and stream switches than the overlap saves), at most the
-        # batch.
+        # Chunks of at least min_chunk tokens (smaller ones lose more GEMM
+        # efficiency and launch time than their shorter first and last copies
+        # save), at most the batch.
         self.chunk = min(max(min_chunk, -(-per // 128) * 128), max(128, -(-T // 128) * 128))
         self.nbuf = nstreams
         self.s_in = torch.cuda.Stream(device=device)
