@@ -5,8 +5,9 @@
 // One CTA owns a 128-token tile (= one histogram chunk of the dispatch) at a
 // time. A producer warp streams the tile through a ring of stages, one
 // 64-feature block per stage: the X block by TMA (128 x 64 bf16, 128-byte
-// swizzle) and the matching 64 rows of W_r ([d_model][E] float32, contiguous)
-// by a bulk copy. W_r is not kept resident: each CTA re-reads it (from L2)
+// swizzle; its lines kept in L2 ahead of other data, since the dispatch reads
+// the rows again right after) and the matching 64 rows of W_r ([d_model][E]
+// float32, contiguous) by a bulk copy. W_r is not kept resident: each CTA re-reads it (from L2)
 // once per tile, which leaves the shared memory to a deep ring.
 //
 // 8 compute warps: warp h owns features 8h .. 8h+7 of every block and all 128
