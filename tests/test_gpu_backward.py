@@ -52,6 +52,7 @@ BWD_CASES = [
     (1000, 512, 256, 16, 2, 0.05, None),
     (333, 256, 512, 6, 3, 0.1, None),
     (257, 256, 256, 8, 2, 0.05, {2: -40.0}),  # one expert without rows
+    (300, 256, 256, 64, 8, 0.1, None),        # the largest E and k: 64 experts of ~37 rows
 ]
 
 
